@@ -38,7 +38,7 @@ def lib():
         L.zo_route.argtypes = [_D, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                _D, _I32, ctypes.c_int, ctypes.c_double,
-                               _U8, _U8, _D, _I64, _I64]
+                               _U8, _U8, _D, _I64, _I64, _D]
         L.zo_attended_set.argtypes = [_U8, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _I64]
         L.zo_attended_set.restype = ctypes.c_int64
         L.zo_attend.argtypes = [_D, _D, ctypes.c_int, _D, _I64, ctypes.c_int64, _D]
@@ -109,6 +109,7 @@ class Route:
     info: np.ndarray            # [L][n_lanes][4] decision margins (see zo_topp)
     kstar: np.ndarray           # [L][n_lanes]
     nfront: np.ndarray          # [L][n_lanes]
+    scores: Optional[List[np.ndarray]] = None   # index l-1: [n_lanes][n_l] frontier estimates
 
 
 def level_sizes(N: int, C: int, L: int) -> List[int]:
@@ -116,7 +117,8 @@ def level_sizes(N: int, C: int, L: int) -> List[int]:
 
 
 def route(K: np.ndarray, qref: np.ndarray, C: int, L: int, N: int, q: np.ndarray,
-          lane_g: np.ndarray, p: float, forced: Optional[List[np.ndarray]] = None) -> Route:
+          lane_g: np.ndarray, p: float, forced: Optional[List[np.ndarray]] = None,
+          return_scores: bool = False) -> Route:
     """Top-down top-p routing of lanes through one sequence's tree.
 
     K [Hkv][ld][d]; qref [Hkv][R][d]; q [n_lanes][d]; lane_g [n_lanes].  ``forced`` (replay
@@ -138,11 +140,14 @@ def route(K: np.ndarray, qref: np.ndarray, C: int, L: int, N: int, q: np.ndarray
     info = np.empty((L, n_lanes, 4))
     kstar = np.empty((L, n_lanes), dtype=np.int64)
     nfront = np.empty((L, n_lanes), dtype=np.int64)
+    sc = np.full((L, n_lanes, n1), np.nan) if return_scores else None
     lib().zo_route(_p(K, _D), ld, N, Hkv, d, _p(qref, _D), R, C, L, _p(q, _D), _p(lane_g, _I32),
                    n_lanes, float(p), _p(kept, _U8),
                    _p(fbuf, _U8) if fbuf is not None else ctypes.cast(None, _U8),
-                   _p(info, _D), _p(kstar, _I64), _p(nfront, _I64))
-    return Route([kept[v, :, :sizes[v]].astype(bool) for v in range(L)], info, kstar, nfront)
+                   _p(info, _D), _p(kstar, _I64), _p(nfront, _I64),
+                   _p(sc, _D) if sc is not None else ctypes.cast(None, _D))
+    return Route([kept[v, :, :sizes[v]].astype(bool) for v in range(L)], info, kstar, nfront,
+                  [sc[v, :, :sizes[v]] for v in range(L)] if sc is not None else None)
 
 
 def attended_set(kept1: np.ndarray, N: int, C: int, L: int) -> np.ndarray:

@@ -222,12 +222,15 @@ int64_t zo_topp(const double* e, const int64_t* idx, int64_t n, double p, uint8_
  * forced (nullable, same layout as kept): replay mode - the level-(l-1) frontier is built
  * from forced[v] instead of kept[v], so each level is judged on the frontier another
  * implementation actually used.
+ * scores (nullable): [L][n_lanes][n1] plane estimates of every frontier node (others
+ * untouched), so a caller can see how close two nodes at the cut were.
  * Node summaries are recomputed from the raw keys for every frontier node at every level.
  */
 void zo_route(const double* K, int64_t ld, int64_t N, int Hkv, int d,
               const double* qref, int R, int C, int L,
               const double* q, const int32_t* lane_g, int n_lanes, double p,
-              uint8_t* kept, const uint8_t* forced, double* info, int64_t* kstar, int64_t* nfront)
+              uint8_t* kept, const uint8_t* forced, double* info, int64_t* kstar, int64_t* nfront,
+              double* scores)
 {
     const int64_t n1 = N / C;
     const size_t lane_stride = (size_t)(n1 > 0 ? n1 : 1);
@@ -293,6 +296,8 @@ void zo_route(const double* K, int64_t ld, int64_t N, int Hkv, int d,
             const size_t o = (size_t)v * n_lanes + x;
             kstar[o] = zo_topp(ec, ic, n, p, kc, info + o * 4);
             nfront[o] = n;
+            if (scores)
+                for (int64_t t = 0; t < n; ++t) scores[o * lane_stride + ic[t]] = ec[t];
             uint8_t* kx = kept + o * lane_stride;
             for (int64_t t = 0; t < n; ++t) if (kc[t]) kx[ic[t]] = 1;
             free(ec); free(ic); free(kc);
