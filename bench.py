@@ -1,0 +1,335 @@
+"""Benchmark: ZHA tree build + append + tree-routed sparse decode on B200.
+
+One step = the whole hot path over one batch of the 1M-token deep-tree workload:
+  zha_build_tree over N = 1,048,576 tokens (chunk summaries + level merges),
+  zha_append of 4,096 tokens, then
+  zha_decode of the 128 needle queries (16 query heads / 2 KV heads each) at p = 0.95
+  (routing level by level + exact attention over sink, kept chunks and tail).
+value = decoded queries per second of device time (max over ranks, summed over ranks).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs an independent replica (no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_tree_indexed_build_b200 import inputs  # noqa: E402
+
+METRIC = "ZHA decode queries/s at 256K & 1M ctx; achieved HBM GB/s vs peak"
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max SM clock
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--p", type=float, default=0.95)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return pk["hbm_gbs"], "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, dev: int):
+        self.proc = None
+        self.path = None
+        try:
+            bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        except Exception:
+            bus = None
+        self.sel = ["--id=%s" % bus] if bus else []
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, "--query-gpu=" + q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
+    """(bytes, flops) one launch of `name` must move/compute (per-unit figure x units),
+    from the decoder's work counters of one step."""
+    R, d = geom.R, geom.d
+    if name == "k_score":
+        nodes = sum(st.union_nodes)
+        lane_nodes = sum(st.lane_nodes)
+        return ((nodes * st.node_bytes + lane_nodes * 4) / launches, lane_nodes * R * d * 2 / launches)
+    if name == "k_attn":
+        return st.union_tokens * 4 * d / launches, st.lane_tokens * 4 * d / launches
+    if name == "k_select":
+        return sum(st.lane_nodes) * 4 / launches, 0.0
+    if name in ("k_build_stream", "k_merge"):
+        nodes = sum((N + n_append) // geom.C ** l for l in range(1, geom.L + 1))
+        rec = (R * d + 2 * R) * 4
+        reads = geom.Hkv * (N + n_append) * 2 * d if name == "k_build_stream" else 0
+        return (reads + geom.Hkv * nodes * rec) / launches, 0.0
+    return 0.0, 0.0
+
+
+def run_ours(args, rank, world, dev):
+    from hierarchical_tree_indexed_build_b200 import zha
+    torch.cuda.set_device(dev)
+    wl = inputs.deep_1m()
+    seq = wl.seqs[0]
+    g = seq.geom
+    N0, n_app = seq.n_tokens, wl.n_append
+    Q_host = wl.Q[0].contiguous()                    # [1][128][16][128] bf16
+    n_q = Q_host.shape[1]
+    K = seq.K.to(dev)
+    V = seq.V.to(dev)
+    qref = seq.qref.to(dev)
+    Q = Q_host.to(dev)
+    out = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    tree = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, seq.capacity)
+    dec = zha.Decoder([tree], n_q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        tree.build(K, N0, qref)
+        tree.append(K, N0, n_app)
+        dec.decode([K], [V], Q, args.p, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    zha.zha_profile_reset()
+    clocks = Clocks(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    zha.zha_profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    zha.zha_profile_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    prof = zha.zha_profile_read()
+    st = dec.stats()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * n_q / (ms_step / 1e3)
+
+    # dominant kernel and its roofline
+    n_lanes = n_q * g.Hq
+    top = max(prof.items(), key=lambda kv: kv[1][1])
+    name, (launches, tot_ms) = top
+    per_step_launches = launches / args.steps
+    nbytes, nflops = kernel_algorithmic(name, st, g, N0, n_app, n_lanes, per_step_launches)
+    avg_ms = tot_ms / launches
+    hbm_peak, peak_src = measured_peaks()
+    intensity = nflops / nbytes if nbytes else 0.0
+    if nflops and intensity > FP32_PEAK_TFLOPS * 1e12 / (hbm_peak * 1e9):
+        ach = nflops / (avg_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": ach, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": ach / FP32_PEAK_TFLOPS, "traffic": None, "kernel": name,
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+    else:
+        ach = nbytes / (avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                "traffic": None, "kernel": name, "peak_source": peak_src}
+    roof["algorithmic_bytes_per_launch"] = nbytes
+    roof["algorithmic_flops_per_launch"] = nflops
+    roof["avg_launch_ms"] = avg_ms
+    roof["launches"] = launches
+
+    # decode-only throughput and union bytes of the decode
+    dec_ms = sum(v[1] for k, v in prof.items() if k in ("k_union", "k_score", "k_select", "k_attn", "k_combine")) / args.steps
+    union_bytes = sum(st.union_nodes) * st.node_bytes + st.union_tokens * 4 * g.d
+    stages = {k: round(v[1] / args.steps, 4) for k, v in sorted(prof.items())}
+    res = {
+        "ms_per_step": ms_step, "value": value, "prof": prof, "roofline": roof, "clocks": clk,
+        "gpu_launches": int(sum(v[0] for v in prof.values())),
+        "decode_ms": dec_ms, "union_bytes": union_bytes,
+        "stats": {"union_nodes": list(st.union_nodes)[:g.L], "lane_nodes": list(st.lane_nodes)[:g.L],
+                  "union_tokens": st.union_tokens, "lane_tokens": st.lane_tokens},
+        "stages_ms": stages,
+    }
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        Kh = seq.K.pin_memory()
+        Vh = seq.V.pin_memory()
+        qh = seq.qref.pin_memory()
+        Qh = Q_host.pin_memory()
+        outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+
+        def step_e2e():
+            K.copy_(Kh, non_blocking=True)
+            V.copy_(Vh, non_blocking=True)
+            qref.copy_(qh, non_blocking=True)
+            Q.copy_(Qh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            step_e2e()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step_e2e()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = sum(x.numel() * x.element_size() for x in (Kh, Vh, qh, Qh))
+        res["e2e"] = {"value": world * n_q / (ems / args.steps / 1e3), "unit": "queries/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outh.numel() * 4}
+    res["wl"] = wl
+    return res
+
+
+def cpu_baseline(wl, p):
+    """The float64 oracle as it stands on a bounded sample: one query token (16 heads)
+    of the same workload, routed and attended."""
+    from oracle import oracle as O
+    seq = wl.seqs[0]
+    g = seq.geom
+    N = seq.n_tokens + wl.n_append
+    K = seq.K.to(torch.float64).numpy()
+    V = seq.V.to(torch.float64).numpy()
+    qref = seq.qref.to(torch.float64).numpy()
+    q = wl.Q[0, 0, 0].to(torch.float64).numpy()          # [Hq][d]
+    lane_g = np.array([h * g.Hkv // g.Hq for h in range(g.Hq)], dtype=np.int32)
+    O.lib()
+    t0 = time.perf_counter()
+    O.decode(K, V, qref, g.C, g.L, N, q, lane_g, p)
+    dt = time.perf_counter() - t0
+    return {"value": 1.0 / dt, "unit": "queries/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": "1 query token x 16 heads of the 1M-token deep workload (N=%d after append): "
+                      "float64 routing with definition-level summaries + exact attention; %.1f s" % (N, dt)}
+
+
+def base_line(args, world, wl):
+    seq = wl.seqs[0]
+    g = seq.geom
+    return {
+        "metric": METRIC, "unit": "queries/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "n_tokens_build": seq.n_tokens, "n_append": wl.n_append,
+                   "n_queries": int(wl.Q.shape[2]), "p": args.p, "C": g.C, "L": g.L, "R": g.R, "d": g.d,
+                   "Hq": g.Hq, "Hkv": g.Hkv, "step": "build + append + decode of all queries",
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (K+V 1.08 GB, tree 5.8 GB), no flush"},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        wl = inputs.deep_1m()
+        for _ in range(args.warmup):
+            pass   # the oracle has no warm-up state; each step below is a full sample
+        vals = [cpu_baseline(wl, args.p) for _ in range(args.steps)]
+        v = statistics.median(x["value"] for x in vals)
+        line = base_line(args, 1, wl)
+        line.update({"impl": "reference", "value": v, "ms_per_step": 1e3 / v,
+                     "cpu_baseline": dict(vals[0], value=v),
+                     "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        print(json.dumps(line))
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                             timeout=__import__("datetime").timedelta(seconds=120))
+    res = run_ours(args, rank, world, local)
+    wl = res.pop("wl")
+    if rank == 0:
+        line = base_line(args, world, wl)
+        line.update({"value": res["value"], "ms_per_step": res["ms_per_step"], "roofline": res["roofline"],
+                     "gpu_launches": res["gpu_launches"], "clocks": res["clocks"]})
+        if "e2e" in res:
+            line["e2e"] = res["e2e"]
+        hbm_peak, src = measured_peaks()
+        line["decode"] = {"ms_per_step": res["decode_ms"],
+                          "queries_per_s": int(wl.Q.shape[2]) / (res["decode_ms"] / 1e3),
+                          "union_gb": res["union_bytes"] / 1e9,
+                          "union_gbs": res["union_bytes"] / (res["decode_ms"] / 1e3) / 1e9,
+                          "union_frac_of_%s_hbm" % src: res["union_bytes"] / (res["decode_ms"] / 1e3) / 1e9 / hbm_peak,
+                          "keys_touched_frac": res["stats"]["lane_tokens"] / (
+                              int(wl.Q.shape[2]) * wl.seqs[0].geom.Hq * (wl.seqs[0].n_tokens + wl.n_append))}
+        line["stages_ms"] = res["stages_ms"]
+        line["stats"] = res["stats"]
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.p)
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,542 @@
+// zha_api.cu - the C ABI declared in include/zha.h: object lifetime, argument checks and
+// the launch sequences of tree build, append, routing and sparse attention.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "zha_common.cuh"
+#include "zha_launch.h"
+
+using namespace zha;
+
+namespace {
+
+thread_local std::string g_err;
+
+zha_status fail(zha_status s, const std::string& msg) {
+    g_err = msg;
+    return s;
+}
+
+#define ZHA_CUDA(expr)                                                                     \
+    do {                                                                                   \
+        cudaError_t e_ = (expr);                                                           \
+        if (e_ != cudaSuccess) return fail(ZHA_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+    } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ipow(int64_t c, int l) {
+    int64_t r = 1;
+    for (int i = 0; i < l; ++i) r *= c;
+    return r;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+float score_scale(int d) { return (float)(1.0 / sqrt((double)d)); }
+
+}  // namespace
+
+struct zha_tree {
+    zha_geometry g;
+    int32_t ns;
+    int64_t n_tokens;
+    bool built;
+    int64_t cap[kMaxL + 1];
+    float* rec[kMaxL + 1];
+    float* lse[kMaxL + 1];
+    __nv_bfloat16* qref;
+    void* block;
+    size_t bytes;
+    int device;
+};
+
+struct zha_decoder {
+    std::vector<const zha_tree*> trees;
+    int32_t n_seq, max_q, Hq, Hkv, d, G, Lmax;
+    int64_t lanes_cap, groups_cap;
+    Work w;
+    SeqDev* seq_dev;
+    std::vector<SeqDev> seq_host;
+    void* block;
+    size_t bytes;
+    int32_t last_n_q;
+    bool routed;
+};
+
+extern "C" const char* zha_last_error(void) { return g_err.c_str(); }
+
+// ------------------------------------------------------------------------------ tree
+
+static zha_status check_geometry(const zha_geometry* g) {
+    if (!g) return fail(ZHA_ERR_ARG, "geometry is NULL");
+    if (g->C < 2 || g->C > 1024) return fail(ZHA_ERR_ARG, "C must be in [2, 1024]");
+    if (g->L < 1 || g->L > kMaxL) return fail(ZHA_ERR_ARG, "L must be in [1, 16]");
+    if (!(g->R == 1 || g->R == 2 || g->R == 4 || g->R == 8 || g->R == 16 || g->R == 32))
+        return fail(ZHA_ERR_ARG, "R must be 1, 2, 4, 8, 16 or 32");
+    if (g->d != 64 && g->d != 128) return fail(ZHA_ERR_ARG, "d must be 64 or 128");
+    if (g->n_kv_heads < 1 || g->n_q_heads < g->n_kv_heads || g->n_q_heads % g->n_kv_heads)
+        return fail(ZHA_ERR_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+    if (g->capacity < 1 || g->capacity > (int64_t(1) << 31) - 1)
+        return fail(ZHA_ERR_ARG, "capacity must be in [1, 2^31)");
+    if (g->capacity / g->C > (int64_t(1) << 24))
+        return fail(ZHA_ERR_ARG, "capacity / C must be <= 2^24 level-1 nodes");
+    double top = pow((double)g->C, (double)g->L);
+    if (top > 4.0e15) return fail(ZHA_ERR_ARG, "C^L too large");
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_tree_create(const zha_geometry* g, zha_tree** out) {
+    zha_status st = check_geometry(g);
+    if (st != ZHA_OK) return st;
+    if (!out) return fail(ZHA_ERR_ARG, "out is NULL");
+    zha_tree* t = new zha_tree();
+    memset(t, 0, sizeof(*t));
+    t->g = *g;
+    t->ns = record_stride(g->R, g->d);
+    size_t off = 0;
+    size_t rec_off[kMaxL + 1] = {0}, lse_off[kMaxL + 1] = {0};
+    for (int l = 1; l <= g->L; ++l) {
+        const int64_t span = ipow(g->C, l);
+        t->cap[l] = g->capacity / span;
+        rec_off[l] = off;
+        off += up256((size_t)g->n_kv_heads * t->cap[l] * t->ns * sizeof(float));
+        lse_off[l] = off;
+        off += up256((size_t)g->n_kv_heads * t->cap[l] * g->R * sizeof(float));
+    }
+    const size_t qref_off = off;
+    off += up256((size_t)g->n_kv_heads * g->R * g->d * 2);
+    cudaGetDevice(&t->device);
+    cudaError_t e = cudaMalloc(&t->block, off);
+    if (e != cudaSuccess) {
+        delete t;
+        return fail(ZHA_ERR_CUDA, std::string("cudaMalloc(tree): ") + cudaGetErrorString(e));
+    }
+    t->bytes = off;
+    char* base = static_cast<char*>(t->block);
+    for (int l = 1; l <= g->L; ++l) {
+        t->rec[l] = reinterpret_cast<float*>(base + rec_off[l]);
+        t->lse[l] = reinterpret_cast<float*>(base + lse_off[l]);
+    }
+    t->qref = reinterpret_cast<__nv_bfloat16*>(base + qref_off);
+    *out = t;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_tree_destroy(zha_tree* t) {
+    if (!t) return ZHA_OK;
+    cudaDeviceSynchronize();
+    cudaFree(t->block);
+    delete t;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_tree_info(const zha_tree* t, zha_geometry* g, int64_t* n_tokens,
+                                    int64_t* level_nodes, int64_t* device_bytes) {
+    if (!t) return fail(ZHA_ERR_ARG, "tree is NULL");
+    if (g) *g = t->g;
+    if (n_tokens) *n_tokens = t->n_tokens;
+    if (level_nodes)
+        for (int l = 1; l <= t->g.L; ++l) level_nodes[l - 1] = t->n_tokens / ipow(t->g.C, l);
+    if (device_bytes) *device_bytes = (int64_t)t->bytes;
+    return ZHA_OK;
+}
+
+// Summaries of every node completed by growing the token count from n_old to n_new.
+static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t n_new, cudaStream_t st) {
+    const zha_geometry& g = t->g;
+    const int C = g.C, L = g.L;
+    BuildArgs ba;
+    memset(&ba, 0, sizeof(ba));
+    ba.K = static_cast<const __nv_bfloat16*>(K);
+    ba.ld = g.capacity;
+    ba.qref = t->qref;
+    ba.Hkv = g.n_kv_heads;
+    ba.R = g.R;
+    ba.C = C;
+    ba.ns = t->ns;
+    ba.scale = score_scale(g.d);
+    for (int l = 1; l <= L; ++l) {
+        ba.rec[l] = t->rec[l];
+        ba.lse[l] = t->lse[l];
+        ba.cap[l] = t->cap[l];
+    }
+    auto merge = [&](int l, int64_t lo, int64_t hi) -> zha_status {
+        if (hi <= lo) return ZHA_OK;
+        MergeArgs ma;
+        memset(&ma, 0, sizeof(ma));
+        ma.qref = t->qref;
+        ma.Hkv = g.n_kv_heads;
+        ma.R = g.R;
+        ma.C = C;
+        ma.ns = t->ns;
+        ma.p0 = lo;
+        ma.np = hi - lo;
+        ma.scale = score_scale(g.d);
+        ma.child_rec = t->rec[l - 1];
+        ma.child_lse = t->lse[l - 1];
+        ma.child_cap = t->cap[l - 1];
+        ma.rec = t->rec[l];
+        ma.lse = t->lse[l];
+        ma.cap = t->cap[l];
+        ZHA_CUDA(launch_merge(ma, g.d, st));
+        return ZHA_OK;
+    };
+    int first_merge = 2;
+    int64_t lo1 = n_old / C;
+    if (n_old == 0) {
+        // Whole subtrees of up to 256 tokens are streamed by one worker each.
+        int k_emit = 1;
+        while (k_emit < L && ipow(C, k_emit + 1) <= 256) ++k_emit;
+        const int64_t n_emit = n_new / ipow(C, k_emit);
+        ba.k_emit = k_emit;
+        ba.u0 = 0;
+        ba.nu = n_emit;
+        ZHA_CUDA(launch_build_stream(ba, g.d, st));
+        lo1 = n_emit * ipow(C, k_emit - 1);
+        ba.k_emit = 1;
+        ba.u0 = lo1;
+        ba.nu = n_new / C - lo1;
+        ZHA_CUDA(launch_build_stream(ba, g.d, st));
+        for (int l = 2; l <= k_emit; ++l) {
+            zha_status s2 = merge(l, n_emit * ipow(C, k_emit - l), n_new / ipow(C, l));
+            if (s2 != ZHA_OK) return s2;
+        }
+        first_merge = k_emit + 1;
+        for (int l = first_merge; l <= L; ++l) {
+            zha_status s2 = merge(l, 0, n_new / ipow(C, l));
+            if (s2 != ZHA_OK) return s2;
+        }
+        return ZHA_OK;
+    }
+    ba.k_emit = 1;
+    ba.u0 = lo1;
+    ba.nu = n_new / C - lo1;
+    ZHA_CUDA(launch_build_stream(ba, g.d, st));
+    for (int l = 2; l <= L; ++l) {
+        const int64_t span = ipow(C, l);
+        zha_status s2 = merge(l, n_old / span, n_new / span);
+        if (s2 != ZHA_OK) return s2;
+    }
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_build_tree(zha_tree* t, const void* K, int64_t n_tokens, const void* q_ref,
+                                     void* stream) {
+    if (!t) return fail(ZHA_ERR_ARG, "tree is NULL");
+    if (!K || !q_ref) return fail(ZHA_ERR_ARG, "K or q_ref is NULL");
+    if (!aligned16(K) || !aligned16(q_ref)) return fail(ZHA_ERR_ARG, "K and q_ref must be 16-byte aligned");
+    if (n_tokens < 0 || n_tokens > t->g.capacity)
+        return fail(ZHA_ERR_CAPACITY, "n_tokens must be in [0, capacity]");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ZHA_CUDA(cudaMemcpyAsync(t->qref, q_ref, (size_t)t->g.n_kv_heads * t->g.R * t->g.d * 2,
+                             cudaMemcpyDeviceToDevice, st));
+    zha_status s = run_levels(t, K, 0, n_tokens, st);
+    if (s != ZHA_OK) return s;
+    t->n_tokens = n_tokens;
+    t->built = true;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_append(zha_tree* t, const void* K, int64_t n_old, int64_t n_new, void* stream) {
+    if (!t) return fail(ZHA_ERR_ARG, "tree is NULL");
+    if (!t->built) return fail(ZHA_ERR_STATE, "append before zha_build_tree");
+    if (!K || !aligned16(K)) return fail(ZHA_ERR_ARG, "K must be a 16-byte aligned device pointer");
+    if (n_old != t->n_tokens) return fail(ZHA_ERR_STATE, "n_old differs from the tree's token count");
+    if (n_new < 0) return fail(ZHA_ERR_ARG, "n_new must be >= 0");
+    if (n_old + n_new > t->g.capacity) return fail(ZHA_ERR_CAPACITY, "n_old + n_new exceeds capacity");
+    if (n_new == 0) return ZHA_OK;
+    zha_status s = run_levels(t, K, n_old, n_old + n_new, static_cast<cudaStream_t>(stream));
+    if (s != ZHA_OK) return s;
+    t->n_tokens = n_old + n_new;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_tree_export(const zha_tree* t, int32_t level, float* m, float* lse, float* b,
+                                      void* stream) {
+    if (!t) return fail(ZHA_ERR_ARG, "tree is NULL");
+    if (level < 1 || level > t->g.L) return fail(ZHA_ERR_ARG, "level out of range");
+    const zha_geometry& g = t->g;
+    const int64_t nl = t->n_tokens / ipow(g.C, level);
+    if (nl == 0) return ZHA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int h = 0; h < g.n_kv_heads; ++h) {
+        const float* src = t->rec[level] + (int64_t)h * t->cap[level] * t->ns;
+        if (m)
+            ZHA_CUDA(cudaMemcpy2DAsync(m + (int64_t)h * nl * g.R * g.d, (size_t)g.R * g.d * 4, src,
+                                       (size_t)t->ns * 4, (size_t)g.R * g.d * 4, (size_t)nl,
+                                       cudaMemcpyDeviceToDevice, st));
+        if (b)
+            ZHA_CUDA(cudaMemcpy2DAsync(b + (int64_t)h * nl * g.R, (size_t)g.R * 4, src + (int64_t)g.R * g.d,
+                                       (size_t)t->ns * 4, (size_t)g.R * 4, (size_t)nl,
+                                       cudaMemcpyDeviceToDevice, st));
+        if (lse)
+            ZHA_CUDA(cudaMemcpyAsync(lse + (int64_t)h * nl * g.R, t->lse[level] + (int64_t)h * t->cap[level] * g.R,
+                                     (size_t)nl * g.R * 4, cudaMemcpyDeviceToDevice, st));
+    }
+    return ZHA_OK;
+}
+
+// ------------------------------------------------------------------------------ decoder
+
+extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n_seq, int32_t max_queries,
+                                         zha_decoder** out) {
+    if (!trees || n_seq < 1) return fail(ZHA_ERR_ARG, "need at least one tree");
+    if (max_queries < 1) return fail(ZHA_ERR_ARG, "max_queries must be >= 1");
+    if (!out) return fail(ZHA_ERR_ARG, "out is NULL");
+    for (int s = 0; s < n_seq; ++s) {
+        if (!trees[s]) return fail(ZHA_ERR_ARG, "a tree is NULL");
+        const zha_geometry& a = trees[s]->g;
+        const zha_geometry& b0 = trees[0]->g;
+        if (a.d != b0.d || a.n_q_heads != b0.n_q_heads || a.n_kv_heads != b0.n_kv_heads)
+            return fail(ZHA_ERR_ARG, "trees of one decoder must share d, n_q_heads and n_kv_heads");
+    }
+    zha_decoder* dec = new zha_decoder();
+    dec->trees.assign(trees, trees + n_seq);
+    const zha_geometry& g0 = trees[0]->g;
+    dec->n_seq = n_seq;
+    dec->max_q = max_queries;
+    dec->Hq = g0.n_q_heads;
+    dec->Hkv = g0.n_kv_heads;
+    dec->d = g0.d;
+    dec->G = g0.n_q_heads / g0.n_kv_heads;
+    dec->Lmax = 0;
+    for (auto* t : dec->trees) dec->Lmax = t->g.L > dec->Lmax ? t->g.L : dec->Lmax;
+    dec->lanes_cap = (int64_t)n_seq * max_queries * dec->Hq;
+    dec->groups_cap = (int64_t)n_seq * dec->Hkv;
+    dec->last_n_q = 0;
+    dec->routed = false;
+
+    Work& w = dec->w;
+    memset(&w, 0, sizeof(w));
+    int64_t cap1 = 1, s_cap = 1;
+    for (int l = 1; l <= dec->Lmax; ++l) {
+        int64_t W = 1;
+        for (auto* t : dec->trees)
+            if (l <= t->g.L) W = std::max<int64_t>(W, (t->cap[l] + 31) / 32);
+        w.W[l] = W;
+    }
+    for (auto* t : dec->trees) {
+        cap1 = std::max<int64_t>(cap1, t->cap[1]);
+        const int64_t top = ipow(t->g.C, t->g.L);
+        const int64_t nseg_max = 1 + t->cap[1] + (std::min<int64_t>(top, t->g.capacity) + t->g.C - 1) / t->g.C;
+        const int64_t segs = segs_per_split(1, t->g.C);
+        s_cap = std::max<int64_t>(s_cap, (nseg_max + segs - 1) / segs);
+    }
+    w.lanes_cap = dec->lanes_cap;
+    w.es = (cap1 + 3) / 4 * 4;
+    w.us = cap1;
+    w.s_cap = s_cap;
+
+    size_t off = 0;
+    size_t kept_off[kMaxL + 2] = {0};
+    for (int l = 1; l <= dec->Lmax; ++l) {
+        kept_off[l] = off;
+        off += up256((size_t)dec->lanes_cap * w.W[l] * 4);
+    }
+    const size_t kcount_off = off;
+    off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
+    const size_t e_off = off;
+    off += up256((size_t)dec->lanes_cap * w.es * 4);
+    const size_t ulist_off = off;
+    off += up256((size_t)dec->groups_cap * w.us * 4);
+    const size_t ucount_off = off;
+    off += up256((size_t)dec->groups_cap * 4);
+    const size_t part_off = off;
+    off += up256((size_t)dec->lanes_cap * w.s_cap * (dec->d + 4) * 4);
+    const size_t ctr_off = off;
+    off += up256((size_t)kCtrCount * 8);
+    const size_t status_off = off;
+    off += up256(4);
+    const size_t seq_off = off;
+    off += up256((size_t)n_seq * sizeof(SeqDev));
+    cudaError_t e = cudaMalloc(&dec->block, off);
+    if (e != cudaSuccess) {
+        delete dec;
+        return fail(ZHA_ERR_CUDA, std::string("cudaMalloc(decoder workspace): ") + cudaGetErrorString(e));
+    }
+    dec->bytes = off;
+    char* base = static_cast<char*>(dec->block);
+    for (int l = 1; l <= dec->Lmax; ++l) w.kept[l] = reinterpret_cast<uint32_t*>(base + kept_off[l]);
+    w.kcount = reinterpret_cast<int32_t*>(base + kcount_off);
+    w.e = reinterpret_cast<float*>(base + e_off);
+    w.ulist = reinterpret_cast<int32_t*>(base + ulist_off);
+    w.ucount = reinterpret_cast<int32_t*>(base + ucount_off);
+    w.part = reinterpret_cast<float*>(base + part_off);
+    w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);
+    w.status = reinterpret_cast<int32_t*>(base + status_off);
+    dec->seq_dev = reinterpret_cast<SeqDev*>(base + seq_off);
+    dec->seq_host.resize(n_seq);
+    cudaMemset(w.ctr, 0, (size_t)kCtrCount * 8);
+    cudaMemset(w.status, 0, 4);
+    *out = dec;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_decoder_destroy(zha_decoder* dec) {
+    if (!dec) return ZHA_OK;
+    cudaDeviceSynchronize();
+    cudaFree(dec->block);
+    delete dec;
+    return ZHA_OK;
+}
+
+static zha_status fill_seqs(zha_decoder* dec, const void* const* K, const void* const* V) {
+    for (int s = 0; s < dec->n_seq; ++s) {
+        const zha_tree* t = dec->trees[s];
+        if (!t->built) return fail(ZHA_ERR_STATE, "a tree of the decoder has not been built");
+        if (t->n_tokens < 1) return fail(ZHA_ERR_STATE, "a tree of the decoder holds no tokens");
+        SeqDev& sd = dec->seq_host[s];
+        memset(&sd, 0, sizeof(sd));
+        sd.C = t->g.C;
+        sd.L = t->g.L;
+        sd.R = t->g.R;
+        sd.ns = t->ns;
+        sd.N = t->n_tokens;
+        sd.top = ipow(t->g.C, t->g.L);
+        sd.T = sd.N / sd.top;
+        sd.ld = t->g.capacity;
+        for (int l = 1; l <= t->g.L; ++l) {
+            sd.n[l] = sd.N / ipow(t->g.C, l);
+            sd.cap[l] = t->cap[l];
+            sd.rec[l] = t->rec[l];
+        }
+        if (K) sd.K = static_cast<const __nv_bfloat16*>(K[s]);
+        if (V) sd.V = static_cast<const __nv_bfloat16*>(V[s]);
+    }
+    return ZHA_OK;
+}
+
+static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, float p) {
+    Batch b;
+    b.seqs = dec->seq_dev;
+    b.n_seq = dec->n_seq;
+    b.n_q = n_q;
+    b.Hq = dec->Hq;
+    b.Hkv = dec->Hkv;
+    b.G = dec->G;
+    b.d = dec->d;
+    b.n_gl = n_q * dec->G;
+    b.n_lanes = dec->n_seq * n_q * dec->Hq;
+    b.n_groups = dec->n_seq * dec->Hkv;
+    b.Q = static_cast<const __nv_bfloat16*>(Q);
+    b.p = p;
+    return b;
+}
+
+extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (!Q || !aligned16(Q)) return fail(ZHA_ERR_ARG, "Q must be a 16-byte aligned device pointer");
+    if (n_q < 1 || n_q > dec->max_q) return fail(ZHA_ERR_CAPACITY, "n_q must be in [1, max_queries]");
+    if (!(p > 0.0f) || isnan(p)) return fail(ZHA_ERR_ARG, "p must be > 0");
+    zha_status s = fill_seqs(dec, nullptr, nullptr);
+    if (s != ZHA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ZHA_CUDA(cudaMemcpyAsync(dec->seq_dev, dec->seq_host.data(), sizeof(SeqDev) * dec->n_seq,
+                             cudaMemcpyHostToDevice, st));
+    const Batch b = make_batch(dec, Q, n_q, p);
+    for (int l = 1; l <= dec->Lmax; ++l)
+        ZHA_CUDA(cudaMemsetAsync(dec->w.kept[l], 0, (size_t)b.n_lanes * dec->w.W[l] * 4, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.ctr, 0, (size_t)kCtrCount * 8, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.status, 0, 4, st));
+    const float scale = score_scale(dec->d);
+    for (int it = 0; it < dec->Lmax; ++it) {
+        if (it > 0) ZHA_CUDA(launch_union(b, dec->w, it, 0, st));
+        ZHA_CUDA(launch_score(b, dec->w, it, scale, st));
+        ZHA_CUDA(launch_select(b, dec->w, it, st));
+    }
+    dec->routed = true;
+    dec->last_n_q = n_q;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
+                                      const void* Q, int32_t n_q, float* out, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (!dec->routed || n_q != dec->last_n_q) return fail(ZHA_ERR_STATE, "zha_sparse_attn needs a zha_route with the same n_q first");
+    if (!K || !V || !Q || !out) return fail(ZHA_ERR_ARG, "K, V, Q and out must be non-NULL");
+    if (!aligned16(Q) || !aligned16(out)) return fail(ZHA_ERR_ARG, "Q and out must be 16-byte aligned");
+    for (int s = 0; s < dec->n_seq; ++s)
+        if (!K[s] || !V[s] || !aligned16(K[s]) || !aligned16(V[s]))
+            return fail(ZHA_ERR_ARG, "K[s] and V[s] must be 16-byte aligned device pointers");
+    zha_status s = fill_seqs(dec, K, V);
+    if (s != ZHA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ZHA_CUDA(cudaMemcpyAsync(dec->seq_dev, dec->seq_host.data(), sizeof(SeqDev) * dec->n_seq,
+                             cudaMemcpyHostToDevice, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.ctr + kCtrUnionTokens, 0, 2 * 8, st));
+    const Batch b = make_batch(dec, Q, n_q, 1.0f);
+    int64_t max_splits = 0;
+    for (const SeqDev& sd : dec->seq_host) {
+        const int64_t nseg = 1 + sd.n[1] + (std::min<int64_t>(sd.top, sd.N) + sd.C - 1) / sd.C;
+        const int64_t segs = segs_per_split(b.n_gl, sd.C);
+        max_splits = std::max<int64_t>(max_splits, (nseg + segs - 1) / segs);
+    }
+    if (max_splits > dec->w.s_cap) return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
+    ZHA_CUDA(launch_union(b, dec->w, 0, 1, st));
+    ZHA_CUDA(launch_attn(b, dec->w, max_splits, score_scale(dec->d), st));
+    ZHA_CUDA(launch_combine(b, dec->w, out, st));
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
+                                 const void* Q, int32_t n_q, float p, float* out, void* stream) {
+    zha_status s = zha_route(dec, Q, n_q, p, stream);
+    if (s != ZHA_OK) return s;
+    return zha_sparse_attn(dec, K, V, Q, n_q, out, stream);
+}
+
+extern "C" int64_t zha_decoder_words(const zha_decoder* dec, int32_t level) {
+    if (!dec || level < 1 || level > dec->Lmax) return 0;
+    return dec->w.W[level];
+}
+
+extern "C" zha_status zha_decoder_export_kept(const zha_decoder* dec, int32_t level, uint32_t* bits,
+                                              int32_t* counts, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (!dec->routed) return fail(ZHA_ERR_STATE, "no zha_route yet");
+    if (level < 1 || level > dec->Lmax) return fail(ZHA_ERR_ARG, "level out of range");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n_lanes = (int64_t)dec->n_seq * dec->last_n_q * dec->Hq;
+    if (bits)
+        ZHA_CUDA(cudaMemcpyAsync(bits, dec->w.kept[level], (size_t)n_lanes * dec->w.W[level] * 4,
+                                 cudaMemcpyDeviceToDevice, st));
+    if (counts) {
+        // Lanes of trees with fewer levels never write their count at this level.
+        for (int s = 0; s < dec->n_seq; ++s) {
+            const int64_t l0 = (int64_t)s * dec->last_n_q * dec->Hq, nl = (int64_t)dec->last_n_q * dec->Hq;
+            if (level <= dec->trees[s]->g.L)
+                ZHA_CUDA(cudaMemcpyAsync(counts + l0, dec->w.kcount + (int64_t)level * dec->lanes_cap + l0,
+                                         (size_t)nl * 4, cudaMemcpyDeviceToDevice, st));
+            else
+                ZHA_CUDA(cudaMemsetAsync(counts + l0, 0, (size_t)nl * 4, st));
+        }
+    }
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats* out, void* stream) {
+    if (!dec || !out) return fail(ZHA_ERR_ARG, "decoder or out is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned long long ctr[kCtrCount];
+    int32_t status = 0;
+    ZHA_CUDA(cudaMemcpyAsync(ctr, dec->w.ctr, sizeof(ctr), cudaMemcpyDeviceToHost, st));
+    ZHA_CUDA(cudaMemcpyAsync(&status, dec->w.status, 4, cudaMemcpyDeviceToHost, st));
+    ZHA_CUDA(cudaStreamSynchronize(st));
+    memset(out, 0, sizeof(*out));
+    for (int l = 1; l <= kMaxL; ++l) {
+        out->union_nodes[l - 1] = (int64_t)ctr[kCtrUnionNodes + l];
+        out->lane_nodes[l - 1] = (int64_t)ctr[kCtrLaneNodes + l];
+    }
+    out->union_tokens = (int64_t)ctr[kCtrUnionTokens];
+    out->lane_tokens = (int64_t)ctr[kCtrLaneTokens];
+    const zha_geometry& g = dec->trees[0]->g;
+    out->node_bytes = (int64_t)(g.R * g.d + g.R) * 4;
+    out->status = status;
+    return status ? fail(ZHA_ERR_DEVICE, "device status word is set") : ZHA_OK;
+}

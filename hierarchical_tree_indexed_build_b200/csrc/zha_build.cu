@@ -1,0 +1,297 @@
+// zha_build.cu - tree build kernels (level-1 chunk summaries, level-up merges).
+//
+// What is computed (pages: "Zyphra ZHA 稀疏注意力…" fluxbbs.com, section 树形索引是怎么搭的;
+// "Zyphra发布层级注意力ZHA…" wqu.guru, section "Building the tree"): for chunk j of KV head g
+// and reference query q_r,
+//     a_t = s q_r.k_t,   lse_r = log sum_t exp(a_t),   m_r = sum_t exp(a_t - lse_r) k_t,
+//     b_r = lse_r - s q_r.m_r,
+// and a level-l node is the online-softmax merge of its C children, i.e. the same summary
+// over its C^l raw tokens.
+//
+// Thread mapping: a "worker" of 4R threads summarises one node; thread (r, quarter) owns
+// reference query r and the dimensions {16 i + 4 quarter + c : c < 4} (interleaved so the
+// four quarters of a row are 64 contiguous bytes).  The running state of a node is the
+// unnormalised online softmax (mx, z, acc[]) with acc = sum_t exp(a_t - mx) k_t.
+#include <math.h>
+
+#include "zha_common.cuh"
+#include "zha_launch.h"
+#include "zha_profile.h"
+
+namespace zha {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16* row, int q, float (&v)[D / 4]) {
+    const uint2* p = reinterpret_cast<const uint2*>(row);
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+        const uint2 u = __ldg(p + 4 * i + q);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v[4 * i + 0] = a.x;
+        v[4 * i + 1] = a.y;
+        v[4 * i + 2] = b.x;
+        v[4 * i + 3] = b.y;
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void load_row_f32(const float* row, int q, float (&v)[D / 4]) {
+    const float4* p = reinterpret_cast<const float4*>(row);
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+        const float4 u = __ldg(p + 4 * i + q);
+        v[4 * i + 0] = u.x;
+        v[4 * i + 1] = u.y;
+        v[4 * i + 2] = u.z;
+        v[4 * i + 3] = u.w;
+    }
+}
+
+// Sum over the 4 quarter-threads of a row.
+__device__ __forceinline__ float quad_sum(float v) {
+    v += __shfl_xor_sync(kFull, v, 1);
+    v += __shfl_xor_sync(kFull, v, 2);
+    return v;
+}
+
+// Turn a running state into the stored summary of one node and write it:
+// m_r = acc / z, lse_r = mx + log z, b_r = lse_r - s q_r.m_r.  Returns lse_r; m_r is left
+// in `m` so the parent can fold exactly the stored values.
+template <int D>
+__device__ __forceinline__ float finalize_store(float mx, float z, const float (&acc)[D / 4],
+                                                const float (&qv)[D / 4], float scale, float* rec,
+                                                float* lse, int r, int q, int R, bool store,
+                                                float (&m)[D / 4]) {
+    const float inv = 1.0f / z;
+    float qm = 0.0f;
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) {
+        m[k] = acc[k] * inv;
+        qm = fmaf(qv[k], m[k], qm);
+    }
+    qm = quad_sum(qm);
+    const float l = mx + logf(z);
+    if (store) {
+        float4* dst = reinterpret_cast<float4*>(rec + (int64_t)r * D);
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i)
+            dst[4 * i + q] = make_float4(m[4 * i], m[4 * i + 1], m[4 * i + 2], m[4 * i + 3]);
+        if (q == 0) {
+            rec[(int64_t)R * D + r] = fmaf(-scale, qm, l);
+            lse[r] = l;
+        }
+    }
+    return l;
+}
+
+// Online-softmax merge of one child summary (lse_c, m_c) into a parent state (mx, z, acc):
+// the same arithmetic, in the same order, in the streaming build and in k_merge, so a tree
+// grown by appends is bit-identical to one built in one pass.
+template <int D>
+__device__ __forceinline__ void fold_child(float& mx, float& z, float (&acc)[D / 4], float lc,
+                                           const float (&mc)[D / 4]) {
+    const float mn = fmaxf(mx, lc);
+    const float cp = expf(mx - mn);   // mx = -inf -> 0
+    const float cc = expf(lc - mn);
+    z = fmaf(z, cp, cc);
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], cp, mc[k] * cc);
+    mx = mn;
+}
+
+template <int D>
+__device__ __forceinline__ void load_state(const float* st, int stride, float& mx, float& z, float (&acc)[D / 4]) {
+    mx = st[0];
+    z = st[stride];
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) acc[k] = st[(2 + k) * stride];
+}
+
+template <int D>
+__device__ __forceinline__ void store_state(float* st, int stride, float mx, float z, const float (&acc)[D / 4]) {
+    st[0] = mx;
+    st[stride] = z;
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) st[(2 + k) * stride] = acc[k];
+}
+
+template <int D>
+__device__ __forceinline__ void fold_into_smem(float* st, int stride, float lc, const float (&mc)[D / 4]) {
+    float mx, z, acc[D / 4];
+    load_state<D>(st, stride, mx, z, acc);
+    fold_child<D>(mx, z, acc, lc, mc);
+    store_state<D>(st, stride, mx, z, acc);
+}
+
+template <int D>
+__device__ __forceinline__ void reset_smem(float* st, int stride) {
+    st[0] = -INFINITY;
+    st[stride] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) st[(2 + k) * stride] = 0.0f;
+}
+
+// Streams the C^k_emit tokens of one level-k_emit node per worker and emits the summaries of
+// every node of levels 1..k_emit beneath it.  Level-1 state lives in registers, levels
+// 2..k_emit in shared memory ([level][field][thread]).
+template <int D>
+__global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
+    extern __shared__ float smem_state[];
+    const int wt = 4 * a.R;
+    const int wpb = blockDim.x / wt;
+    const int tid = threadIdx.x;
+    const int r = (tid % wt) >> 2;
+    const int q = tid & 3;
+    int64_t widx = (int64_t)blockIdx.x * wpb + tid / wt;
+    const int64_t total = (int64_t)a.Hkv * a.nu;
+    const bool active = widx < total;
+    if (!active) widx = total - 1;
+    const int g = (int)(widx / a.nu);
+    const int64_t u = a.u0 + widx % a.nu;
+    const int C = a.C;
+
+    float qv[D / 4];
+    load_row_bf16<D>(a.qref + ((int64_t)g * a.R + r) * D, q, qv);
+
+    const int nst = a.k_emit - 1;   // shared-memory levels (2..k_emit)
+    const int stride = blockDim.x;
+    for (int l = 0; l < nst; ++l) reset_smem<D>(smem_state + (int64_t)l * (D / 4 + 2) * stride + tid, stride);
+
+    int64_t span_emit = 1;
+    for (int l = 0; l < a.k_emit; ++l) span_emit *= C;
+    const int64_t t0 = u * span_emit;
+    const __nv_bfloat16* Kg = a.K + ((int64_t)g * a.ld + t0) * D;
+
+    float mx = -INFINITY, z = 0.0f, acc[D / 4];
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
+
+    float kv[D / 4], kn[D / 4];
+    load_row_bf16<D>(Kg, q, kn);
+    int left = C;   // tokens left in the current level-1 chunk
+    for (int64_t tt = 0; tt < span_emit; ++tt) {
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) kv[k] = kn[k];
+        if (tt + 1 < span_emit) load_row_bf16<D>(Kg + (tt + 1) * D, q, kn);
+        float dot = 0.0f;
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) dot = fmaf(qv[k], kv[k], dot);
+        const float sc = a.scale * quad_sum(dot);
+        const float mn = fmaxf(mx, sc);
+        const float c = expf(mx - mn);
+        const float w = expf(sc - mn);
+        z = fmaf(z, c, w);
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], c, w * kv[k]);
+        mx = mn;
+        if (--left == 0) {
+            left = C;
+            const int64_t t = t0 + tt;
+            const int64_t j1 = t / C;
+            float m1[D / 4];
+            const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
+                                               a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
+                                               a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
+                                               active, m1);
+            if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
+            mx = -INFINITY;
+            z = 0.0f;
+#pragma unroll
+            for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
+            // cascade completed ancestors (levels 2..k_emit)
+            int64_t span = C;
+            for (int l = 2; l <= a.k_emit; ++l) {
+                span *= C;
+                if ((tt + 1) % span != 0) break;
+                float* st = smem_state + (int64_t)(l - 2) * (D / 4 + 2) * stride + tid;
+                float smx, sz, sacc[D / 4], ml[D / 4];
+                load_state<D>(st, stride, smx, sz, sacc);
+                const int64_t jl = t / span;
+                const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
+                                                   a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
+                                                   a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
+                                                   active, ml);
+                if (l < a.k_emit)
+                    fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
+                reset_smem<D>(st, stride);
+            }
+        }
+    }
+}
+
+// Merges the C children (level l-1) of each parent node P in [p0, p0+np) at level l:
+// lse_P = log sum_c exp(lse_c), m_P = sum_c exp(lse_c - lse_P) m_c, b_P = lse_P - s q_r.m_P.
+template <int D>
+__global__ void __launch_bounds__(128) k_merge(MergeArgs a) {
+    const int wt = 4 * a.R;
+    const int wpb = blockDim.x / wt;
+    const int tid = threadIdx.x;
+    const int r = (tid % wt) >> 2;
+    const int q = tid & 3;
+    int64_t widx = (int64_t)blockIdx.x * wpb + tid / wt;
+    const int64_t total = (int64_t)a.Hkv * a.np;
+    const bool active = widx < total;
+    if (!active) widx = total - 1;
+    const int g = (int)(widx / a.np);
+    const int64_t P = a.p0 + widx % a.np;
+
+    float qv[D / 4];
+    load_row_bf16<D>(a.qref + ((int64_t)g * a.R + r) * D, q, qv);
+
+    const float* crec = a.child_rec + ((int64_t)g * a.child_cap + P * a.C) * a.ns;
+    const float* clse = a.child_lse + ((int64_t)g * a.child_cap + P * a.C) * a.R;
+    float mx = -INFINITY, z = 0.0f, acc[D / 4], mc[D / 4], mo[D / 4];
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
+    for (int c = 0; c < a.C; ++c) {
+        load_row_f32<D>(crec + (int64_t)c * a.ns + (int64_t)r * D, q, mc);
+        const float lc = __ldg(clse + (int64_t)c * a.R + r);
+        fold_child<D>(mx, z, acc, lc, mc);
+    }
+    finalize_store<D>(mx, z, acc, qv, a.scale, a.rec + ((int64_t)g * a.cap + P) * a.ns,
+                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, mo);
+}
+
+int workers_per_block(int R) {
+    const int wt = 4 * R;
+    return wt >= 128 ? 1 : 128 / wt;
+}
+
+}  // namespace
+
+cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st) {
+    if (a.nu <= 0) return cudaSuccess;
+    const int wpb = workers_per_block(a.R);
+    const int threads = wpb * 4 * a.R;
+    const int64_t blocks = ((int64_t)a.Hkv * a.nu + wpb - 1) / wpb;
+    const size_t smem = (size_t)(a.k_emit - 1) * (d / 4 + 2) * threads * sizeof(float);
+    ProfScope ps_("k_build_stream", st);
+    if (d == 128) {
+        cudaFuncSetAttribute(k_build_stream<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_build_stream<128><<<(unsigned)blocks, threads, smem, st>>>(a);
+    } else {
+        cudaFuncSetAttribute(k_build_stream<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_build_stream<64><<<(unsigned)blocks, threads, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st) {
+    if (a.np <= 0) return cudaSuccess;
+    const int wpb = workers_per_block(a.R);
+    const int threads = wpb * 4 * a.R;
+    const int64_t blocks = ((int64_t)a.Hkv * a.np + wpb - 1) / wpb;
+    ProfScope ps_("k_merge", st);
+    if (d == 128)
+        k_merge<128><<<(unsigned)blocks, threads, 0, st>>>(a);
+    else
+        k_merge<64><<<(unsigned)blocks, threads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace zha

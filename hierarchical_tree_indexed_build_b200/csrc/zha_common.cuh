@@ -1,0 +1,84 @@
+// zha_common.cuh - device-side tables and helpers shared by the libzha kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zha.h"
+
+namespace zha {
+
+constexpr int kMaxL = ZHA_MAX_LEVELS;
+
+// Node record layout in HBM (per level, per KV head, per node): m [R][d] f32 followed by
+// b [R] f32, stride `ns` floats = R*(d+1) rounded up to 8 floats (32-byte sectors).
+// lse [R] f32 is kept in a separate array per level (read only by merges and export).
+inline __host__ __device__ int32_t record_stride(int R, int d) { return ((R * (d + 1) + 7) / 8) * 8; }
+
+// One sequence of a decode batch, as the kernels see it.
+struct SeqDev {
+    int32_t C, L, R, ns;
+    int64_t N;                       // tokens present
+    int64_t T;                       // complete top-level nodes = N / C^L
+    int64_t top;                     // C^L
+    int64_t ld;                      // K/V rows per KV head (capacity)
+    int64_t n[kMaxL + 1];            // complete nodes per level (index = level)
+    int64_t cap[kMaxL + 1];          // node capacity per level
+    const float* rec[kMaxL + 1];     // [Hkv][cap_l][ns]
+    const __nv_bfloat16* K;          // [Hkv][ld][d]
+    const __nv_bfloat16* V;
+};
+
+// Counter slots (unsigned long long).
+constexpr int kCtrUnionNodes = 0;              // + level
+constexpr int kCtrLaneNodes = kMaxL + 1;       // + level
+constexpr int kCtrUnionTokens = 2 * kMaxL + 2;
+constexpr int kCtrLaneTokens = 2 * kMaxL + 3;
+constexpr int kCtrCount = 2 * kMaxL + 4;
+
+// Decoder workspace as the kernels see it.
+struct Work {
+    uint32_t* kept[kMaxL + 2];       // kept[l]: [lanes_cap][W[l]] bitmaps
+    int64_t W[kMaxL + 2];
+    int32_t* kcount;                 // [(kMaxL+1)][lanes_cap]
+    int64_t lanes_cap;
+    float* e;                        // [lanes_cap][es] scores of the current level
+    int64_t es;
+    int32_t* ulist;                  // [groups_cap][us] union lists
+    int64_t us;
+    int32_t* ucount;                 // [groups_cap]
+    float* part;                     // [lanes_cap][s_cap][d+2] attention partials
+    int64_t s_cap;
+    unsigned long long* ctr;         // kCtrCount counters
+    int32_t* status;                 // device status word (0 = ok)
+};
+
+// A decode call's shape.
+struct Batch {
+    const SeqDev* seqs;
+    int32_t n_seq, n_q, Hq, Hkv, G, d;
+    int32_t n_gl;                    // lanes per (sequence, KV head) group = n_q * G
+    int32_t n_lanes, n_groups;
+    const __nv_bfloat16* Q;          // [n_seq][n_q][Hq][d]
+    float p;
+};
+
+// Global lane index of group lane y of group (s, g): lane = (s*n_q + i)*Hq + h.
+__host__ __device__ inline int64_t lane_of(const Batch& b, int s, int g, int y) {
+    const int i = y / b.G, hh = y % b.G;
+    return ((int64_t)s * b.n_q + i) * b.Hq + (int64_t)g * b.G + hh;
+}
+
+// Device status bits.
+constexpr int32_t kStatusSelectFallbackLimit = 1;
+constexpr int32_t kStatusCapacity = 2;
+
+// Split size (tokens) of the attention work for a call with n_gl lanes per group.
+inline __host__ __device__ int split_tokens(int n_gl) { return n_gl <= 64 ? 1024 : 4096; }
+inline __host__ __device__ int64_t segs_per_split(int n_gl, int C) {
+    const int64_t s = split_tokens(n_gl) / C;
+    return s > 0 ? s : 1;
+}
+
+}  // namespace zha

@@ -1,0 +1,52 @@
+// zha_launch.h - kernel argument blocks and launchers (internal to libzha).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zha_common.cuh"
+
+namespace zha {
+
+// Streaming build: workers summarise level-k_emit nodes [u0, u0+nu) of every KV head and
+// write levels 1..k_emit beneath them.
+struct BuildArgs {
+    const __nv_bfloat16* K;      // [Hkv][ld][d]
+    int64_t ld;
+    const __nv_bfloat16* qref;   // [Hkv][R][d]
+    int32_t Hkv, R, C, ns, k_emit;
+    int64_t u0, nu;
+    float scale;
+    float* rec[kMaxL + 1];
+    float* lse[kMaxL + 1];
+    int64_t cap[kMaxL + 1];
+};
+
+// Merge: parents [p0, p0+np) of one level from their C children.
+struct MergeArgs {
+    const __nv_bfloat16* qref;
+    int32_t Hkv, R, C, ns;
+    int64_t p0, np;
+    float scale;
+    const float* child_rec;
+    const float* child_lse;
+    int64_t child_cap;
+    float* rec;
+    float* lse;
+    int64_t cap;
+};
+
+cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st);
+cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st);
+
+// Decode (routing + attention).  `it` is the level iteration: sequence s works on level
+// L_s - it.  mode 0 of the union kernel prepares routing iteration it (union of the kept
+// sets of level L_s - it + 1); mode 1 prepares attention (union of level-1 kept sets).
+cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaStream_t st);
+cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
+cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st);
+cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
+cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);
+
+}  // namespace zha

@@ -1,0 +1,562 @@
+// zha_route.cu - top-down top-p routing kernels.
+//
+// What is computed (pages: fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的 —
+// 先给顶层节点打分，保留覆盖估计注意力质量比例 p 的最小节点集合，再逐层展开; wqu.guru, section
+// "How does top-p routing pick tokens?"): for every lane (query token, query head h, KV head
+// g = h*Hkv/Hq) and level l from L down to 1, each frontier node j gets the plane estimate
+//     e_j = max_r ( s q.m_r(j) + b_r(j) ),
+// the frontier's softmax masses P_j = exp(e_j - max e) / sum exp(e - max e) are ordered by
+// (e desc, j asc), and the shortest prefix with cumulative mass >= p is kept (p >= 1 keeps
+// all).  The next frontier is the C children of each kept node.
+//
+// One level of one launch covers every lane of the batch:
+//   k_union  - per (sequence, KV head) group: sorted union of the lanes' kept nodes of the
+//              previous level (their children are the group's candidates);
+//   k_score  - each candidate node record (m, b) is read once per group and scored against
+//              all of the group's lanes (GQA heads and query tokens share the read);
+//   k_select - per lane: deterministic top-p cut (fixed-point masses, radix-style bins on
+//              max e - e, exact (e, j) ordering inside the boundary bin), kept bitmap out.
+#include <math.h>
+
+#include "zha_common.cuh"
+#include "zha_launch.h"
+#include "zha_profile.h"
+
+namespace zha {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ----------------------------------------------------------------------------- block helpers
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+// Block-wide reductions; `red` holds >= 32 elements; all threads get the result.
+template <typename T>
+__device__ T block_sum(T v, T* red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    v = warp_sum(v);
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    T t = (lane < nw) ? red[lane] : T(0);
+    t = warp_sum(t);
+    return t;
+}
+
+__device__ float block_max(float v, float* red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    v = warp_max(v);
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    float t = (lane < nw) ? red[lane] : -INFINITY;
+    return warp_max(t);
+}
+
+template <typename T>
+__device__ __forceinline__ T block_min_t(T v, T* red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const T u = __shfl_xor_sync(kFull, v, o);
+        v = u < v ? u : v;
+    }
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    T t = (lane < nw) ? red[lane] : red[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const T u = __shfl_xor_sync(kFull, t, o);
+        t = u < t ? u : t;
+    }
+    return t;
+}
+
+template <typename T>
+__device__ __forceinline__ T block_max_t(T v, T* red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const T u = __shfl_xor_sync(kFull, v, o);
+        v = u > v ? u : v;
+    }
+    __syncthreads();
+    if (lane == 0) red[wid] = v;
+    __syncthreads();
+    T t = (lane < nw) ? red[lane] : red[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const T u = __shfl_xor_sync(kFull, t, o);
+        t = u > t ? u : t;
+    }
+    return t;
+}
+
+// Block-wide exclusive scan; red holds >= 33 elements; total returned through `total`.
+template <typename T>
+__device__ T block_excl_scan(T v, T* red, T& total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    T incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const T t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    __syncthreads();
+    if (lane == 31) red[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        const T ws = lane < nw ? red[lane] : T(0);
+        T wi = ws;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const T t = __shfl_up_sync(kFull, wi, o);
+            if (lane >= o) wi += t;
+        }
+        red[lane] = wi - ws;
+        if (lane == 31) red[32] = wi;
+    }
+    __syncthreads();
+    total = red[32];
+    return red[wid] + incl - v;
+}
+
+// ----------------------------------------------------------------------------- union
+
+// Sorted union over a group's lanes of the kept nodes at level `ulev`.  Mode 0: ulev =
+// L_s - it + 1 (routing iteration it >= 1); mode 1: ulev = 1 (attention).
+__global__ void __launch_bounds__(1024) k_union(Batch b, Work w, int it, int mode) {
+    __shared__ int red[33];
+    const int grp = blockIdx.x;
+    const int s = grp / b.Hkv, g = grp % b.Hkv;
+    const SeqDev& sq = b.seqs[s];
+    int ulev;
+    if (mode == 0) {
+        const int lev = sq.L - it;
+        if (it == 0 || lev < 1) {
+            if (threadIdx.x == 0) w.ucount[grp] = 0;
+            return;
+        }
+        ulev = lev + 1;
+    } else {
+        ulev = 1;
+        if (sq.T == 0) {
+            if (threadIdx.x == 0) {
+                w.ucount[grp] = 0;
+                atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)sq.N);
+            }
+            return;
+        }
+    }
+    const int64_t nl = sq.n[ulev];
+    const int64_t nwords = (nl + 31) / 32;
+    const uint32_t* kb = w.kept[ulev];
+    const int64_t W = w.W[ulev];
+    int32_t* out = w.ulist + (int64_t)grp * w.us;
+    int base = 0;
+    bool has0 = false;
+    for (int64_t w0 = 0; w0 < nwords; w0 += blockDim.x) {
+        const int64_t wi = w0 + threadIdx.x;
+        uint32_t word = 0;
+        if (wi < nwords)
+            for (int y = 0; y < b.n_gl; ++y) word |= kb[lane_of(b, s, g, y) * W + wi];
+        if (wi == 0) has0 = word & 1u;
+        int total;
+        const int excl = block_excl_scan<int>(__popc(word), red, total);
+        int k = base + excl;
+        while (word) {
+            const int bit = __ffs(word) - 1;
+            word &= word - 1;
+            out[k++] = (int32_t)(wi * 32 + bit);
+        }
+        base += total;
+    }
+    if (threadIdx.x == 0) w.ucount[grp] = base;
+    if (mode == 1 && threadIdx.x == 0) {
+        // attended tokens of the group: sink + kept chunks (token 0 once) + tail
+        const int64_t tail = sq.N - sq.T * sq.top;
+        atomicAdd(&w.ctr[kCtrUnionTokens],
+                  (unsigned long long)(tail + 1 + (int64_t)base * sq.C - (has0 ? 1 : 0)));
+    }
+}
+
+// ----------------------------------------------------------------------------- score
+
+// Warp = 8 lanes x 4 quarter-threads; thread (lane, quarter) keeps its lane's query
+// dimensions {16 i + 4 quarter + c} in registers.  WB warps split a block of 8*WB lanes,
+// 8/WB node slots run concurrently.  Each node record is read with 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float scale) {
+    const int grp = blockIdx.z;
+    const int s = grp / b.Hkv, g = grp % b.Hkv;
+    const SeqDev& sq = b.seqs[s];
+    const int lev = sq.L - it;
+    if (lev < 1) return;
+    const bool top = (lev == sq.L);
+    const int C = sq.C;
+    const int64_t nc = top ? sq.T : (int64_t)w.ucount[grp] * C;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
+    if (nc == 0) return;
+    const int WB = min(8, (b.n_gl + 7) / 8);
+    const int NPC = 8 / WB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= WB * NPC) return;
+    const int lb = warp % WB, slot = warp / WB;
+    const int y = (blockIdx.y * WB + lb) * 8 + (lane >> 2);
+    const int q = lane & 3;
+    const bool lane_ok = y < b.n_gl;
+    const int64_t x = lane_of(b, s, g, lane_ok ? y : 0);
+
+    float qv[D / 4];
+    {
+        const uint2* p = reinterpret_cast<const uint2*>(b.Q + x * D);
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+            const uint2 u = __ldg(p + 4 * i + q);
+            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+            const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+            qv[4 * i] = a0.x; qv[4 * i + 1] = a0.y; qv[4 * i + 2] = a1.x; qv[4 * i + 3] = a1.y;
+        }
+    }
+    const int R = sq.R;
+    const int64_t ns = sq.ns;
+    const float* base = sq.rec[lev] + (int64_t)g * sq.cap[lev] * ns;
+    const int32_t* ul = w.ulist + (int64_t)grp * w.us;
+    float* ex = w.e + x * w.es;
+    for (int64_t k = (int64_t)blockIdx.x * NPC + slot; k < nc; k += (int64_t)gridDim.x * NPC) {
+        const int64_t j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
+        const float* rec = base + j * ns;
+        float best = -INFINITY;
+        for (int r = 0; r < R; ++r) {
+            const float4* row = reinterpret_cast<const float4*>(rec + (int64_t)r * D);
+            float dot = 0.0f;
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) {
+                const float4 m = __ldg(row + 4 * i + q);
+                dot = fmaf(qv[4 * i], m.x, dot);
+                dot = fmaf(qv[4 * i + 1], m.y, dot);
+                dot = fmaf(qv[4 * i + 2], m.z, dot);
+                dot = fmaf(qv[4 * i + 3], m.w, dot);
+            }
+            dot += __shfl_xor_sync(kFull, dot, 1);
+            dot += __shfl_xor_sync(kFull, dot, 2);
+            best = fmaxf(best, fmaf(scale, dot, __ldg(rec + (int64_t)R * D + r)));
+        }
+        if (lane_ok && q == 0) ex[j] = best;
+    }
+}
+
+// ----------------------------------------------------------------------------- select
+
+constexpr int kSelThreads = 512;
+constexpr int kNB = 4096;            // bins over (max e - e) * kBinScale
+constexpr float kBinScale = 128.0f;
+constexpr int kCap = 4096;           // boundary-bin candidates sorted in shared memory
+constexpr float kMassScale = 1099511627776.0f;   // 2^40: fixed-point masses, exact sums (<= 2^24 candidates)
+
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o ^ 0x80000000u) : ~o);
+}
+// Ascending key order == (e descending, node index ascending).
+__device__ __forceinline__ unsigned long long sel_key(float e, int64_t j) {
+    return ((unsigned long long)(~ord_f32(e)) << 32) | (unsigned long long)(uint32_t)j;
+}
+__device__ __forceinline__ float key_score(unsigned long long k) {
+    return unord_f32(~(uint32_t)(k >> 32));
+}
+__device__ __forceinline__ unsigned long long mass_of(float e, float M) {
+    return (unsigned long long)(expf(e - M) * kMassScale);
+}
+__device__ __forceinline__ int bin_of(float e, float M) {
+    const float t = (M - e) * kBinScale;
+    return t >= (float)(kNB - 1) ? kNB - 1 : (int)t;
+}
+
+__global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it) {
+    extern __shared__ unsigned long long sel_smem[];
+    unsigned long long* hist = sel_smem;                                    // [kNB]
+    unsigned long long* keys = hist + kNB;                                  // [kCap]
+    unsigned int* hcnt = reinterpret_cast<unsigned int*>(keys + kCap);      // [kNB]
+    __shared__ unsigned long long red_u[33];
+    __shared__ float red_f[33];
+    __shared__ int s_bstar;
+    __shared__ unsigned long long s_cumb, s_kstar;
+    __shared__ unsigned int s_nkeys;
+
+    const int64_t x = blockIdx.x;
+    const int s = (int)(x / ((int64_t)b.n_q * b.Hq));
+    const int h = (int)(x % b.Hq);
+    const SeqDev& sq = b.seqs[s];
+    const int lev = sq.L - it;
+    if (lev < 1) return;
+    const int64_t nl = sq.n[lev];
+    int32_t* kcount = w.kcount + (int64_t)lev * w.lanes_cap + x;
+    if (nl == 0) {
+        if (threadIdx.x == 0) *kcount = 0;
+        return;
+    }
+    (void)h;
+    const bool top = (lev == sq.L);
+    const int64_t C = sq.C;
+    const uint32_t* P = top ? nullptr : w.kept[lev + 1] + x * w.W[lev + 1];
+    const float* e = w.e + x * w.es;
+    uint32_t* outw = w.kept[lev] + x * w.W[lev];
+    const int64_t nwords = (nl + 31) / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+
+    const int64_t np1 = top ? 0 : sq.n[lev + 1];   // complete parents
+    auto valid_at = [&](int64_t j) -> bool {
+        if (j >= nl) return false;
+        if (top) return true;
+        const int64_t pj = j / C;
+        if (pj >= np1) return false;                 // child of an incomplete parent
+        return (__ldg(P + (pj >> 5)) >> (pj & 31)) & 1u;
+    };
+
+    // pass 1: frontier max and size
+    float mloc = -INFINITY;
+    unsigned long long floc = 0;
+    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+        const int64_t j = wi * 32 + lane;
+        if (valid_at(j)) {
+            mloc = fmaxf(mloc, e[j]);
+            ++floc;
+        }
+    }
+    const float M = block_max(mloc, red_f);
+    const unsigned long long F = block_sum<unsigned long long>(floc, red_u);
+    if (threadIdx.x == 0) atomicAdd(&w.ctr[kCtrLaneNodes + lev], F);
+    if (F == 0) {
+        if (threadIdx.x == 0) *kcount = 0;
+        return;
+    }
+    if (b.p >= 1.0f) {
+        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+            const unsigned bal = __ballot_sync(kFull, valid_at(wi * 32 + lane));
+            if (lane == 0) outw[wi] = bal;
+        }
+        if (threadIdx.x == 0) *kcount = (int32_t)F;
+        return;
+    }
+
+    // pass 2: fixed-point masses, total, histogram over bins of (M - e)
+    for (int i = threadIdx.x; i < kNB; i += blockDim.x) {
+        hist[i] = 0ull;
+        hcnt[i] = 0u;
+    }
+    __syncthreads();
+    unsigned long long zloc = 0;
+    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+        const int64_t j = wi * 32 + lane;
+        if (valid_at(j)) {
+            const float ev = e[j];
+            const unsigned long long u = mass_of(ev, M);
+            zloc += u;
+            const int bn = bin_of(ev, M);
+            atomicAdd(&hist[bn], u);
+            atomicAdd(&hcnt[bn], 1u);
+        }
+    }
+    const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
+    unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
+    if (target < 1ull) target = 1ull;
+    if (target > Z) target = Z;
+
+    // pass 3: boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
+    if (warp == 0) {
+        constexpr int per = kNB / 32;
+        unsigned long long ls = 0;
+        for (int k = 0; k < per; ++k) ls += hist[lane * per + k];
+        unsigned long long incl = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long t = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const unsigned long long excl = incl - ls;
+        const unsigned bal = __ballot_sync(kFull, excl < target && target <= incl);
+        const int src = bal ? __ffs(bal) - 1 : 31;
+        if (lane == src) {
+            unsigned long long cum = excl;
+            int bs = lane * per + per - 1;
+            for (int k = 0; k < per; ++k) {
+                const int bb = lane * per + k;
+                if (cum + hist[bb] >= target) {
+                    bs = bb;
+                    break;
+                }
+                cum += hist[bb];
+            }
+            s_bstar = bs;
+            s_cumb = cum;
+        }
+        if (threadIdx.x == 0) s_nkeys = 0;
+    }
+    __syncthreads();
+    const int bstar = s_bstar;
+    const unsigned long long need = target - s_cumb;
+    const unsigned nb = hcnt[bstar];
+
+    if (nb <= (unsigned)kCap) {
+        // pass 4: collect the boundary bin, sort by (e desc, j asc), find the crossing
+        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+            const int64_t j = wi * 32 + lane;
+            if (valid_at(j)) {
+                const float ev = e[j];
+                if (bin_of(ev, M) == bstar) keys[atomicAdd(&s_nkeys, 1u)] = sel_key(ev, j);
+            }
+        }
+        __syncthreads();
+        const int n = (int)s_nkeys;
+        int npow = 1;
+        while (npow < n) npow <<= 1;
+        for (int i = threadIdx.x; i < npow; i += blockDim.x)
+            if (i >= n) keys[i] = ~0ull;
+        __syncthreads();
+        for (int k = 2; k <= npow; k <<= 1) {
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int i = threadIdx.x; i < npow; i += blockDim.x) {
+                    const int ixj = i ^ jj;
+                    if (ixj > i) {
+                        const unsigned long long a0 = keys[i], a1 = keys[ixj];
+                        const bool asc = (i & k) == 0;
+                        if ((a0 > a1) == asc) {
+                            keys[i] = a1;
+                            keys[ixj] = a0;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        const int per = (n + blockDim.x - 1) / blockDim.x;
+        const int i0 = threadIdx.x * per;
+        unsigned long long run = 0;
+        for (int i = i0; i < min(n, i0 + per); ++i) run += mass_of(key_score(keys[i]), M);
+        unsigned long long tot;
+        unsigned long long cum = block_excl_scan<unsigned long long>(run, red_u, tot);
+        int found = n;
+        for (int i = i0; i < min(n, i0 + per); ++i) {
+            cum += mass_of(key_score(keys[i]), M);
+            if (cum >= need) {
+                found = i;
+                break;
+            }
+        }
+        __syncthreads();
+        found = block_min_t<int>(found, reinterpret_cast<int*>(red_f));
+        if (threadIdx.x == 0) s_kstar = keys[found < n ? found : n - 1];
+    } else {
+        // rare: too many candidates in one bin - bisection on the exact key order
+        unsigned long long klo = ~0ull, khi = 0ull;
+        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+            const int64_t j = wi * 32 + lane;
+            if (valid_at(j)) {
+                const float ev = e[j];
+                if (bin_of(ev, M) == bstar) {
+                    const unsigned long long kk = sel_key(ev, j);
+                    klo = kk < klo ? kk : klo;
+                    khi = kk > khi ? kk : khi;
+                }
+            }
+        }
+        unsigned long long lo = block_min_t<unsigned long long>(klo, red_u);
+        unsigned long long hi = block_max_t<unsigned long long>(khi, red_u);
+        int iters = 0;
+        while (lo < hi && iters < 70) {
+            const unsigned long long mid = lo + (hi - lo) / 2;
+            unsigned long long acc = 0;
+            for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+                const int64_t j = wi * 32 + lane;
+                if (valid_at(j)) {
+                    const float ev = e[j];
+                    if (bin_of(ev, M) == bstar && sel_key(ev, j) <= mid) acc += mass_of(ev, M);
+                }
+            }
+            acc = block_sum<unsigned long long>(acc, red_u);
+            if (acc >= need) hi = mid;
+            else lo = mid + 1;
+            ++iters;
+        }
+        if (threadIdx.x == 0) {
+            s_kstar = lo;
+            if (iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
+        }
+    }
+    __syncthreads();
+    const unsigned long long kstar = s_kstar;
+
+    // pass 5: kept bitmap
+    unsigned long long cnt = 0;
+    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
+        const int64_t j = wi * 32 + lane;
+        bool keep = false;
+        if (valid_at(j)) {
+            const float ev = e[j];
+            const int bn = bin_of(ev, M);
+            keep = bn < bstar || (bn == bstar && sel_key(ev, j) <= kstar);
+        }
+        const unsigned bal = __ballot_sync(kFull, keep);
+        if (lane == 0) {
+            outw[wi] = bal;
+            cnt += __popc(bal);
+        }
+    }
+    cnt = block_sum<unsigned long long>(cnt, red_u);
+    if (threadIdx.x == 0) *kcount = (int32_t)cnt;
+}
+
+int score_blocks_x(int lane_blocks, int groups) {
+    const int target = 148 * 8;
+    int nb = target / max(1, lane_blocks * groups);
+    return nb < 1 ? 1 : (nb > 65535 ? 65535 : nb);
+}
+
+}  // namespace
+
+cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaStream_t st) {
+    ProfScope ps_("k_union", st);
+    k_union<<<b.n_groups, 1024, 0, st>>>(b, w, it, mode);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
+    const int WB = min(8, (b.n_gl + 7) / 8);
+    const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
+    dim3 grid(score_blocks_x(lane_blocks, b.n_groups), lane_blocks, b.n_groups);
+    ProfScope ps_("k_score", st);
+    if (b.d == 128)
+        k_score<128><<<grid, 256, 0, st>>>(b, w, it, scale);
+    else
+        k_score<64><<<grid, 256, 0, st>>>(b, w, it, scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st) {
+    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8 + (size_t)kNB * 4;
+    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ProfScope ps_("k_select", st);
+    k_select<<<b.n_lanes, kSelThreads, smem, st>>>(b, w, it);
+    return cudaGetLastError();
+}
+
+}  // namespace zha

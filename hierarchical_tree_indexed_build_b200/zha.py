@@ -1,0 +1,315 @@
+"""ctypes binding of libzha (include/zha.h).
+
+Argument marshalling only: every step of tree build, routing and attention runs in the
+CUDA kernels of libzha.so.  Functions named ``zha_*`` mirror the C entry points one to
+one; ``Tree`` and ``Decoder`` wrap them for torch tensors (device pointers and the
+current CUDA stream).  There is no fallback: if libzha.so is missing or no CUDA device
+is present, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzha.so")
+MAX_LEVELS = 16
+
+ZHA_OK, ZHA_ERR_ARG, ZHA_ERR_CAPACITY, ZHA_ERR_CUDA, ZHA_ERR_STATE, ZHA_ERR_DEVICE = range(6)
+_STATUS = {0: "ZHA_OK", 1: "ZHA_ERR_ARG", 2: "ZHA_ERR_CAPACITY", 3: "ZHA_ERR_CUDA",
+           4: "ZHA_ERR_STATE", 5: "ZHA_ERR_DEVICE"}
+
+# Every function declared in include/zha.h.
+EXPORTS = ["zha_last_error", "zha_tree_create", "zha_tree_destroy", "zha_tree_info", "zha_build_tree",
+           "zha_append", "zha_tree_export", "zha_decoder_create", "zha_decoder_destroy", "zha_route",
+           "zha_sparse_attn", "zha_decode", "zha_decoder_export_kept", "zha_decoder_words",
+           "zha_decoder_stats", "zha_profile_enable", "zha_profile_read", "zha_profile_reset"]
+
+
+class ZhaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__("%s: %s" % (_STATUS.get(status, status), msg))
+        self.status = status
+
+
+class Geometry(ctypes.Structure):
+    _fields_ = [("C", ctypes.c_int32), ("L", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("capacity", ctypes.c_int64)]
+
+
+class DecodeStats(ctypes.Structure):
+    _fields_ = [("union_nodes", ctypes.c_int64 * MAX_LEVELS), ("lane_nodes", ctypes.c_int64 * MAX_LEVELS),
+                ("union_tokens", ctypes.c_int64), ("lane_tokens", ctypes.c_int64),
+                ("node_bytes", ctypes.c_int64), ("status", ctypes.c_int32)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+
+
+def lib() -> ctypes.CDLL:
+    """Load libzha.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libzha.so not found at %s; build it with "
+                               "hierarchical_tree_indexed_build_b200.build_ext.build()" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        L.zha_last_error.restype = ctypes.c_char_p
+        L.zha_tree_create.argtypes = [ctypes.POINTER(Geometry), ctypes.POINTER(_vp)]
+        L.zha_tree_destroy.argtypes = [_vp]
+        L.zha_tree_info.argtypes = [_vp, ctypes.POINTER(Geometry), ctypes.POINTER(_i64), ctypes.POINTER(_i64),
+                                    ctypes.POINTER(_i64)]
+        L.zha_build_tree.argtypes = [_vp, _vp, _i64, _vp, _vp]
+        L.zha_append.argtypes = [_vp, _vp, _i64, _i64, _vp]
+        L.zha_tree_export.argtypes = [_vp, _i32, _vp, _vp, _vp, _vp]
+        L.zha_decoder_create.argtypes = [ctypes.POINTER(_vp), _i32, _i32, ctypes.POINTER(_vp)]
+        L.zha_decoder_destroy.argtypes = [_vp]
+        L.zha_route.argtypes = [_vp, _vp, _i32, ctypes.c_float, _vp]
+        L.zha_sparse_attn.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, _vp, _vp]
+        L.zha_decode.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, ctypes.c_float,
+                                 _vp, _vp]
+        L.zha_decoder_export_kept.argtypes = [_vp, _i32, _vp, _vp, _vp]
+        L.zha_decoder_words.argtypes = [_vp, _i32]
+        L.zha_decoder_words.restype = _i64
+        L.zha_decoder_stats.argtypes = [_vp, ctypes.POINTER(DecodeStats), _vp]
+        L.zha_profile_enable.argtypes = [_i32]
+        L.zha_profile_read.argtypes = [ctypes.c_char_p, _i32, ctypes.POINTER(_i64),
+                                       ctypes.POINTER(ctypes.c_double), _i32]
+        L.zha_profile_read.restype = _i32
+        L.zha_profile_reset.argtypes = []
+        for name in EXPORTS:
+            if name not in ("zha_last_error", "zha_decoder_words", "zha_profile_read"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != ZHA_OK:
+        raise ZhaError(status, lib().zha_last_error().decode())
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _ptr_array(ts: Sequence[torch.Tensor]):
+    arr = (_vp * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = t.data_ptr()
+    return arr
+
+
+# ----------------------------------------------------------------------------- C names
+
+def zha_tree_create(geom: Geometry) -> int:
+    h = _vp()
+    _check(lib().zha_tree_create(ctypes.byref(geom), ctypes.byref(h)))
+    return h.value
+
+
+def zha_tree_destroy(tree: int):
+    _check(lib().zha_tree_destroy(tree))
+
+
+def zha_tree_info(tree: int):
+    g = Geometry()
+    n = _i64()
+    lv = (_i64 * MAX_LEVELS)()
+    nb = _i64()
+    _check(lib().zha_tree_info(tree, ctypes.byref(g), ctypes.byref(n), lv, ctypes.byref(nb)))
+    return g, n.value, list(lv)[:g.L], nb.value
+
+
+def zha_build_tree(tree: int, K: int, n_tokens: int, q_ref: int, stream: int):
+    _check(lib().zha_build_tree(tree, K, n_tokens, q_ref, stream))
+
+
+def zha_append(tree: int, K: int, n_old: int, n_new: int, stream: int):
+    _check(lib().zha_append(tree, K, n_old, n_new, stream))
+
+
+def zha_tree_export(tree: int, level: int, m: Optional[int], lse: Optional[int], b: Optional[int], stream: int):
+    _check(lib().zha_tree_export(tree, level, m, lse, b, stream))
+
+
+def zha_decoder_create(trees: Sequence[int], max_queries: int) -> int:
+    arr = (_vp * len(trees))(*trees)
+    h = _vp()
+    _check(lib().zha_decoder_create(arr, len(trees), max_queries, ctypes.byref(h)))
+    return h.value
+
+
+def zha_decoder_destroy(dec: int):
+    _check(lib().zha_decoder_destroy(dec))
+
+
+def zha_route(dec: int, Q: int, n_q: int, p: float, stream: int):
+    _check(lib().zha_route(dec, Q, n_q, p, stream))
+
+
+def zha_sparse_attn(dec: int, K, V, Q: int, n_q: int, out: int, stream: int):
+    _check(lib().zha_sparse_attn(dec, K, V, Q, n_q, out, stream))
+
+
+def zha_decode(dec: int, K, V, Q: int, n_q: int, p: float, out: int, stream: int):
+    _check(lib().zha_decode(dec, K, V, Q, n_q, p, out, stream))
+
+
+def zha_decoder_export_kept(dec: int, level: int, bits: int, counts: Optional[int], stream: int):
+    _check(lib().zha_decoder_export_kept(dec, level, bits, counts, stream))
+
+
+def zha_decoder_words(dec: int, level: int) -> int:
+    return lib().zha_decoder_words(dec, level)
+
+
+def zha_decoder_stats(dec: int, stream: int) -> DecodeStats:
+    st = DecodeStats()
+    _check(lib().zha_decoder_stats(dec, ctypes.byref(st), stream))
+    return st
+
+
+def zha_profile_enable(on: bool):
+    _check(lib().zha_profile_enable(1 if on else 0))
+
+
+def zha_profile_reset():
+    _check(lib().zha_profile_reset())
+
+
+def zha_profile_read(max_kernels: int = 32, name_len: int = 64):
+    """{kernel name: (launches, total device ms)} of the recorded launches."""
+    names = ctypes.create_string_buffer(max_kernels * name_len)
+    launches = (_i64 * max_kernels)()
+    total = (ctypes.c_double * max_kernels)()
+    n = lib().zha_profile_read(names, name_len, launches, total, max_kernels)
+    out = {}
+    for k in range(min(n, max_kernels)):
+        nm = names.raw[k * name_len:(k + 1) * name_len].split(b"\0", 1)[0].decode()
+        out[nm] = (int(launches[k]), float(total[k]))
+    return out
+
+
+# ----------------------------------------------------------------------------- tensors
+
+def _need(t: torch.Tensor, dtype, what: str):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous CUDA %s tensor" % (what, dtype))
+
+
+class Tree:
+    """A summary tree over one sequence's KV cache (device memory owned by libzha)."""
+
+    def __init__(self, C: int, L: int, R: int, d: int, n_q_heads: int, n_kv_heads: int, capacity: int):
+        self.geom = Geometry(C, L, R, d, n_q_heads, n_kv_heads, capacity)
+        self.handle = zha_tree_create(self.geom)
+
+    def close(self):
+        if self.handle:
+            zha_tree_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def n_tokens(self) -> int:
+        return zha_tree_info(self.handle)[1]
+
+    def level_nodes(self) -> List[int]:
+        return zha_tree_info(self.handle)[2]
+
+    def build(self, K: torch.Tensor, n_tokens: int, q_ref: torch.Tensor, stream=None):
+        _need(K, torch.bfloat16, "K")
+        _need(q_ref, torch.bfloat16, "q_ref")
+        zha_build_tree(self.handle, K.data_ptr(), n_tokens, q_ref.data_ptr(), _stream(stream))
+
+    def append(self, K: torch.Tensor, n_old: int, n_new: int, stream=None):
+        _need(K, torch.bfloat16, "K")
+        zha_append(self.handle, K.data_ptr(), n_old, n_new, _stream(stream))
+
+    def export(self, level: int, stream=None):
+        g = self.geom
+        nl = self.level_nodes()[level - 1]
+        dev = torch.device("cuda", torch.cuda.current_device())
+        m = torch.empty((g.n_kv_heads, nl, g.R, g.d), dtype=torch.float32, device=dev)
+        lse = torch.empty((g.n_kv_heads, nl, g.R), dtype=torch.float32, device=dev)
+        b = torch.empty((g.n_kv_heads, nl, g.R), dtype=torch.float32, device=dev)
+        zha_tree_export(self.handle, level, m.data_ptr(), lse.data_ptr(), b.data_ptr(), _stream(stream))
+        return m, lse, b
+
+
+class Decoder:
+    """Routing + attention workspace for a batch of trees."""
+
+    def __init__(self, trees: Sequence[Tree], max_queries: int):
+        self.trees = list(trees)
+        self.handle = zha_decoder_create([t.handle for t in self.trees], max_queries)
+        g = self.trees[0].geom
+        self.Hq, self.Hkv, self.d = g.n_q_heads, g.n_kv_heads, g.d
+        self.n_q = None
+
+    def close(self):
+        if self.handle:
+            zha_decoder_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def route(self, Q: torch.Tensor, p: float, stream=None):
+        _need(Q, torch.bfloat16, "Q")
+        n_q = Q.shape[1]
+        zha_route(self.handle, Q.data_ptr(), n_q, p, _stream(stream))
+        self.n_q = n_q
+
+    def sparse_attn(self, Ks, Vs, Q: torch.Tensor, out: torch.Tensor, stream=None):
+        _need(out, torch.float32, "out")
+        zha_sparse_attn(self.handle, _ptr_array(Ks), _ptr_array(Vs), Q.data_ptr(), Q.shape[1], out.data_ptr(),
+                        _stream(stream))
+
+    def decode(self, Ks, Vs, Q: torch.Tensor, p: float, out: Optional[torch.Tensor] = None, stream=None):
+        _need(Q, torch.bfloat16, "Q")
+        if out is None:
+            out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+        _need(out, torch.float32, "out")
+        zha_decode(self.handle, _ptr_array(Ks), _ptr_array(Vs), Q.data_ptr(), Q.shape[1], p, out.data_ptr(),
+                   _stream(stream))
+        self.n_q = Q.shape[1]
+        return out
+
+    def words(self, level: int) -> int:
+        return zha_decoder_words(self.handle, level)
+
+    def export_kept(self, level: int, stream=None):
+        """Kept bitmaps (int32 view of uint32 words) [n_lanes][words] and counts [n_lanes]."""
+        n_lanes = len(self.trees) * self.n_q * self.Hq
+        W = self.words(level)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        bits = torch.empty((n_lanes, W), dtype=torch.int32, device=dev)
+        counts = torch.empty((n_lanes,), dtype=torch.int32, device=dev)
+        zha_decoder_export_kept(self.handle, level, bits.data_ptr(), counts.data_ptr(), _stream(stream))
+        return bits, counts
+
+    def stats(self, stream=None) -> DecodeStats:
+        return zha_decoder_stats(self.handle, _stream(stream))

@@ -1,0 +1,177 @@
+/*
+ * zha.h - C ABI of libzha: B200 (sm_100a) tree build and tree-routed sparse decode for
+ * Zyphra Hierarchical Attention (ZHA).
+ *
+ * What the operations compute (pages cited by title and section):
+ *  - Tree build: "Zyphra ZHA 稀疏注意力：8.2 万参数与 373 倍加速推算" (fluxbbs.com),
+ *    section "树形索引是怎么搭的"; "Zyphra发布层级注意力ZHA：稀疏搜索实现亚二次复杂度"
+ *    (wqu.guru), section "Building the tree".  Keys are cut into contiguous chunks of C
+ *    tokens; for each of R reference queries q_r a chunk is summarised by the tangent
+ *    plane of its log attention mass at q_r: lse_r = log sum_t exp(s q_r.k_t) and slope
+ *    m_r = softmax-weighted mean of the keys (s = 1/sqrt(d)); b_r = lse_r - s q_r.m_r.
+ *    Summaries are compressed again level by level: a level-l node covers C^l tokens;
+ *    this library merges the C children's (lse_r, m_r) with the online-softmax combine,
+ *    which equals the summary of the C^l raw tokens.
+ *  - Routing: fluxbbs section "树形索引是怎么搭的" (解码时的路由是自顶向下的); wqu.guru
+ *    section "How does top-p routing pick tokens?".  Per query head, the complete
+ *    top-level nodes are scored by max_r (s q.m_r + b_r); at each level the smallest
+ *    (score desc, index asc) prefix of the candidates whose softmax mass over the
+ *    candidates reaches p is kept, and only the kept nodes' children are scored next.
+ *  - Sparse attention: fluxbbs (只对少量保留下来的原始 KV 条目做精确注意力), wqu.guru
+ *    ("The first token is always kept as an attention sink").  Exact softmax attention
+ *    over token 0, the tokens of the kept level-1 chunks and the tail of tokens after the
+ *    last complete top node.
+ *
+ * Conventions
+ *  - Every device pointer is a CUDA device address on the current device; the caller
+ *    owns K, V, Q, q_ref and output buffers.  The library owns tree storage and decode
+ *    workspace (allocated at create time, freed at destroy time).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is enqueued
+ *    asynchronously on it; functions do not synchronise unless stated.
+ *  - bf16 means IEEE bfloat16 bit patterns (uint16); f32 outputs are IEEE binary32.
+ *  - Device pointers must be 16-byte aligned.
+ *  - Functions return a zha_status; on failure nothing was enqueued, and
+ *    zha_last_error() returns a message for the calling thread.  No exception crosses
+ *    the ABI.  Objects are not thread-safe; use one thread per object at a time.
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZHA_MAX_LEVELS 16
+
+typedef enum zha_status {
+    ZHA_OK = 0,
+    ZHA_ERR_ARG = 1,       /* null/misaligned pointer, bad size or geometry */
+    ZHA_ERR_CAPACITY = 2,  /* a size exceeds what the object was created for */
+    ZHA_ERR_CUDA = 3,      /* a CUDA runtime call failed (message in zha_last_error) */
+    ZHA_ERR_STATE = 4,     /* call out of order (append before build, n_old mismatch, ...) */
+    ZHA_ERR_DEVICE = 5     /* a kernel flagged an internal failure in the device status word */
+} zha_status;
+
+/* Tree geometry and the shape of the KV cache it indexes. */
+typedef struct zha_geometry {
+    int32_t C;            /* children per node = tokens per level-1 chunk, 2..1024 */
+    int32_t L;            /* levels, 1..ZHA_MAX_LEVELS; a top node covers C^L tokens */
+    int32_t R;            /* reference queries per KV head: 1, 2, 4, 8, 16 or 32 */
+    int32_t d;            /* head dimension: 64 or 128 */
+    int32_t n_q_heads;    /* query heads Hq (multiple of n_kv_heads) */
+    int32_t n_kv_heads;   /* KV heads Hkv; query head h reads KV head h*Hkv/Hq */
+    int64_t capacity;     /* rows per KV head of the K/V buffers (max tokens) */
+} zha_geometry;
+
+typedef struct zha_tree zha_tree;        /* per-sequence summary tree (device memory) */
+typedef struct zha_decoder zha_decoder;  /* routing + attention workspace for a batch of trees */
+
+/* Message for the last failed call on this thread ("" if none).  Never NULL. */
+const char* zha_last_error(void);
+
+/* ------------------------------------------------------------------ tree */
+
+/* Allocates the tree for `g` (levels 1..L at capacity: node records of R*(d+1) f32
+ * rounded up to 8 floats, plus lse [R] f32 per node, plus q_ref).  *out receives the
+ * handle.  ZHA_ERR_ARG on invalid geometry, ZHA_ERR_CUDA on allocation failure. */
+zha_status zha_tree_create(const zha_geometry* g, zha_tree** out);
+
+/* Frees the tree (synchronises the device first).  NULL is accepted. */
+zha_status zha_tree_destroy(zha_tree* t);
+
+/* Geometry, current token count, complete nodes per level (level_nodes[l-1] = n_tokens
+ * / C^l, array of L entries, nullable) and device bytes held (nullable). Host only. */
+zha_status zha_tree_info(const zha_tree* t, zha_geometry* g, int64_t* n_tokens,
+                         int64_t* level_nodes, int64_t* device_bytes);
+
+/* Builds every complete node of levels 1..L over the first n_tokens rows of K.
+ *   K      bf16 [n_kv_heads][capacity][d] (device), row t of head g at (g*capacity+t)*d
+ *   q_ref  bf16 [n_kv_heads][R][d] (device), copied into the tree (used by append too)
+ * 0 <= n_tokens <= capacity, else ZHA_ERR_CAPACITY. */
+zha_status zha_build_tree(zha_tree* t, const void* K, int64_t n_tokens, const void* q_ref,
+                          void* stream);
+
+/* Grows the tree by n_new tokens whose keys are already in K rows [n_old, n_old+n_new):
+ * summarises the chunks these tokens complete and merges every ancestor that becomes
+ * complete.  n_old must equal the tree's token count (ZHA_ERR_STATE otherwise, also
+ * before the first build); n_old + n_new <= capacity (ZHA_ERR_CAPACITY). */
+zha_status zha_append(zha_tree* t, const void* K, int64_t n_old, int64_t n_new, void* stream);
+
+/* Copies level `level` (1..L) summaries of all KV heads into device buffers:
+ *   m [n_kv_heads][n_l][R][d], lse [n_kv_heads][n_l][R], b [n_kv_heads][n_l][R]  (f32)
+ * with n_l = level_nodes[level-1].  Any pointer may be NULL to skip that array. */
+zha_status zha_tree_export(const zha_tree* t, int32_t level, float* m, float* lse, float* b,
+                           void* stream);
+
+/* ------------------------------------------------------------------ decode */
+
+/* Creates a decoder for a batch of n_seq trees (same d, Hq, Hkv; C, L, R may differ per
+ * tree) and up to max_queries query tokens per sequence per call.  Workspace is sized
+ * from the trees' capacities; trees must outlive the decoder. */
+zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n_seq, int32_t max_queries,
+                              zha_decoder** out);
+zha_status zha_decoder_destroy(zha_decoder* dec);
+
+/* Routing for n_q query tokens per sequence.
+ *   Q  bf16 [n_seq][n_q][Hq][d] (device).
+ *   p  top-p mass, 0 < p <= 1 (p >= 1 keeps every node).
+ * Lane x = (s*n_q + i)*Hq + h.  Kept sets of every level stay in the decoder (see
+ * zha_decoder_export_kept).  Uses each tree's current token count. */
+zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream);
+
+/* Exact attention of the routed lanes over token 0, the kept level-1 chunks and the tail.
+ *   K, V  arrays of n_seq device pointers, bf16 [n_kv_heads][capacity][d] each
+ *   Q     the same buffer given to zha_route
+ *   out   f32 [n_seq][n_q][Hq][d] (device). */
+zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
+                           const void* Q, int32_t n_q, float* out, void* stream);
+
+/* zha_route followed by zha_sparse_attn. */
+zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
+                      const void* Q, int32_t n_q, float p, float* out, void* stream);
+
+/* Kept sets of the last zha_route at `level` (1..max L of the batch), as bitmaps:
+ *   bits   uint32 [n_lanes][words] (device), bit j of lane x set iff node j kept;
+ *          words = zha_decoder_words(dec, level); lanes whose tree has fewer levels
+ *          get all-zero rows
+ *   counts int32 [n_lanes] (device, nullable): kept nodes per lane. */
+zha_status zha_decoder_export_kept(const zha_decoder* dec, int32_t level, uint32_t* bits,
+                                   int32_t* counts, void* stream);
+int64_t zha_decoder_words(const zha_decoder* dec, int32_t level);
+
+/* Work counters of the last zha_route / zha_sparse_attn (synchronises `stream`):
+ * nodes scored per level as the union over each (sequence, KV head) group of lanes and
+ * as the per-lane sum, attended tokens (union per group and per-lane sum), and the
+ * device status word (0 = ok). */
+typedef struct zha_decode_stats {
+    int64_t union_nodes[ZHA_MAX_LEVELS];      /* index l-1 */
+    int64_t lane_nodes[ZHA_MAX_LEVELS];
+    int64_t union_tokens;
+    int64_t lane_tokens;
+    int64_t node_bytes;                       /* bytes read per scored node (m and b, f32) */
+    int32_t status;
+} zha_decode_stats;
+zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats* out, void* stream);
+
+
+/* ------------------------------------------------------------------ profile */
+
+/* Device-time profile of this library's own kernels (off by default; not part of the
+ * method).  While enabled, every kernel launch is bracketed by two CUDA events recorded
+ * on its launch stream (so launches must not be under stream capture).
+ * zha_profile_read synchronises the device, sums the recorded intervals per kernel and
+ * returns the number of distinct kernels seen; at most max_kernels entries are written:
+ *   names     char [max_kernels][name_len] (host), NUL-terminated kernel names
+ *   launches  int64 [max_kernels] (host);  total_ms  double [max_kernels] (host).
+ * Any output pointer may be NULL.  zha_profile_reset drops the recorded intervals. */
+zha_status zha_profile_enable(int32_t on);
+int32_t zha_profile_read(char* names, int32_t name_len, int64_t* launches, double* total_ms,
+                         int32_t max_kernels);
+zha_status zha_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZHA_H */

@@ -1,0 +1,232 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on the same
+seeded inputs.  Small cases run every lane; full-size cases run the batch the benchmark
+times and compare sampled lanes."""
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_tree_indexed_build_b200 import inputs, zha
+from oracle import oracle as O
+import zha_testlib as TL
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _report(name, rep, e1, e2):
+    print("[%s] levels=%d exact=%d mass_ties=%d score_ties=%d  out/own max=%.2e  out/e2e max=%s"
+          % (name, rep.levels, rep.exact, rep.mass_ties, rep.score_ties, e1.max(),
+             "%.2e" % e2.max() if e2.size else "-"))
+
+
+# ----------------------------------------------------------------------------- build
+
+@needs_cuda
+@pytest.mark.parametrize("geom,n_tokens", [
+    (inputs.TINY, 4096),                 # the tiny workload's tree
+    (inputs.TINY, 4096 + 77),            # ragged: incomplete chunk and nodes at the end
+    (inputs.DEEP, 3 * 4096 + 1234),      # C4 L6, ragged
+    (inputs.MID, 2 * 4096 + 700),        # C16 L3, ragged
+    (inputs.WIDE, 256 * 40 + 100),       # C256 L1, ragged
+])
+def test_build_summaries_match_oracle(geom, n_tokens):
+    seq = inputs.make_sequence(geom, n_tokens, n_tokens, seed=11)
+    tree, K, V, qr = TL.make_tree(seq)
+    w = TL.compare_summaries(tree, seq, n_tokens)
+    print("[build %s N=%d] worst lse %.2e m %.2e b %.2e" % (geom, n_tokens, w["lse"], w["m"], w["b"]))
+    assert w["lse"] <= TL.SUM_TOL and w["m"] <= TL.SUM_TOL and w["b"] <= TL.SUM_TOL
+
+
+@needs_cuda
+def test_build_deep64k_all_nodes():
+    wl = inputs.deep_64k()
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    w = TL.compare_summaries(tree, seq, seq.n_tokens)
+    print("[build deep64k] worst", w)
+    assert max(w.values()) <= TL.SUM_TOL
+
+
+@needs_cuda
+@pytest.mark.parametrize("geom", [inputs.DEEP, inputs.MID, inputs.WIDE, inputs.TINY])
+def test_append_is_bit_identical_to_rebuild(geom):
+    """Growing a tree by appends (single tokens, then a bulk range) gives exactly the
+    summaries of a tree built over the final length in one pass."""
+    n0, singles, bulk = 4096 * 2 + 13, 70, 4096 + 501
+    cap = n0 + singles + bulk
+    seq = inputs.make_sequence(geom, cap, cap, seed=5)
+    K = seq.K.cuda(); qr = seq.qref.cuda()
+    g = geom
+    grown = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, cap)
+    grown.build(K, n0, qr)
+    n = n0
+    for _ in range(singles):
+        grown.append(K, n, 1)
+        n += 1
+    grown.append(K, n, bulk)
+    n += bulk
+    once = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, cap)
+    once.build(K, n, qr)
+    assert grown.n_tokens == once.n_tokens == cap
+    for lev in range(1, g.L + 1):
+        if grown.level_nodes()[lev - 1] == 0:
+            continue
+        a, b = grown.export(lev), once.export(lev)
+        for x, y in zip(a, b):
+            assert torch.equal(x, y), lev
+
+
+# ----------------------------------------------------------------------------- decode
+
+@needs_cuda
+@pytest.mark.parametrize("p", [0.9, 1.0, 0.5])
+def test_decode_tiny(p):
+    wl = inputs.tiny_4k()
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0]                                   # [1][16][1][64]
+    res = TL.gpu_decode([tree], [K], [V], Q, p)
+    rep, e1, e2, toks = TL.check_decode(seq, seq.n_tokens, Q[0], p, res.out[0], res.kept[0], range(16))
+    _report("tiny p=%g" % p, rep, e1, e2)
+    if p == 1.0:
+        assert all(t.size == seq.n_tokens for t in toks)
+        dense = O.attend_batch(TL.f64(seq.K), TL.f64(seq.V), TL.lanes_for(seq, Q[0], range(16))[0],
+                               np.zeros(16, np.int32), [np.arange(seq.n_tokens)] * 16)
+        assert TL.rel_err(res.out[0].reshape(16, -1), dense).max() <= TL.OUT_TOL
+    # sink always attended; per-lane token counts match the stats
+    assert all(t[0] == 0 for t in toks)
+    assert res.stats.lane_tokens == sum(t.size for t in toks)
+
+
+@needs_cuda
+def test_decode_deep_ragged_tail():
+    """C4 L6 with 4 complete top nodes and a 1,500-token dense tail, 16 queries."""
+    n = 4 * 4096 + 1500
+    seq = inputs.make_sequence(inputs.DEEP, n, n, seed=21)
+    rq = np.random.default_rng(3)
+    Q, _ = inputs.make_queries(seq, 16, 8, n, rq)
+    tree, K, V, qr = TL.make_tree(seq)
+    res = TL.gpu_decode([tree], [K], [V], Q[None], 0.95)
+    rep, e1, e2, toks = TL.check_decode(seq, n, Q, 0.95, res.out[0], res.kept[0], range(16))
+    _report("deep ragged", rep, e1, e2)
+    assert all(np.all(t[-1500:] == np.arange(n - 1500, n)) for t in toks)
+
+
+@needs_cuda
+def test_decode_no_complete_top_node_is_dense():
+    n = 4000                                     # < 4096 = C^L: no top node, A = [0, N)
+    seq = inputs.make_sequence(inputs.DEEP, n, n, seed=2)
+    Q, _ = inputs.make_queries(seq, 2, 8, n, np.random.default_rng(0))
+    tree, K, V, qr = TL.make_tree(seq)
+    res = TL.gpu_decode([tree], [K], [V], Q[None], 0.95)
+    q, lane_g, ids = TL.lanes_for(seq, Q, range(2))
+    dense = O.attend_batch(TL.f64(seq.K), TL.f64(seq.V), q, lane_g, [np.arange(n)] * len(ids))
+    assert TL.rel_err(res.out[0].reshape(-1, 128)[ids], dense).max() <= TL.OUT_TOL
+
+
+@needs_cuda
+def test_decode_deep64k_full_batch():
+    """The 64K deep workload: all 64 queries routed in one batch, 16 compared lane by lane."""
+    wl = inputs.deep_64k()
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0]
+    res = TL.gpu_decode([tree], [K], [V], Q, 0.95)
+    rep, e1, e2, _ = TL.check_decode(seq, seq.n_tokens, Q[0], 0.95, res.out[0], res.kept[0], range(0, 64, 4))
+    _report("deep64k", rep, e1, e2)
+
+
+@needs_cuda
+def test_decode_wide256k():
+    wl = inputs.wide_256k()
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0]
+    res = TL.gpu_decode([tree], [K], [V], Q, 0.95)
+    rep, e1, e2, _ = TL.check_decode(seq, seq.n_tokens, Q[0], 0.95, res.out[0], res.kept[0], [0, 9, 31, 63])
+    _report("wide256k", rep, e1, e2)
+
+
+@needs_cuda
+@pytest.mark.parametrize("p", [0.7, 0.9, 0.99])
+def test_decode_deep_p_sweep(p):
+    n = 32 * 4096 + 333
+    seq = inputs.make_sequence(inputs.DEEP, n, n, seed=31)
+    Q, _ = inputs.make_queries(seq, 8, 8, n, np.random.default_rng(1))
+    tree, K, V, qr = TL.make_tree(seq)
+    res = TL.gpu_decode([tree], [K], [V], Q[None], p)
+    rep, e1, e2, _ = TL.check_decode(seq, n, Q, p, res.out[0], res.kept[0], range(8))
+    _report("deep128k p=%g" % p, rep, e1, e2)
+
+
+@needs_cuda
+def test_decode_batched_mixed_geometries_with_appends():
+    """8 sequences (4 x C16 L3, 4 x C4 L6), ragged lengths, 3 decode steps each preceded
+    by a one-token append; every lane compared."""
+    seqs = []
+    for s in range(8):
+        geom = inputs.MID if s < 4 else inputs.DEEP
+        n = 2 * 4096 + 97 * s + 5
+        seqs.append(inputs.make_sequence(geom, n, n + 3, seed=100 + s))
+    trees, Ks, Vs = [], [], []
+    for sq in seqs:
+        t, K, V, _ = TL.make_tree(sq, sq.n_tokens)
+        trees.append(t); Ks.append(K); Vs.append(V)
+    dec = zha.Decoder(trees, 1)
+    rng = np.random.default_rng(9)
+    for step in range(3):
+        Qs = []
+        for s, sq in enumerate(seqs):
+            trees[s].append(Ks[s], sq.n_tokens + step, 1)
+            q, _ = inputs.make_queries(sq, 1, 8, sq.n_tokens + step + 1, rng)
+            Qs.append(q)
+        Q = torch.stack(Qs)                      # [8][1][16][128]
+        res = TL.gpu_decode(trees, Ks, Vs, Q, 0.95, dec=dec)
+        for s, sq in enumerate(seqs):
+            rep, e1, e2, _ = TL.check_decode(sq, sq.n_tokens + step + 1, Q[s], 0.95, res.out[s], res.kept[s], [0])
+            _report("batched step %d seq %d" % (step, s), rep, e1, e2)
+
+
+@needs_cuda
+def test_decode_is_deterministic():
+    wl = inputs.deep_64k(n_q=8)
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    a = TL.gpu_decode([tree], [K], [V], wl.Q[0], 0.95)
+    b = TL.gpu_decode([tree], [K], [V], wl.Q[0], 0.95)
+    assert np.array_equal(a.out, b.out)
+    for x, y in zip(a.kept[0], b.kept[0]):
+        assert np.array_equal(x, y)
+
+
+@needs_cuda
+def test_error_paths_on_device():
+    seq = inputs.make_sequence(inputs.DEEP, 5000, 5000, seed=1)
+    K = seq.K.cuda(); qr = seq.qref.cuda()
+    g = inputs.DEEP
+    t = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, 5000)
+    with pytest.raises(zha.ZhaError) as ei:
+        t.append(K, 0, 10)                        # before build
+    assert ei.value.status == zha.ZHA_ERR_STATE
+    t.build(K, 4000, qr)
+    with pytest.raises(zha.ZhaError) as ei:
+        t.append(K, 3999, 1)                      # wrong n_old
+    assert ei.value.status == zha.ZHA_ERR_STATE
+    with pytest.raises(zha.ZhaError) as ei:
+        t.append(K, 4000, 1001)                   # past capacity
+    assert ei.value.status == zha.ZHA_ERR_CAPACITY
+    with pytest.raises(zha.ZhaError) as ei:
+        t.build(K, 5001, qr)
+    assert ei.value.status == zha.ZHA_ERR_CAPACITY
+    dec = zha.Decoder([t], 2)
+    Q = torch.zeros((1, 3, 16, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.route(Q, 0.9)                         # more queries than the decoder holds
+    assert ei.value.status == zha.ZHA_ERR_CAPACITY
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.route(Q[:, :2].contiguous(), 0.0)     # p must be > 0
+    assert ei.value.status == zha.ZHA_ERR_ARG
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.sparse_attn([K], [K], Q[:, :1].contiguous(), torch.zeros((1, 1, 16, 128), device="cuda"))
+    assert ei.value.status == zha.ZHA_ERR_STATE   # attention before routing
