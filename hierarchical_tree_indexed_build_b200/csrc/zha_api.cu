@@ -67,6 +67,8 @@ struct zha_decoder {
     size_t bytes;
     int32_t last_n_q;
     bool routed;
+    int32_t score_path;
+    int32_t all_r16;
 };
 
 extern "C" const char* zha_last_error(void) { return g_err.c_str(); }
@@ -311,6 +313,9 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     dec->groups_cap = (int64_t)n_seq * dec->Hkv;
     dec->last_n_q = 0;
     dec->routed = false;
+    dec->score_path = ZHA_SCORE_AUTO;
+    dec->all_r16 = 1;
+    for (auto* t : dec->trees) dec->all_r16 &= (t->g.R == 16) ? 1 : 0;
 
     Work& w = dec->w;
     memset(&w, 0, sizeof(w));
@@ -426,6 +431,8 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     b.n_groups = dec->n_seq * dec->Hkv;
     b.Q = static_cast<const __nv_bfloat16*>(Q);
     b.p = p;
+    b.score_path = dec->score_path;
+    b.all_r16 = dec->all_r16;
     return b;
 }
 
@@ -489,6 +496,16 @@ extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const v
     zha_status s = zha_route(dec, Q, n_q, p, stream);
     if (s != ZHA_OK) return s;
     return zha_sparse_attn(dec, K, V, Q, n_q, out, stream);
+}
+
+extern "C" zha_status zha_decoder_set_score_path(zha_decoder* dec, int32_t path) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (path != ZHA_SCORE_AUTO && path != ZHA_SCORE_SIMT && path != ZHA_SCORE_TENSOR)
+        return fail(ZHA_ERR_ARG, "unknown score path");
+    if (path == ZHA_SCORE_TENSOR && !dec->all_r16)
+        return fail(ZHA_ERR_ARG, "the tensor-core scorer needs R = 16 in every tree");
+    dec->score_path = path;
+    return ZHA_OK;
 }
 
 extern "C" int64_t zha_decoder_words(const zha_decoder* dec, int32_t level) {

@@ -62,6 +62,8 @@ struct Batch {
     int32_t n_lanes, n_groups;
     const __nv_bfloat16* Q;          // [n_seq][n_q][Hq][d]
     float p;
+    int32_t score_path;              // 0 auto, 1 CUDA cores, 2 tensor cores (R = 16 only)
+    int32_t all_r16;                 // every tree of the batch has R = 16
 };
 
 // Global lane index of group lane y of group (s, g): lane = (s*n_q + i)*Hq + h.
@@ -73,6 +75,7 @@ __host__ __device__ inline int64_t lane_of(const Batch& b, int s, int g, int y) 
 // Device status bits.
 constexpr int32_t kStatusSelectFallbackLimit = 1;
 constexpr int32_t kStatusCapacity = 2;
+constexpr int32_t kStatusTimeout = 4;        // a bounded wait on the tensor-core pipeline gave up
 
 // Split size (tokens) of the attention work for a call with n_gl lanes per group.
 inline __host__ __device__ int split_tokens(int n_gl) { return n_gl <= 64 ? 1024 : 4096; }

@@ -45,6 +45,9 @@ cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st);
 // sets of level L_s - it + 1); mode 1 prepares attention (union of level-1 kept sets).
 cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaStream_t st);
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
+cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
+// Lanes per group from which the automatic choice scores on tensor cores.
+constexpr int kTensorScoreMinLanes = 64;
 cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st);
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);

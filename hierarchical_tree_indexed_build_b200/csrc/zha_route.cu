@@ -540,6 +540,8 @@ cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaSt
 }
 
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
+    const bool tc = b.all_r16 && (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
+    if (tc) return launch_score_tc(b, w, it, scale, st);
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
     dim3 grid(score_blocks_x(lane_blocks, b.n_groups), lane_blocks, b.n_groups);

@@ -128,6 +128,14 @@ zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void
 zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
                            const void* Q, int32_t n_q, float* out, void* stream);
 
+/* Which kernels compute the plane estimates (same result up to float32 rounding):
+ *   ZHA_SCORE_AUTO    tensor cores (tcgen05, tf32 hi+lo passes) when a (sequence, KV head)
+ *                     group has >= 64 lanes and every tree has R = 16, else CUDA cores
+ *   ZHA_SCORE_SIMT    CUDA cores (fp32 FMA) always
+ *   ZHA_SCORE_TENSOR  tensor cores always (ZHA_ERR_ARG unless every tree has R = 16) */
+typedef enum zha_score_path { ZHA_SCORE_AUTO = 0, ZHA_SCORE_SIMT = 1, ZHA_SCORE_TENSOR = 2 } zha_score_path;
+zha_status zha_decoder_set_score_path(zha_decoder* dec, int32_t path);
+
 /* zha_route followed by zha_sparse_attn. */
 zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                       const void* Q, int32_t n_q, float p, float* out, void* stream);

@@ -230,3 +230,40 @@ def test_error_paths_on_device():
     with pytest.raises(zha.ZhaError) as ei:
         dec.sparse_attn([K], [K], Q[:, :1].contiguous(), torch.zeros((1, 1, 16, 128), device="cuda"))
     assert ei.value.status == zha.ZHA_ERR_STATE   # attention before routing
+
+
+@needs_cuda
+@pytest.mark.parametrize("n_q", [1, 8, 64])
+def test_tensor_core_and_cuda_core_scoring_agree(n_q):
+    """The tcgen05 scorer (tf32 hi + lo passes) and the fp32 CUDA-core scorer route the
+    64K deep workload to the same kept sets (up to logged ties) and the same outputs; the
+    tensor-core result is also checked against the oracle."""
+    wl = inputs.deep_64k(n_q=n_q)
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0]
+    res = {}
+    for path in (zha.ZHA_SCORE_SIMT, zha.ZHA_SCORE_TENSOR):
+        dec = zha.Decoder([tree], n_q)
+        dec.set_score_path(path)
+        res[path] = TL.gpu_decode([tree], [K], [V], Q, 0.95, dec=dec)
+        dec.close()
+    a, b = res[zha.ZHA_SCORE_SIMT], res[zha.ZHA_SCORE_TENSOR]
+    differ = sum(int((x != y).any(axis=1).sum()) for x, y in zip(a.kept[0], b.kept[0]))
+    lanes = a.kept[0][0].shape[0]
+    print("[tc vs simt n_q=%d] lane-levels differing: %d of %d" % (n_q, differ, lanes * len(a.kept[0])))
+    assert differ <= max(1, lanes * len(a.kept[0]) // 100)
+    qs = list(range(min(n_q, 4)))
+    rep, e1, e2, _ = TL.check_decode(seq, seq.n_tokens, Q[0], 0.95, b.out[0], b.kept[0], qs)
+    _report("tensor n_q=%d" % n_q, rep, e1, e2)
+
+
+@needs_cuda
+def test_tensor_core_scoring_needs_r16():
+    n = 4096 * 2
+    seq = inputs.make_sequence(inputs.TINY, n, n, seed=3, key_mean_std=0.0)
+    tree, K, V, qr = TL.make_tree(seq)
+    dec = zha.Decoder([tree], 1)
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.set_score_path(zha.ZHA_SCORE_TENSOR)
+    assert ei.value.status == zha.ZHA_ERR_ARG
