@@ -73,6 +73,8 @@ struct zha_decoder {
 
 extern "C" const char* zha_last_error(void) { return g_err.c_str(); }
 
+zha_status zha::set_last_error(zha_status s, const char* msg) { return fail(s, msg); }
+
 // ------------------------------------------------------------------------------ tree
 
 static zha_status check_geometry(const zha_geometry* g) {

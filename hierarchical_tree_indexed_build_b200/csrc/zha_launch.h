@@ -52,4 +52,7 @@ cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);
 
+// Records the message returned by zha_last_error() on this thread; returns s.
+zha_status set_last_error(zha_status s, const char* msg);
+
 }  // namespace zha

@@ -25,7 +25,7 @@ _STATUS = {0: "ZHA_OK", 1: "ZHA_ERR_ARG", 2: "ZHA_ERR_CAPACITY", 3: "ZHA_ERR_CUD
 # Every function declared in include/zha.h.
 EXPORTS = ["zha_last_error", "zha_tree_create", "zha_tree_destroy", "zha_tree_info", "zha_build_tree",
            "zha_append", "zha_tree_export", "zha_decoder_create", "zha_decoder_destroy", "zha_route",
-           "zha_sparse_attn", "zha_decode", "zha_decoder_set_score_path", "zha_decoder_export_kept", "zha_decoder_words",
+           "zha_sparse_attn", "zha_sparse_attn_static", "zha_decode", "zha_decoder_set_score_path", "zha_decoder_export_kept", "zha_decoder_words",
            "zha_decoder_stats", "zha_profile_enable", "zha_profile_read", "zha_profile_reset"]
 
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.zha_decoder_destroy.argtypes = [_vp]
         L.zha_route.argtypes = [_vp, _vp, _i32, ctypes.c_float, _vp]
         L.zha_sparse_attn.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, _vp, _vp]
+        L.zha_sparse_attn_static.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _i32,
+                                             _vp, _i64, _vp, _vp]
         L.zha_decode.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, ctypes.c_float,
                                  _vp, _vp]
         L.zha_decoder_set_score_path.argtypes = [_vp, _i32]
@@ -164,6 +166,11 @@ def zha_route(dec: int, Q: int, n_q: int, p: float, stream: int):
 
 def zha_sparse_attn(dec: int, K, V, Q: int, n_q: int, out: int, stream: int):
     _check(lib().zha_sparse_attn(dec, K, V, Q, n_q, out, stream))
+
+
+def zha_sparse_attn_static(K: int, V: int, ld: int, n_tokens: int, C: int, L: int, Hq: int, Hkv: int, d: int,
+                           Q: int, n_q: int, kept1: int, words: int, out: int, stream: int):
+    _check(lib().zha_sparse_attn_static(K, V, ld, n_tokens, C, L, Hq, Hkv, d, Q, n_q, kept1, words, out, stream))
 
 
 def zha_decode(dec: int, K, V, Q: int, n_q: int, p: float, out: int, stream: int):

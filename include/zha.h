@@ -136,6 +136,33 @@ zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* c
 typedef enum zha_score_path { ZHA_SCORE_AUTO = 0, ZHA_SCORE_SIMT = 1, ZHA_SCORE_TENSOR = 2 } zha_score_path;
 zha_status zha_decoder_set_score_path(zha_decoder* dec, int32_t path);
 
+/* Exact attention over a routed token set that allocates no device memory.  The pages
+ * have no counterpart: this is a service for callers that cannot allocate where they
+ * attend (a process whose device memory is owned by someone else's allocator, or a
+ * latency-critical loop that must not pay for an allocation and the synchronisation it
+ * may imply).  It computes what zha_sparse_attn computes for one sequence, from the
+ * caller's buffers alone:
+ *   K, V   bf16 [Hkv][ld][d] (device); rows [0, n_tokens) are the cache
+ *   C, L   the tree geometry (chunk size; the tail starts at (n_tokens / C^L) C^L)
+ *   Q      bf16 [n_q][Hq][d] (device)
+ *   kept1  uint32 [n_q*Hq][words] (device): level-1 kept bitmaps, lane x = i*Hq + h,
+ *          e.g. from zha_decoder_export_kept(dec, 1, ...); words >= ceil(n_tokens/C/32)
+ *   out    f32 [n_q][Hq][d] (device)
+ * Working memory comes from one 16 MiB array in the library's device image, reserved on
+ * every device that loads the library until the process exits; a call needing more
+ * returns ZHA_ERR_CAPACITY with the byte count in zha_last_error() (about 11 MB for one
+ * query token of 16 heads over 1M tokens at C = 4).  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls share the array and leave their
+ * contents in it; each call clears what must start at zero, so back-to-back calls on one
+ * stream are independent, but calls that can overlap on the GPU (different streams or
+ * threads, same device) race on the array.  No cudaMalloc/cudaFree or allocating
+ * library routine is called. */
+zha_status zha_sparse_attn_static(const void* K, const void* V, int64_t ld, int64_t n_tokens,
+                                  int32_t C, int32_t L, int32_t Hq, int32_t Hkv, int32_t d,
+                                  const void* Q, int32_t n_q, const uint32_t* kept1, int64_t words,
+                                  float* out, void* stream);
+
 /* zha_route followed by zha_sparse_attn. */
 zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                       const void* Q, int32_t n_q, float p, float* out, void* stream);
