@@ -31,6 +31,7 @@ from hierarchical_tree_indexed_build_b200 import inputs  # noqa: E402
 
 METRIC = "ZHA decode queries/s at 256K & 1M ctx; achieved HBM GB/s vs peak"
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max SM clock
+TENSOR_KERNELS = {"k_score_tc": "tf32", "k_attn_tc": "bf16"}
 
 
 def parse():
@@ -52,6 +53,17 @@ def measured_peaks():
         return pk["hbm_gbs"], "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def tensor_peak(dtype):
+    """Dense tensor peak for the kernel's MMA dtype: the measured bf16 burst figure, halved
+    for tf32 (kind::tf32 runs at half the bf16 rate)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16, src = json.load(f)["bf16_tflops"], "measured"
+    except Exception:
+        bf16, src = 1590.0, "fallback"
+    return (bf16 / 2 if dtype == "tf32" else bf16), "%s bf16 %s" % (src, "x 1/2 (tf32)" if dtype == "tf32" else "")
 
 
 class Clocks:
@@ -107,11 +119,11 @@ def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
     """(bytes, flops) one launch of `name` must move/compute (per-unit figure x units),
     from the decoder's work counters of one step."""
     R, d = geom.R, geom.d
-    if name == "k_score":
+    if name in ("k_score", "k_score_tc"):
         nodes = sum(st.union_nodes)
         lane_nodes = sum(st.lane_nodes)
         return ((nodes * st.node_bytes + lane_nodes * 4) / launches, lane_nodes * R * d * 2 / launches)
-    if name == "k_attn":
+    if name in ("k_attn", "k_attn_tc"):
         return st.union_tokens * 4 * d / launches, st.lane_tokens * 4 * d / launches
     if name == "k_select":
         return sum(st.lane_nodes) * 4 / launches, 0.0
@@ -185,7 +197,15 @@ def run_ours(args, rank, world, dev):
     avg_ms = tot_ms / launches
     hbm_peak, peak_src = measured_peaks()
     intensity = nflops / nbytes if nbytes else 0.0
-    if nflops and intensity > FP32_PEAK_TFLOPS * 1e12 / (hbm_peak * 1e9):
+    if name in TENSOR_KERNELS:
+        # executed tensor work: every lane of a group is scored against every union node
+        # (resp. attends every union token); the algorithmic figure counts only each lane's
+        # own frontier (resp. attended set)
+        peak, src = tensor_peak(TENSOR_KERNELS[name])
+        ach = nflops / (avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": None, "kernel": name, "peak_source": src}
+    elif nflops and intensity > FP32_PEAK_TFLOPS * 1e12 / (hbm_peak * 1e9):
         ach = nflops / (avg_ms / 1e3) / 1e12
         roof = {"bound": "alu", "achieved": ach, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                 "frac": ach / FP32_PEAK_TFLOPS, "traffic": None, "kernel": name,
@@ -200,7 +220,8 @@ def run_ours(args, rank, world, dev):
     roof["launches"] = launches
 
     # decode-only throughput and union bytes of the decode
-    dec_ms = sum(v[1] for k, v in prof.items() if k in ("k_union", "k_score", "k_select", "k_attn", "k_combine")) / args.steps
+    dec_ms = sum(v[1] for k, v in prof.items()
+                 if k in ("k_union", "k_score", "k_score_tc", "k_select", "k_attn", "k_attn_tc", "k_combine")) / args.steps
     union_bytes = sum(st.union_nodes) * st.node_bytes + st.union_tokens * 4 * g.d
     stages = {k: round(v[1] / args.steps, 4) for k, v in sorted(prof.items())}
     res = {

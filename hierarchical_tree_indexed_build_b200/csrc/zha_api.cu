@@ -68,6 +68,7 @@ struct zha_decoder {
     int32_t last_n_q;
     bool routed;
     int32_t score_path;
+    int32_t attn_path;
     int32_t all_r16;
 };
 
@@ -315,7 +316,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     dec->groups_cap = (int64_t)n_seq * dec->Hkv;
     dec->last_n_q = 0;
     dec->routed = false;
-    dec->score_path = ZHA_SCORE_AUTO;
+    dec->score_path = ZHA_KERNELS_AUTO;
+    dec->attn_path = ZHA_KERNELS_AUTO;
     dec->all_r16 = 1;
     for (auto* t : dec->trees) dec->all_r16 &= (t->g.R == 16) ? 1 : 0;
 
@@ -434,6 +436,7 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     b.Q = static_cast<const __nv_bfloat16*>(Q);
     b.p = p;
     b.score_path = dec->score_path;
+    b.attn_path = dec->attn_path;
     b.all_r16 = dec->all_r16;
     return b;
 }
@@ -500,13 +503,14 @@ extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const v
     return zha_sparse_attn(dec, K, V, Q, n_q, out, stream);
 }
 
-extern "C" zha_status zha_decoder_set_score_path(zha_decoder* dec, int32_t path) {
+extern "C" zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, int32_t attn) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
-    if (path != ZHA_SCORE_AUTO && path != ZHA_SCORE_SIMT && path != ZHA_SCORE_TENSOR)
-        return fail(ZHA_ERR_ARG, "unknown score path");
-    if (path == ZHA_SCORE_TENSOR && !dec->all_r16)
+    auto ok = [](int32_t v) { return v == ZHA_KERNELS_AUTO || v == ZHA_KERNELS_SIMT || v == ZHA_KERNELS_TENSOR; };
+    if (!ok(score) || !ok(attn)) return fail(ZHA_ERR_ARG, "unknown kernel choice");
+    if (score == ZHA_KERNELS_TENSOR && !dec->all_r16)
         return fail(ZHA_ERR_ARG, "the tensor-core scorer needs R = 16 in every tree");
-    dec->score_path = path;
+    dec->score_path = score;
+    dec->attn_path = attn;
     return ZHA_OK;
 }
 

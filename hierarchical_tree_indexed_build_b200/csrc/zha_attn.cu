@@ -231,6 +231,8 @@ __global__ void k_combine(Batch b, Work w, float* out) {
 
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
     if (max_splits <= 0) return cudaSuccess;
+    if (b.attn_path == 2 || (b.attn_path == 0 && b.n_gl >= kTensorAttnMinLanes))
+        return launch_attn_tc(b, w, max_splits, scale, st);
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
     dim3 grid((unsigned)max_splits, lane_blocks, b.n_groups);

@@ -63,6 +63,7 @@ struct Batch {
     const __nv_bfloat16* Q;          // [n_seq][n_q][Hq][d]
     float p;
     int32_t score_path;              // 0 auto, 1 CUDA cores, 2 tensor cores (R = 16 only)
+    int32_t attn_path;               // 0 auto, 1 CUDA cores, 2 tensor cores
     int32_t all_r16;                 // every tree of the batch has R = 16
 };
 

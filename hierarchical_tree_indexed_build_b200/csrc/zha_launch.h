@@ -50,6 +50,9 @@ cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, 
 constexpr int kTensorScoreMinLanes = 64;
 cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st);
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
+cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
+// Lanes per group from which the automatic choice attends on tensor cores.
+constexpr int kTensorAttnMinLanes = 64;
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);
 
 // Records the message returned by zha_last_error() on this thread; returns s.

@@ -32,7 +32,7 @@ constexpr int kTileN = 128;          // rows (node, plane) per tile
 constexpr int kR = 16;               // planes per node on this path
 constexpr int kNodes = kTileN / kR;  // nodes per tile
 constexpr int kThreads = 256;
-constexpr long long kSpinLimit = 1ll << 26;
+constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -67,8 +67,11 @@ __device__ __forceinline__ void mma_commit(uint32_t mbar) {
                  : "memory");
 }
 
+// Waits for the mbarrier phase with the given parity; gives up after about 2 s of wall time.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-    for (long long it = 0; it < kSpinLimit; ++it) {
+    uint64_t t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -78,8 +81,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
             : "r"(mbar), "r"(parity)
             : "memory");
         if (done) return true;
+        uint64_t t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > kWaitNs) return false;
     }
-    return false;
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -162,22 +167,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
     const int64_t ns = sq.ns;
     const float* recb = sq.rec[lev] + (int64_t)g * sq.cap[lev] * ns;
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
-    uint32_t phase = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        // node ids of this tile
-        if (tid < kNodes) {
-            const int64_t k = t * kNodes + tid;
-            int64_t j = -1;
-            if (k < nc) j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
-            sJ[tid] = j;
+
+    // Thread `tid` moves float4 c4 = tid % (D/4) of rows tid/(D/4) + u*(kThreads/(D/4)),
+    // u < kU, of a node tile (kTileN rows of D floats); threads < kTileN also move one b.
+    constexpr int kRowStep = kThreads / (D / 4);
+    constexpr int kU = kTileN / kRowStep;
+    const int c4 = tid % (D / 4);
+    const int row0 = tid / (D / 4);
+    float4 pre[kU];
+    float preb = 0.0f;
+    int64_t prej = -1;                          // node id of row tid (threads < kTileN)
+    auto node_of = [&](int64_t t, int nl) -> int64_t {
+        const int64_t k = t * kNodes + nl;
+        if (k >= nc) return -1;
+        return top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
+    };
+    auto prefetch = [&](int64_t t) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int row = row0 + u * kRowStep;
+            const int64_t j = node_of(t, row / kR);
+            pre[u] = j >= 0 ? __ldg(reinterpret_cast<const float4*>(recb + j * ns + (int64_t)(row % kR) * D) + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
-        // B: rows (node, plane) split into tf32 hi and f32 residual lo
-        for (int i = tid; i < kTileN * (D / 4); i += kThreads) {
-            const int row = i / (D / 4), c4 = i % (D / 4);
-            const int64_t j = sJ[row / kR];
-            float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j >= 0) m = __ldg(reinterpret_cast<const float4*>(recb + j * ns + (int64_t)(row % kR) * D) + c4);
+        if (tid < kTileN) {
+            prej = node_of(t, tid / kR);
+            preb = prej >= 0 ? __ldg(recb + prej * ns + (int64_t)kR * D + tid % kR) : 0.0f;
+        }
+    };
+
+    uint32_t phase = 0;
+    int64_t t = blockIdx.x;
+    prefetch(t);
+    for (; t < ntiles; t += gridDim.x) {
+        // B: rows (node, plane) split into tf32 hi and f32 residual lo, from the prefetch
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int row = row0 + u * kRowStep;
+            const float4 m = pre[u];
             float4 hi, lo;
             hi.x = __uint_as_float(__float_as_uint(m.x) & 0xFFFFE000u); lo.x = m.x - hi.x;
             hi.y = __uint_as_float(__float_as_uint(m.y) & 0xFFFFE000u); lo.y = m.y - hi.y;
@@ -188,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
             *reinterpret_cast<float4*>(sLo + off) = lo;
         }
         if (tid < kTileN) {
-            const int64_t j = sJ[tid / kR];
-            sB[tid] = j >= 0 ? __ldg(recb + j * ns + (int64_t)kR * D + tid % kR) : 0.0f;
+            sB[tid] = preb;
+            if (tid % kR == 0) sJ[tid / kR] = prej;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -212,6 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
             mma_commit(smem_u32(&mbar));
         }
         __syncwarp();
+        // next tile's loads overlap this tile's MMAs and epilogue
+        if (t + gridDim.x < ntiles) prefetch(t + gridDim.x);
         if (!mbar_wait(smem_u32(&mbar), phase)) {
             if (lane == 0) {
                 atomicOr(w.status, kStatusTimeout);

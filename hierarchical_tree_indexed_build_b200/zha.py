@@ -25,7 +25,7 @@ _STATUS = {0: "ZHA_OK", 1: "ZHA_ERR_ARG", 2: "ZHA_ERR_CAPACITY", 3: "ZHA_ERR_CUD
 # Every function declared in include/zha.h.
 EXPORTS = ["zha_last_error", "zha_tree_create", "zha_tree_destroy", "zha_tree_info", "zha_build_tree",
            "zha_append", "zha_tree_export", "zha_decoder_create", "zha_decoder_destroy", "zha_route",
-           "zha_sparse_attn", "zha_sparse_attn_static", "zha_decode", "zha_decoder_set_score_path", "zha_decoder_export_kept", "zha_decoder_words",
+           "zha_sparse_attn", "zha_sparse_attn_static", "zha_decode", "zha_decoder_set_kernels", "zha_decoder_export_kept", "zha_decoder_words",
            "zha_decoder_stats", "zha_profile_enable", "zha_profile_read", "zha_profile_reset"]
 
 
@@ -77,7 +77,7 @@ def lib() -> ctypes.CDLL:
                                              _vp, _i64, _vp, _vp]
         L.zha_decode.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, ctypes.c_float,
                                  _vp, _vp]
-        L.zha_decoder_set_score_path.argtypes = [_vp, _i32]
+        L.zha_decoder_set_kernels.argtypes = [_vp, _i32, _i32]
         L.zha_decoder_export_kept.argtypes = [_vp, _i32, _vp, _vp, _vp]
         L.zha_decoder_words.argtypes = [_vp, _i32]
         L.zha_decoder_words.restype = _i64
@@ -177,11 +177,11 @@ def zha_decode(dec: int, K, V, Q: int, n_q: int, p: float, out: int, stream: int
     _check(lib().zha_decode(dec, K, V, Q, n_q, p, out, stream))
 
 
-ZHA_SCORE_AUTO, ZHA_SCORE_SIMT, ZHA_SCORE_TENSOR = 0, 1, 2
+ZHA_KERNELS_AUTO, ZHA_KERNELS_SIMT, ZHA_KERNELS_TENSOR = 0, 1, 2
 
 
-def zha_decoder_set_score_path(dec: int, path: int):
-    _check(lib().zha_decoder_set_score_path(dec, path))
+def zha_decoder_set_kernels(dec: int, score: int, attn: int):
+    _check(lib().zha_decoder_set_kernels(dec, score, attn))
 
 
 def zha_decoder_export_kept(dec: int, level: int, bits: int, counts: Optional[int], stream: int):
@@ -313,8 +313,8 @@ class Decoder:
         self.n_q = Q.shape[1]
         return out
 
-    def set_score_path(self, path: int):
-        zha_decoder_set_score_path(self.handle, path)
+    def set_kernels(self, score: int = ZHA_KERNELS_AUTO, attn: int = ZHA_KERNELS_AUTO):
+        zha_decoder_set_kernels(self.handle, score, attn)
 
     def words(self, level: int) -> int:
         return zha_decoder_words(self.handle, level)

@@ -128,13 +128,16 @@ zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void
 zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
                            const void* Q, int32_t n_q, float* out, void* stream);
 
-/* Which kernels compute the plane estimates (same result up to float32 rounding):
- *   ZHA_SCORE_AUTO    tensor cores (tcgen05, tf32 hi+lo passes) when a (sequence, KV head)
- *                     group has >= 64 lanes and every tree has R = 16, else CUDA cores
- *   ZHA_SCORE_SIMT    CUDA cores (fp32 FMA) always
- *   ZHA_SCORE_TENSOR  tensor cores always (ZHA_ERR_ARG unless every tree has R = 16) */
-typedef enum zha_score_path { ZHA_SCORE_AUTO = 0, ZHA_SCORE_SIMT = 1, ZHA_SCORE_TENSOR = 2 } zha_score_path;
-zha_status zha_decoder_set_score_path(zha_decoder* dec, int32_t path);
+/* Which kernels a decoder uses (both choices give the same result up to float32
+ * rounding).  ZHA_KERNELS_AUTO picks the tensor cores (tcgen05) when a (sequence, KV
+ * head) group has >= 64 lanes - for scoring only if every tree has R = 16 - and the CUDA
+ * cores otherwise; SIMT and TENSOR force one kind.
+ *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::tf32 with hi+lo passes
+ *          (ZHA_ERR_ARG for TENSOR unless every tree has R = 16)
+ *   attn   exact attention: CUDA-core split-KV, or tcgen05 kind::f16 (S = Q K^T exact
+ *          products, P split into bf16 hi + lo for P V) */
+typedef enum zha_kernels { ZHA_KERNELS_AUTO = 0, ZHA_KERNELS_SIMT = 1, ZHA_KERNELS_TENSOR = 2 } zha_kernels;
+zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, int32_t attn);
 
 /* Exact attention over a routed token set that allocates no device memory.  The pages
  * have no counterpart: this is a service for callers that cannot allocate where they

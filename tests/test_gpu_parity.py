@@ -243,12 +243,12 @@ def test_tensor_core_and_cuda_core_scoring_agree(n_q):
     tree, K, V, qr = TL.make_tree(seq)
     Q = wl.Q[0]
     res = {}
-    for path in (zha.ZHA_SCORE_SIMT, zha.ZHA_SCORE_TENSOR):
+    for path in (zha.ZHA_KERNELS_SIMT, zha.ZHA_KERNELS_TENSOR):
         dec = zha.Decoder([tree], n_q)
-        dec.set_score_path(path)
+        dec.set_kernels(score=path, attn=zha.ZHA_KERNELS_SIMT)
         res[path] = TL.gpu_decode([tree], [K], [V], Q, 0.95, dec=dec)
         dec.close()
-    a, b = res[zha.ZHA_SCORE_SIMT], res[zha.ZHA_SCORE_TENSOR]
+    a, b = res[zha.ZHA_KERNELS_SIMT], res[zha.ZHA_KERNELS_TENSOR]
     differ = sum(int((x != y).any(axis=1).sum()) for x, y in zip(a.kept[0], b.kept[0]))
     lanes = a.kept[0][0].shape[0]
     print("[tc vs simt n_q=%d] lane-levels differing: %d of %d" % (n_q, differ, lanes * len(a.kept[0])))
@@ -265,5 +265,31 @@ def test_tensor_core_scoring_needs_r16():
     tree, K, V, qr = TL.make_tree(seq)
     dec = zha.Decoder([tree], 1)
     with pytest.raises(zha.ZhaError) as ei:
-        dec.set_score_path(zha.ZHA_SCORE_TENSOR)
+        dec.set_kernels(score=zha.ZHA_KERNELS_TENSOR)
     assert ei.value.status == zha.ZHA_ERR_ARG
+
+
+@needs_cuda
+@pytest.mark.parametrize("n_q,p", [(1, 0.95), (8, 0.9), (64, 0.95), (64, 1.0)])
+def test_tensor_core_and_cuda_core_attention_agree(n_q, p):
+    """The tcgen05 attention (exact QK^T, bf16 hi+lo P) and the CUDA-core attention give the
+    same outputs on the same routed sets, and the tensor-core output matches the oracle."""
+    wl = inputs.deep_64k(n_q=n_q)
+    seq = wl.seqs[0]
+    n = seq.n_tokens - 1234                        # ragged: dense tail after the last top node
+    tree, K, V, qr = TL.make_tree(seq, n)
+    Q = wl.Q[0]
+    outs = {}
+    for path in (zha.ZHA_KERNELS_SIMT, zha.ZHA_KERNELS_TENSOR):
+        dec = zha.Decoder([tree], n_q)
+        dec.set_kernels(score=zha.ZHA_KERNELS_SIMT, attn=path)
+        outs[path] = TL.gpu_decode([tree], [K], [V], Q, p, dec=dec)
+        dec.close()
+    a, b = outs[zha.ZHA_KERNELS_SIMT], outs[zha.ZHA_KERNELS_TENSOR]
+    for x, y in zip(a.kept[0], b.kept[0]):
+        assert np.array_equal(x, y)               # same scorer: identical routing
+    e = TL.rel_err(b.out.reshape(-1, 128), a.out.reshape(-1, 128)).max()
+    print("[attn tc vs simt n_q=%d p=%g] max rel diff %.2e" % (n_q, p, e))
+    assert e <= 1e-4
+    rep, e1, e2, _ = TL.check_decode(seq, n, Q[0], p, b.out[0], b.kept[0], list(range(min(n_q, 3))))
+    _report("attn tensor n_q=%d p=%g" % (n_q, p), rep, e1, e2)
