@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--p", type=float, default=0.95)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default="deep1m", choices=["deep1m", "deep64k", "wide256k"],
+                    help="deep1m is the benchmark; the smaller ones serve profiling runs")
     return ap.parse_args()
 
 
@@ -138,7 +140,7 @@ def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
 def run_ours(args, rank, world, dev):
     from hierarchical_tree_indexed_build_b200 import zha
     torch.cuda.set_device(dev)
-    wl = inputs.deep_1m()
+    wl = load_workload(args.workload)
     seq = wl.seqs[0]
     g = seq.geom
     N0, n_app = seq.n_tokens, wl.n_append
@@ -155,7 +157,8 @@ def run_ours(args, rank, world, dev):
 
     def step():
         tree.build(K, N0, qref)
-        tree.append(K, N0, n_app)
+        if n_app:
+            tree.append(K, N0, n_app)
         dec.decode([K], [V], Q, args.p, out)
 
     for _ in range(args.warmup):
@@ -271,6 +274,18 @@ def run_ours(args, rank, world, dev):
     return res
 
 
+def load_workload(name):
+    if name == "deep64k":
+        wl = inputs.deep_64k()
+        wl.n_append = 0
+        return wl
+    if name == "wide256k":
+        wl = inputs.wide_256k()
+        wl.n_append = 0
+        return wl
+    return inputs.deep_1m()
+
+
 def cpu_baseline(wl, p, min_s=10.0, max_queries=64):
     """The float64 oracle as it stands on a bounded sample of the same workload: query
     tokens (16 heads each) routed and attended one after another until about min_s
@@ -292,9 +307,8 @@ def cpu_baseline(wl, p, min_s=10.0, max_queries=64):
         done += 1
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": "queries/s", "cores": O.num_threads(), "kind": "oracle",
-            "sample": "%d query tokens x 16 heads of the 1M-token deep workload (N=%d after append), "
-                      "float64 routing with definition-level summaries + exact attention, %.1f s"
-                      % (done, N, dt)}
+            "sample": "%d query tokens x %d heads of the %s workload (N=%d), float64 routing with "
+                      "definition-level summaries + exact attention, %.1f s" % (done, g.Hq, wl.name, N, dt)}
 
 
 def base_line(args, world, wl):
@@ -319,7 +333,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        wl = inputs.deep_1m()
+        wl = load_workload(args.workload)
         for _ in range(args.warmup):
             pass   # the oracle has no warm-up state; each step below is a full sample
         vals = [cpu_baseline(wl, args.p) for _ in range(args.steps)]

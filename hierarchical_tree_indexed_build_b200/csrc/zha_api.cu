@@ -356,6 +356,9 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     off += up256((size_t)dec->groups_cap * w.us * 4);
     const size_t ucount_off = off;
     off += up256((size_t)dec->groups_cap * 4);
+    w.uw = w.W[1];
+    const size_t uword_off = off;
+    off += up256((size_t)dec->groups_cap * w.uw * 4);
     const size_t part_off = off;
     off += up256((size_t)dec->lanes_cap * w.s_cap * (dec->d + 4) * 4);
     const size_t ctr_off = off;
@@ -376,6 +379,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.e = reinterpret_cast<float*>(base + e_off);
     w.ulist = reinterpret_cast<int32_t*>(base + ulist_off);
     w.ucount = reinterpret_cast<int32_t*>(base + ucount_off);
+    w.uword = reinterpret_cast<uint32_t*>(base + uword_off);
     w.part = reinterpret_cast<float*>(base + part_off);
     w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);
     w.status = reinterpret_cast<int32_t*>(base + status_off);

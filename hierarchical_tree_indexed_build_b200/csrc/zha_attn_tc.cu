@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     unsigned char* sPl = sPh + 2 * kBlock;                  // 2 blocks
     int32_t* s_tok0 = reinterpret_cast<int32_t*>(sPl + 2 * kBlock);  // [2][kPos]
     int32_t* s_cid0 = s_tok0 + 2 * kPos;                             // [2][kPos]
+    uint32_t* s_mem0 = reinterpret_cast<uint32_t*>(s_cid0 + 2 * kPos);  // [2][kRows][kPos/32] lane masks
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_sh;
     __shared__ int abort_sh;
@@ -181,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     // Softmax state of lane row `tid` (threads 0..127; warp w reads TMEM lanes 32w..32w+31).
     const int row = tid & 127;
     const int y = y0 + row;
-    const bool row_ok = tid < kRows && y < b.n_gl;
+    const bool y_ok = y < b.n_gl;                  // lane row `row` is one of the group's lanes
+    const bool row_ok = tid < kRows && y_ok;      // ... and this thread runs its softmax
     const int64_t x = lane_of(b, s, g, y < b.n_gl ? y : 0);
     const uint32_t* kb1 = w.kept[1] + x * w.W[1];
     const uint32_t lane_t = (uint32_t)((warp & 3) * 32) << 16;
@@ -237,8 +239,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
+    // Membership masks of tile p0 (buffer bs) for lane row `row`: position pp is attended
+    // by the lane iff it holds a token and its segment is the sink, the tail, or a chunk
+    // the lane kept.  Run by warps 4-7 (one lane row per thread) ahead of the softmax.
+    auto build_mem = [&](int64_t p0, int bs) {
+        uint32_t mw[kPos / 32];
+#pragma unroll
+        for (int k = 0; k < kPos / 32; ++k) mw[k] = 0;
+        const int64_t segA = p0 / C;
+        const int64_t segB = min((p0 + kPos - 1) / C, nseg - sg0 - 1);
+        for (int64_t sr = segA; sr <= segB; sr += 8) {
+            uint32_t lb[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int64_t seg = sg0 + sr + i;
+                uint32_t bit = 0;
+                if (sr + i <= segB) {
+                    if (has_sink && seg == 0) {
+                        bit = 1;
+                    } else {
+                        const int64_t k = seg - has_sink;
+                        if (k < nu) {
+                            const int32_t j = __ldg(ul + k);
+                            bit = (__ldg(kb1 + (j >> 5)) >> (j & 31)) & 1u;
+                        } else {
+                            bit = 1;
+                        }
+                    }
+                }
+                lb[i] = bit;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (!lb[i]) continue;
+                const int64_t a = max((int64_t)0, (sr + i) * C - p0);
+                const int64_t e = min((int64_t)kPos, (sr + i + 1) * C - p0);
+                for (int64_t pp = a; pp < e; ++pp) mw[pp >> 5] |= 1u << (pp & 31);
+            }
+        }
+        const int32_t* tk = s_tok0 + bs * kPos;
+#pragma unroll
+        for (int k = 0; k < kPos / 32; ++k) {
+            uint32_t valid = 0;
+            for (int i = 0; i < 32; ++i) valid |= (tk[k * 32 + i] >= 0 ? 1u : 0u) << i;
+            s_mem0[(bs * kRows + row) * (kPos / 32) + k] = y_ok ? (mw[k] & valid) : 0u;
+        }
+    };
+
     resolve(0, 0);
     __syncthreads();
+    if (warp >= 4) build_mem(0, 0);
     issue_kv(0, true);
     int st = 0;
     for (int64_t p0 = 0; p0 < npos; p0 += kPos, st ^= 1) {
@@ -270,32 +320,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         __syncthreads();                       // next tile's tokens visible; K buffer free
         if (more) issue_kv(st ^ 1, true);      // overlaps this tile's softmax and P V
-        const int32_t* s_cid = s_cid0 + st * kPos;
 
-        // softmax of the lane rows (warps 0-3)
-        if (warp < 4) {
-            // membership of this lane at each position (cached per chunk id)
+        // warps 4-7: next tile's membership masks; warps 0-3: softmax of this tile
+        if (warp >= 4) {
+            if (more) build_mem(p0 + kPos, st ^ 1);
+        } else {
             uint32_t mem[kPos / 32];
-            int32_t last = -3;
-            uint32_t lastbit = 0;
 #pragma unroll
-            for (int k = 0; k < kPos / 32; ++k) mem[k] = 0;
-            for (int pp = 0; pp < kPos; ++pp) {
-                const int32_t cid = s_cid[pp];
-                uint32_t bit;
-                if (cid == -1) bit = 1;
-                else if (cid < 0) bit = 0;
-                else {
-                    if (cid != last) {
-                        last = cid;
-                        lastbit = (__ldg(kb1 + (cid >> 5)) >> (cid & 31)) & 1u;
-                    }
-                    bit = lastbit;
-                }
-                mem[pp >> 5] |= bit << (pp & 31);
-            }
+            for (int k = 0; k < kPos / 32; ++k) mem[k] = s_mem0[(st * kRows + row) * (kPos / 32) + k];
             float tmax = -INFINITY;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < kPos / 16; ++c) {
                 float v[16];
                 tld16(tS + lane_t + c * 16, v);
@@ -317,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 m_ref = tmax;
             }
             if (__any_sync(0xffffffffu, need) && !first_pv) {
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
                     float o[16];
                     tld16(tO + lane_t + c * 16, o);
@@ -327,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 }
             }
             // warps read/write TMEM uniformly; rows without members write zero P
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < kPos / 16; ++c) {
                 float v[16];
                 tld16(tS + lane_t + c * 16, v);
@@ -415,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
-    return (size_t)(4 * kbd + 4) * kBlock + 4 * kPos * 4 + 1024;
+    return (size_t)(4 * kbd + 4) * kBlock + 4 * kPos * 4 + 2 * kRows * (kPos / 32) * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {

@@ -48,6 +48,8 @@ struct Work {
     int32_t* ulist;                  // [groups_cap][us] union lists
     int64_t us;
     int32_t* ucount;                 // [groups_cap]
+    uint32_t* uword;                 // [groups_cap][uw] union bitmap being built
+    int64_t uw;
     float* part;                     // [lanes_cap][s_cap][d+2] attention partials
     int64_t s_cap;
     unsigned long long* ctr;         // kCtrCount counters

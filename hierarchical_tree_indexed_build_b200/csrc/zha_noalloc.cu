@@ -69,6 +69,8 @@ extern "C" zha_status zha_sparse_attn_static(const void* K, const void* V, int64
     const size_t status_off = off;  off += up256(4);
     const size_t ucount_off = off;  off += up256((size_t)Hkv * 4);
     const size_t ulist_off = off;   off += up256((size_t)Hkv * std::max<int64_t>(n1, 1) * 4);
+    const int64_t uw = std::max<int64_t>(words, 1);
+    const size_t uword_off = off;   off += up256((size_t)Hkv * uw * 4);
     const size_t kcount_off = off;  off += up256((size_t)(kMaxL + 1) * lanes * 4);
     const size_t part_off = off;    off += up256((size_t)lanes * splits * (d + 4) * 4);
     if (off > kStaticScratchBytes) {
@@ -125,6 +127,8 @@ extern "C" zha_status zha_sparse_attn_static(const void* K, const void* V, int64
     w.ulist = reinterpret_cast<int32_t*>(base + ulist_off);
     w.us = std::max<int64_t>(n1, 1);
     w.ucount = reinterpret_cast<int32_t*>(base + ucount_off);
+    w.uword = reinterpret_cast<uint32_t*>(base + uword_off);
+    w.uw = uw;
     w.part = reinterpret_cast<float*>(base + part_off);
     w.s_cap = splits;
     w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);

@@ -137,44 +137,59 @@ __device__ T block_excl_scan(T v, T* red, T& total) {
 
 // ----------------------------------------------------------------------------- union
 
-// Sorted union over a group's lanes of the kept nodes at level `ulev`.  Mode 0: ulev =
-// L_s - it + 1 (routing iteration it >= 1); mode 1: ulev = 1 (attention).
-__global__ void __launch_bounds__(1024) k_union(Batch b, Work w, int it, int mode) {
-    __shared__ int red[33];
-    const int grp = blockIdx.x;
-    const int s = grp / b.Hkv, g = grp % b.Hkv;
-    const SeqDev& sq = b.seqs[s];
-    int ulev;
+// Level whose kept sets a union call gathers for sequence sq, 0 if none.  Mode 0: routing
+// iteration it >= 1 needs the kept nodes of level L_s - it + 1 (their children are the
+// candidates); mode 1: attention needs the kept level-1 chunks.
+__device__ __forceinline__ int union_level(const SeqDev& sq, int it, int mode) {
     if (mode == 0) {
         const int lev = sq.L - it;
-        if (it == 0 || lev < 1) {
-            if (threadIdx.x == 0) w.ucount[grp] = 0;
-            return;
-        }
-        ulev = lev + 1;
-    } else {
-        ulev = 1;
-        if (sq.T == 0) {
-            if (threadIdx.x == 0) {
-                w.ucount[grp] = 0;
-                atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)sq.N);
-            }
-            return;
-        }
+        return (it == 0 || lev < 1) ? 0 : lev + 1;
     }
-    const int64_t nl = sq.n[ulev];
-    const int64_t nwords = (nl + 31) / 32;
+    return sq.T == 0 ? 0 : 1;
+}
+
+// OR of the kept bitmaps of a chunk of a group's lanes into the group's union bitmap.
+// Grid: (word blocks, lane chunks of `lanes_per_block`, groups).
+__global__ void __launch_bounds__(256) k_union_or(Batch b, Work w, int it, int mode, int lanes_per_block) {
+    const int grp = blockIdx.z;
+    const int s = grp / b.Hkv, g = grp % b.Hkv;
+    const SeqDev& sq = b.seqs[s];
+    const int ulev = union_level(sq, it, mode);
+    if (ulev == 0) return;
+    const int64_t nwords = (sq.n[ulev] + 31) / 32;
+    const int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (wi >= nwords) return;
+    const int y0 = blockIdx.y * lanes_per_block;
+    const int y1 = min(b.n_gl, y0 + lanes_per_block);
     const uint32_t* kb = w.kept[ulev];
     const int64_t W = w.W[ulev];
+    uint32_t word = 0;
+#pragma unroll 8
+    for (int y = y0; y < y1; ++y) word |= __ldg(kb + lane_of(b, s, g, y) * W + wi);
+    if (word) atomicOr(w.uword + (int64_t)grp * w.uw + wi, word);
+}
+
+// Compacts a group's union bitmap into the sorted list of set bits.
+__global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it, int mode) {
+    __shared__ int red[33];
+    const int grp = blockIdx.x;
+    const int s = grp / b.Hkv;
+    const SeqDev& sq = b.seqs[s];
+    const int ulev = union_level(sq, it, mode);
+    if (ulev == 0) {
+        if (threadIdx.x == 0) {
+            w.ucount[grp] = 0;
+            if (mode == 1) atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)sq.N);   // dense: A = [0, N)
+        }
+        return;
+    }
+    const int64_t nwords = (sq.n[ulev] + 31) / 32;
+    const uint32_t* uwp = w.uword + (int64_t)grp * w.uw;
     int32_t* out = w.ulist + (int64_t)grp * w.us;
     int base = 0;
-    bool has0 = false;
     for (int64_t w0 = 0; w0 < nwords; w0 += blockDim.x) {
         const int64_t wi = w0 + threadIdx.x;
-        uint32_t word = 0;
-        if (wi < nwords)
-            for (int y = 0; y < b.n_gl; ++y) word |= kb[lane_of(b, s, g, y) * W + wi];
-        if (wi == 0) has0 = word & 1u;
+        uint32_t word = wi < nwords ? uwp[wi] : 0u;
         int total;
         const int excl = block_excl_scan<int>(__popc(word), red, total);
         int k = base + excl;
@@ -185,12 +200,14 @@ __global__ void __launch_bounds__(1024) k_union(Batch b, Work w, int it, int mod
         }
         base += total;
     }
-    if (threadIdx.x == 0) w.ucount[grp] = base;
-    if (mode == 1 && threadIdx.x == 0) {
-        // attended tokens of the group: sink + kept chunks (token 0 once) + tail
-        const int64_t tail = sq.N - sq.T * sq.top;
-        atomicAdd(&w.ctr[kCtrUnionTokens],
-                  (unsigned long long)(tail + 1 + (int64_t)base * sq.C - (has0 ? 1 : 0)));
+    if (threadIdx.x == 0) {
+        w.ucount[grp] = base;
+        if (mode == 1) {
+            // attended tokens of the group: sink + kept chunks (token 0 once) + tail
+            const int64_t tail = sq.N - sq.T * sq.top;
+            const int has0 = nwords > 0 ? (int)(uwp[0] & 1u) : 0;
+            atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)(tail + 1 + (int64_t)base * sq.C - has0));
+        }
     }
 }
 
@@ -535,7 +552,12 @@ int score_blocks_x(int lane_blocks, int groups) {
 
 cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaStream_t st) {
     ProfScope ps_("k_union", st);
-    k_union<<<b.n_groups, 1024, 0, st>>>(b, w, it, mode);
+    cudaError_t e = cudaMemsetAsync(w.uword, 0, (size_t)b.n_groups * w.uw * 4, st);
+    if (e != cudaSuccess) return e;
+    const int lanes_per_block = 64;
+    dim3 grid((unsigned)((w.uw + 255) / 256), (b.n_gl + lanes_per_block - 1) / lanes_per_block, b.n_groups);
+    k_union_or<<<grid, 256, 0, st>>>(b, w, it, mode, lanes_per_block);
+    k_union_compact<<<b.n_groups, 1024, 0, st>>>(b, w, it, mode);
     return cudaGetLastError();
 }
 
