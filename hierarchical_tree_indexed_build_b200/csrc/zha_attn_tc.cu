@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     constexpr int KBD = D / 64;                 // 128-byte blocks along d (bf16)
     constexpr int PR = D + 4;
     constexpr int TCOLS = 256;                  // S: columns [0,128), O: [128, 128+D)
+    constexpr int kHalf = kPos / 2;             // positions per warp of a row pair
+    constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~uintptr_t(1023));
@@ -131,12 +133,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     unsigned char* sV0 = sK + KBD * kBlock;                 // 2 x KBD blocks (MN-major, double buffer)
     unsigned char* sPh = sV0 + 2 * KBD * kBlock;            // 2 blocks
     unsigned char* sPl = sPh + 2 * kBlock;                  // 2 blocks
-    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sPl + 2 * kBlock);  // [2][kPos]
-    int32_t* s_cid0 = s_tok0 + 2 * kPos;                             // [2][kPos]
-    uint32_t* s_mem0 = reinterpret_cast<uint32_t*>(s_cid0 + 2 * kPos);  // [2][kRows][kPos/32] lane masks
+    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sPl + 2 * kBlock);  // [2][kPos] token (-1: none)
+    int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: chunk id, -1 all, -2 none
+    uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_slot0 + 2 * kPos);   // [2][kPos] slot of each position
+    uint32_t* s_valid0 = reinterpret_cast<uint32_t*>(s_pslot0 + 2 * kPos); // [2][kPos/32] positions with a token
+    float* s_xmax = reinterpret_cast<float*>(s_valid0 + 2 * (kPos / 32));  // [2][kRows] tile max per half
+    float* s_xsum = s_xmax + 2 * kRows;                                     // [2][kRows] row sums per half
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_sh;
-    __shared__ int abort_sh;
+    __shared__ int abort_flag;
+    volatile int& abort_sh = abort_flag;
 
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
@@ -179,15 +185,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const uint32_t tmem = tmem_sh;
     const uint32_t tS = tmem, tO = tmem + 128;
 
-    // Softmax state of lane row `tid` (threads 0..127; warp w reads TMEM lanes 32w..32w+31).
-    const int row = tid & 127;
+    // Row (lane) state.  Warps w and w+4 read the same TMEM lanes 32(w%4).. and share the
+    // row; `half` selects positions [64 half, 64 half + 64) and O columns [D/2 half, ...).
+    const int half = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
     const int y = y0 + row;
-    const bool y_ok = y < b.n_gl;                  // lane row `row` is one of the group's lanes
-    const bool row_ok = tid < kRows && y_ok;      // ... and this thread runs its softmax
-    const int64_t x = lane_of(b, s, g, y < b.n_gl ? y : 0);
+    const bool y_ok = y < b.n_gl;
+    const int64_t x = lane_of(b, s, g, y_ok ? y : 0);
     const uint32_t* kb1 = w.kept[1] + x * w.W[1];
     const uint32_t lane_t = (uint32_t)((warp & 3) * 32) << 16;
-    float m_ref = -INFINITY, lsum = 0.0f;
+    float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in both warps of a row
 
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     const __nv_bfloat16* Kg = sq.K + (int64_t)g * sq.ld * D;
@@ -195,101 +202,61 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     uint32_t phase = 0;
     bool first_pv = true;
 
-    // Token of each position of tile p0 into buffer `st`: sink segment (position 0 only),
-    // kept chunks, tail.  cid -2: no token, -1: every lane, >= 0: chunk id.
+    // Tokens of tile p0 into buffer st (threads 0..127, one position each): sink segment
+    // (position 0 only), kept chunks, tail.  Also the slot table: slot k of the tile is the
+    // k-th segment it touches; s_slot holds its chunk id (-1: every lane, -2: none) and
+    // s_pslot the slot of each position; s_valid marks positions holding a token.
     auto resolve = [&](int64_t p0, int st) {
         if (tid < kPos) {
             const int64_t pp = p0 + tid;
-            int32_t tok = -1, cid = -2;
+            int32_t tok = -1, code = -2;
             if (pp < npos) {
                 const int64_t seg = sg0 + pp / C, off = pp % C;
                 if (has_sink && seg == 0) {
-                    if (off == 0) { tok = 0; cid = -1; }
+                    code = -1;
+                    if (off == 0) tok = 0;
                 } else {
                     const int64_t k = seg - has_sink;
                     if (k < nu) {
                         const int64_t j = ul[k];
                         const int64_t t = j * C + off;
-                        if (t != 0) { tok = (int32_t)t; cid = (int32_t)j; }
+                        code = (int32_t)j;
+                        if (t != 0) tok = (int32_t)t;
                     } else {
                         const int64_t t = tail0 + (k - nu) * C + off;
-                        if (t < N) { tok = (int32_t)t; cid = -1; }
+                        code = -1;
+                        if (t < N) tok = (int32_t)t;
                     }
                 }
             }
+            const int slot = (int)((p0 + tid) / C - p0 / C);
             s_tok0[st * kPos + tid] = tok;
-            s_cid0[st * kPos + tid] = cid;
+            s_pslot0[st * kPos + tid] = (uint8_t)slot;
+            if (tid == 0 || (p0 + tid) % C == 0) s_slot0[st * kPos + slot] = code;
+            const unsigned vb = __ballot_sync(0xffffffffu, tok >= 0);
+            if (lane == 0) s_valid0[st * (kPos / 32) + warp] = vb;
         }
     };
     // Asynchronous gather of the K (K-major) and V (MN-major) rows of buffer st's tokens;
     // empty positions are zero-filled.
-    auto issue_kv = [&](int st, bool with_k) {
+    auto issue_kv = [&](int st) {
         for (int i = tid; i < kPos * (D / 8); i += kThreads) {
             const int t = i / (D / 8), c16 = i % (D / 8);
             const int32_t tok = s_tok0[st * kPos + t];
             const uint32_t n = tok >= 0 ? 16u : 0u;
-            const int64_t row = tok >= 0 ? tok : 0;
-            const void* gk = reinterpret_cast<const uint4*>(Kg + row * D) + c16;
-            const void* gv = reinterpret_cast<const uint4*>(Vg + row * D) + c16;
-            if (with_k)
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sK + kmaj(t, c16))), "l"(gk), "r"(n) : "memory");
+            const int64_t rw = tok >= 0 ? tok : 0;
+            const void* gk = reinterpret_cast<const uint4*>(Kg + rw * D) + c16;
+            const void* gv = reinterpret_cast<const uint4*>(Vg + rw * D) + c16;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sK + kmaj(t, c16))), "l"(gk), "r"(n) : "memory");
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sV0 + st * KBD * kBlock + mnmaj(t, c16))),
                          "l"(gv), "r"(n) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    // Membership masks of tile p0 (buffer bs) for lane row `row`: position pp is attended
-    // by the lane iff it holds a token and its segment is the sink, the tail, or a chunk
-    // the lane kept.  Run by warps 4-7 (one lane row per thread) ahead of the softmax.
-    auto build_mem = [&](int64_t p0, int bs) {
-        uint32_t mw[kPos / 32];
-#pragma unroll
-        for (int k = 0; k < kPos / 32; ++k) mw[k] = 0;
-        const int64_t segA = p0 / C;
-        const int64_t segB = min((p0 + kPos - 1) / C, nseg - sg0 - 1);
-        for (int64_t sr = segA; sr <= segB; sr += 8) {
-            uint32_t lb[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int64_t seg = sg0 + sr + i;
-                uint32_t bit = 0;
-                if (sr + i <= segB) {
-                    if (has_sink && seg == 0) {
-                        bit = 1;
-                    } else {
-                        const int64_t k = seg - has_sink;
-                        if (k < nu) {
-                            const int32_t j = __ldg(ul + k);
-                            bit = (__ldg(kb1 + (j >> 5)) >> (j & 31)) & 1u;
-                        } else {
-                            bit = 1;
-                        }
-                    }
-                }
-                lb[i] = bit;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (!lb[i]) continue;
-                const int64_t a = max((int64_t)0, (sr + i) * C - p0);
-                const int64_t e = min((int64_t)kPos, (sr + i + 1) * C - p0);
-                for (int64_t pp = a; pp < e; ++pp) mw[pp >> 5] |= 1u << (pp & 31);
-            }
-        }
-        const int32_t* tk = s_tok0 + bs * kPos;
-#pragma unroll
-        for (int k = 0; k < kPos / 32; ++k) {
-            uint32_t valid = 0;
-            for (int i = 0; i < 32; ++i) valid |= (tk[k * 32 + i] >= 0 ? 1u : 0u) << i;
-            s_mem0[(bs * kRows + row) * (kPos / 32) + k] = y_ok ? (mw[k] & valid) : 0u;
-        }
-    };
-
     resolve(0, 0);
     __syncthreads();
-    if (warp >= 4) build_mem(0, 0);
-    issue_kv(0, true);
+    issue_kv(0);
     int st = 0;
     for (int64_t p0 = 0; p0 < npos; p0 += kPos, st ^= 1) {
         const bool more = p0 + kPos < npos;
@@ -311,6 +278,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             commit(su32(&mbar));
         }
         __syncwarp();
+
+        // This row's membership on its half of the tile: one bitmap load per chunk slot,
+        // all independent, expanded to positions through the slot index.
+        uint64_t mem = 0;
+        {
+            const uint8_t* ps = s_pslot0 + st * kPos + half * kHalf;
+            const int k0 = ps[0], k1 = ps[kHalf - 1];
+            uint64_t slotbits = 0;
+            for (int kb = k0; kb <= k1; kb += 16) {
+                uint32_t wv[16];
+                int32_t code[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    code[i] = kb + i <= k1 ? s_slot0[st * kPos + kb + i] : -2;
+                    wv[i] = code[i] >= 0 ? __ldg(kb1 + (code[i] >> 5)) : 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t bit = code[i] == -1 ? 1u : (code[i] >= 0 ? (wv[i] >> (code[i] & 31)) & 1u : 0u);
+                    slotbits |= (uint64_t)bit << (kb + i - k0);
+                }
+            }
+#pragma unroll 8
+            for (int i = 0; i < kHalf; ++i) mem |= ((slotbits >> (ps[i] - k0)) & 1ull) << i;
+            const uint32_t* vw = s_valid0 + st * (kPos / 32) + half * 2;
+            mem &= (uint64_t)vw[0] | ((uint64_t)vw[1] << 32);
+            if (!y_ok) mem = 0;
+        }
         if (more) resolve(p0 + kPos, st ^ 1);
         if (!wait_phase(su32(&mbar), phase) && lane == 0) {
             atomicOr(w.status, kStatusTimeout);
@@ -318,74 +313,71 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         }
         phase ^= 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        __syncthreads();                       // next tile's tokens visible; K buffer free
-        if (more) issue_kv(st ^ 1, true);      // overlaps this tile's softmax and P V
 
-        // warps 4-7: next tile's membership masks; warps 0-3: softmax of this tile
-        if (warp >= 4) {
-            if (more) build_mem(p0 + kPos, st ^ 1);
-        } else {
-            uint32_t mem[kPos / 32];
-#pragma unroll
-            for (int k = 0; k < kPos / 32; ++k) mem[k] = s_mem0[(st * kRows + row) * (kPos / 32) + k];
-            float tmax = -INFINITY;
+        // tile max over this half's member positions, combined with the partner warp
+        float tmax = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < kPos / 16; ++c) {
-                float v[16];
-                tld16(tS + lane_t + c * 16, v);
+        for (int c = 0; c < kHalf / 16; ++c) {
+            float v[16];
+            tld16(tS + lane_t + half * kHalf + c * 16, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int pp = c * 16 + i;
-                    if ((mem[pp >> 5] >> (pp & 31)) & 1u) tmax = fmaxf(tmax, scale * v[i]);
-                }
-            }
-            if (!row_ok) tmax = -INFINITY;
-            // Raise this lane's reference max if the tile exceeds it by more than kLazy.
-            // The O rescale reads and writes tensor memory with warp-collective
-            // instructions, so the whole warp runs it (factor 1 on lanes that keep theirs).
-            const bool need = tmax > -INFINITY && m_ref > -INFINITY && tmax > m_ref + kLazy;
-            const float f = need ? expf(m_ref - tmax) : 1.0f;
-            if (tmax > -INFINITY && m_ref == -INFINITY) m_ref = tmax;
-            if (need) {
-                lsum *= f;
-                m_ref = tmax;
-            }
-            if (__any_sync(0xffffffffu, need) && !first_pv) {
+            for (int i = 0; i < 16; ++i)
+                if ((mem >> (c * 16 + i)) & 1ull) tmax = fmaxf(tmax, v[i]);
+        }
+        s_xmax[half * kRows + row] = tmax;
+        __syncthreads();                       // partner maxima visible; next tile's tokens visible
+        if (more) issue_kv(st ^ 1);            // overlaps this tile's softmax and P V
+        tmax = fmaxf(s_xmax[row], s_xmax[kRows + row]);
+        tmax = tmax > -INFINITY ? scale * tmax : -INFINITY;
+
+        // Raise the row's reference max if the tile exceeds it by more than kLazy; both warps
+        // of the row take the same decision.  O is rescaled warp-collectively (factor 1 on
+        // rows that keep theirs), each warp its half of the columns.
+        const bool need = tmax > -INFINITY && m_ref > -INFINITY && tmax > m_ref + kLazy;
+        const float f = need ? exp2f((m_ref - tmax) * kLog2e) : 1.0f;
+        if (tmax > -INFINITY && m_ref == -INFINITY) m_ref = tmax;
+        if (need) {
+            lsum *= f;
+            m_ref = tmax;
+        }
+        if (__any_sync(0xffffffffu, need) && !first_pv) {
 #pragma unroll 1
-                for (int c = 0; c < D / 16; ++c) {
-                    float o[16];
-                    tld16(tO + lane_t + c * 16, o);
+            for (int c = 0; c < D / 32; ++c) {
+                float o[16];
+                const uint32_t col = tO + lane_t + half * (D / 2) + c * 16;
+                tld16(col, o);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] *= f;
-                    tst16(tO + lane_t + c * 16, o);
-                }
+                for (int i = 0; i < 16; ++i) o[i] *= f;
+                tst16(col, o);
             }
-            // warps read/write TMEM uniformly; rows without members write zero P
+        }
+        // P = exp(s S - m) on member positions, split into bf16 hi + lo
+        const float sl = scale * kLog2e, ml = m_ref * kLog2e;
 #pragma unroll 1
-            for (int c = 0; c < kPos / 16; ++c) {
-                float v[16];
-                tld16(tS + lane_t + c * 16, v);
-                uint32_t hi[8], lo[8];
+        for (int c = 0; c < kHalf / 16; ++c) {
+            float v[16];
+            tld16(tS + lane_t + half * kHalf + c * 16, v);
+            uint32_t hi[8], lo[8];
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    const int pp = c * 16 + i;
-                    float p0v = 0.0f, p1v = 0.0f;
-                    if (row_ok && ((mem[pp >> 5] >> (pp & 31)) & 1u)) p0v = expf(fmaf(scale, v[i], -m_ref));
-                    if (row_ok && ((mem[(pp + 1) >> 5] >> ((pp + 1) & 31)) & 1u)) p1v = expf(fmaf(scale, v[i + 1], -m_ref));
-                    lsum += p0v;
-                    lsum += p1v;
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0v, p1v);
-                    const float2 hf = __bfloat1622float2(h);
-                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0v - hf.x, p1v - hf.y);
-                    hi[i / 2] = *reinterpret_cast<const uint32_t*>(&h);
-                    lo[i / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-                }
-                // positions c*16 .. c*16+15 are 16-byte chunks 2c and 2c+1 of this row
-                *reinterpret_cast<uint4*>(sPh + kmaj(row, 2 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(sPh + kmaj(row, 2 * c + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-                *reinterpret_cast<uint4*>(sPl + kmaj(row, 2 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                *reinterpret_cast<uint4*>(sPl + kmaj(row, 2 * c + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            for (int i = 0; i < 16; i += 2) {
+                const float e0 = exp2f(fmaf(sl, v[i], -ml));
+                const float e1 = exp2f(fmaf(sl, v[i + 1], -ml));
+                const float p0v = ((mem >> (c * 16 + i)) & 1ull) ? e0 : 0.0f;
+                const float p1v = ((mem >> (c * 16 + i + 1)) & 1ull) ? e1 : 0.0f;
+                lsum += p0v;
+                lsum += p1v;
+                const __nv_bfloat162 h = __floats2bfloat162_rn(p0v, p1v);
+                const float2 hf = __bfloat1622float2(h);
+                const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0v - hf.x, p1v - hf.y);
+                hi[i / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                lo[i / 2] = *reinterpret_cast<const uint32_t*>(&l2);
             }
+            // positions 64 half + 16 c .. +15 are 16-byte chunks 8 half + 2c, +1 of this row
+            const int c16 = half * 8 + 2 * c;
+            *reinterpret_cast<uint4*>(sPh + kmaj(row, c16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sPh + kmaj(row, c16 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            *reinterpret_cast<uint4*>(sPl + kmaj(row, c16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4*>(sPl + kmaj(row, c16 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -419,24 +411,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         if (abort_sh) break;
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // partial (o, m, l) of every lane row of the tile
-    if (warp < 4) {
+    // partial (o, m, l) of every lane row of the tile: each warp writes its half of o
+    s_xsum[half * kRows + row] = lsum;
+    __syncthreads();
+    {
         float* pp = w.part + (x * w.s_cap + split) * PR;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
             float o[16];
-            tld16(tO + lane_t + c * 16, o);
-            if (row_ok && !abort_sh) {
-                float4* po = reinterpret_cast<float4*>(pp + c * 16);
+            tld16(tO + lane_t + half * (D / 2) + c * 16, o);
+            if (y_ok && !abort_sh) {
+                float4* po = reinterpret_cast<float4*>(pp + half * (D / 2) + c * 16);
                 po[0] = make_float4(o[0], o[1], o[2], o[3]);
                 po[1] = make_float4(o[4], o[5], o[6], o[7]);
                 po[2] = make_float4(o[8], o[9], o[10], o[11]);
                 po[3] = make_float4(o[12], o[13], o[14], o[15]);
             }
         }
-        if (row_ok && !abort_sh) {
+        if (half == 0 && y_ok && !abort_sh) {
             pp[D] = m_ref;
-            pp[D + 1] = lsum;
+            pp[D + 1] = s_xsum[row] + s_xsum[kRows + row];
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -449,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
-    return (size_t)(4 * kbd + 4) * kBlock + 4 * kPos * 4 + 2 * kRows * (kPos / 32) * 4 + 1024;
+    return (size_t)(4 * kbd + 4) * kBlock + 2 * kPos * 4 + 2 * kPos * 4 + 2 * kPos + 2 * (kPos / 32) * 4 +
+           4 * kRows * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {

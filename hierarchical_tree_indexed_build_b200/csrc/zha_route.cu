@@ -316,12 +316,12 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
     __shared__ unsigned long long red_u[33];
     __shared__ float red_f[33];
     __shared__ int s_bstar;
-    __shared__ unsigned long long s_cumb, s_kstar;
+    __shared__ unsigned long long s_cumb;
     __shared__ unsigned int s_nkeys;
+    __shared__ int s_found;
 
     const int64_t x = blockIdx.x;
     const int s = (int)(x / ((int64_t)b.n_q * b.Hq));
-    const int h = (int)(x % b.Hq);
     const SeqDev& sq = b.seqs[s];
     const int lev = sq.L - it;
     if (lev < 1) return;
@@ -331,7 +331,6 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
         if (threadIdx.x == 0) *kcount = 0;
         return;
     }
-    (void)h;
     const bool top = (lev == sq.L);
     const int64_t C = sq.C;
     const uint32_t* P = top ? nullptr : w.kept[lev + 1] + x * w.W[lev + 1];
@@ -339,26 +338,55 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
     uint32_t* outw = w.kept[lev] + x * w.W[lev];
     const int64_t nwords = (nl + 31) / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-
     const int64_t np1 = top ? 0 : sq.n[lev + 1];   // complete parents
-    auto valid_at = [&](int64_t j) -> bool {
-        if (j >= nl) return false;
-        if (top) return true;
-        const int64_t pj = j / C;
-        if (pj >= np1) return false;                 // child of an incomplete parent
-        return (__ldg(P + (pj >> 5)) >> (pj & 31)) & 1u;
+
+    // Candidate j = 32 wi + lane: its score and whether it is on the lane's frontier (a child
+    // of a kept complete parent).  Both loads are issued unconditionally and independently so
+    // a warp keeps several words in flight; scores off the frontier are never used.
+    auto fetch = [&](int64_t wi, float& ev, bool& v) {
+        const int64_t j = wi * 32 + lane;
+        const bool in = j < nl;
+        const int64_t jj = in ? j : nl - 1;
+        ev = e[jj];
+        if (top) {
+            v = in;
+        } else {
+            const int64_t pj = jj / C;
+            const uint32_t pw = __ldg(P + (min(pj, np1 > 0 ? np1 - 1 : 0) >> 5));
+            v = in && pj < np1 && ((pw >> (pj & 31)) & 1u);
+        }
     };
+    constexpr int kUn = 4;   // words per warp in flight
+#define ZHA_FOR_WORDS(BODY)                                                                  \
+    for (int64_t w0 = warp; w0 < nwords; w0 += kUn * nwarps) {                               \
+        float ev_[kUn];                                                                      \
+        bool v_[kUn];                                                                        \
+        _Pragma("unroll") for (int u = 0; u < kUn; ++u) {                                    \
+            const int64_t wi_ = w0 + (int64_t)u * nwarps;                                    \
+            v_[u] = false;                                                                   \
+            ev_[u] = 0.0f;                                                                   \
+            if (wi_ < nwords) fetch(wi_, ev_[u], v_[u]);                                     \
+        }                                                                                    \
+        _Pragma("unroll") for (int u = 0; u < kUn; ++u) {                                    \
+            const int64_t wi = w0 + (int64_t)u * nwarps;                                     \
+            if (wi >= nwords) break;                                                         \
+            const int64_t j = wi * 32 + lane;                                                \
+            const float ev = ev_[u];                                                         \
+            const bool valid = v_[u];                                                        \
+            BODY                                                                             \
+        }                                                                                    \
+    }
 
     // pass 1: frontier max and size
     float mloc = -INFINITY;
     unsigned long long floc = 0;
-    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-        const int64_t j = wi * 32 + lane;
-        if (valid_at(j)) {
-            mloc = fmaxf(mloc, e[j]);
+    ZHA_FOR_WORDS({
+        (void)j;
+        if (valid) {
+            mloc = fmaxf(mloc, ev);
             ++floc;
         }
-    }
+    })
     const float M = block_max(mloc, red_f);
     const unsigned long long F = block_sum<unsigned long long>(floc, red_u);
     if (threadIdx.x == 0) atomicAdd(&w.ctr[kCtrLaneNodes + lev], F);
@@ -367,10 +395,12 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
         return;
     }
     if (b.p >= 1.0f) {
-        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-            const unsigned bal = __ballot_sync(kFull, valid_at(wi * 32 + lane));
+        ZHA_FOR_WORDS({
+            (void)j;
+            (void)ev;
+            const unsigned bal = __ballot_sync(kFull, valid);
             if (lane == 0) outw[wi] = bal;
-        }
+        })
         if (threadIdx.x == 0) *kcount = (int32_t)F;
         return;
     }
@@ -382,23 +412,22 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
     }
     __syncthreads();
     unsigned long long zloc = 0;
-    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-        const int64_t j = wi * 32 + lane;
-        if (valid_at(j)) {
-            const float ev = e[j];
+    ZHA_FOR_WORDS({
+        (void)j;
+        if (valid) {
             const unsigned long long u = mass_of(ev, M);
             zloc += u;
             const int bn = bin_of(ev, M);
             atomicAdd(&hist[bn], u);
             atomicAdd(&hcnt[bn], 1u);
         }
-    }
+    })
     const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
     unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
     if (target < 1ull) target = 1ull;
     if (target > Z) target = Z;
 
-    // pass 3: boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
+    // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
     if (warp == 0) {
         constexpr int per = kNB / 32;
         unsigned long long ls = 0;
@@ -432,17 +461,27 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
     const int bstar = s_bstar;
     const unsigned long long need = target - s_cumb;
     const unsigned nb = hcnt[bstar];
+    const bool collect = nb <= (unsigned)kCap;
 
-    if (nb <= (unsigned)kCap) {
-        // pass 4: collect the boundary bin, sort by (e desc, j asc), find the crossing
-        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-            const int64_t j = wi * 32 + lane;
-            if (valid_at(j)) {
-                const float ev = e[j];
-                if (bin_of(ev, M) == bstar) keys[atomicAdd(&s_nkeys, 1u)] = sel_key(ev, j);
-            }
+    // pass 3: kept bitmap for bins above the boundary; boundary-bin candidates collected
+    unsigned long long cnt = 0;
+    ZHA_FOR_WORDS({
+        bool keep = false;
+        if (valid) {
+            const int bn = bin_of(ev, M);
+            keep = bn < bstar;
+            if (bn == bstar && collect) keys[atomicAdd(&s_nkeys, 1u)] = sel_key(ev, j);
         }
-        __syncthreads();
+        const unsigned bal = __ballot_sync(kFull, keep);
+        if (lane == 0) {
+            outw[wi] = bal;
+            cnt += __popc(bal);
+        }
+    })
+    __syncthreads();
+
+    if (collect) {
+        // sort the boundary bin by (e desc, j asc) and take the prefix reaching the target
         const int n = (int)s_nkeys;
         int npow = 1;
         while (npow < n) npow <<= 1;
@@ -481,65 +520,53 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
         }
         __syncthreads();
         found = block_min_t<int>(found, reinterpret_cast<int*>(red_f));
-        if (threadIdx.x == 0) s_kstar = keys[found < n ? found : n - 1];
-    } else {
-        // rare: too many candidates in one bin - bisection on the exact key order
-        unsigned long long klo = ~0ull, khi = 0ull;
-        for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-            const int64_t j = wi * 32 + lane;
-            if (valid_at(j)) {
-                const float ev = e[j];
-                if (bin_of(ev, M) == bstar) {
-                    const unsigned long long kk = sel_key(ev, j);
-                    klo = kk < klo ? kk : klo;
-                    khi = kk > khi ? kk : khi;
-                }
-            }
+        if (found >= n) found = n - 1;
+        // set the bits of the boundary prefix (the words were written in pass 3)
+        for (int i = threadIdx.x; i <= found; i += blockDim.x) {
+            const uint32_t jk = (uint32_t)keys[i];
+            atomicOr(outw + (jk >> 5), 1u << (jk & 31));
         }
+        if (threadIdx.x == 0) s_found = found + 1;
+    } else {
+        // rare: too many candidates in one bin - bisection on the exact key order, then a pass
+        unsigned long long klo = ~0ull, khi = 0ull;
+        ZHA_FOR_WORDS({
+            if (valid && bin_of(ev, M) == bstar) {
+                const unsigned long long kk = sel_key(ev, j);
+                klo = kk < klo ? kk : klo;
+                khi = kk > khi ? kk : khi;
+            }
+        })
         unsigned long long lo = block_min_t<unsigned long long>(klo, red_u);
         unsigned long long hi = block_max_t<unsigned long long>(khi, red_u);
         int iters = 0;
         while (lo < hi && iters < 70) {
             const unsigned long long mid = lo + (hi - lo) / 2;
             unsigned long long acc = 0;
-            for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-                const int64_t j = wi * 32 + lane;
-                if (valid_at(j)) {
-                    const float ev = e[j];
-                    if (bin_of(ev, M) == bstar && sel_key(ev, j) <= mid) acc += mass_of(ev, M);
-                }
-            }
+            ZHA_FOR_WORDS({
+                if (valid && bin_of(ev, M) == bstar && sel_key(ev, j) <= mid) acc += mass_of(ev, M);
+            })
             acc = block_sum<unsigned long long>(acc, red_u);
             if (acc >= need) hi = mid;
             else lo = mid + 1;
             ++iters;
         }
-        if (threadIdx.x == 0) {
-            s_kstar = lo;
-            if (iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
-        }
+        if (threadIdx.x == 0 && iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
+        unsigned long long extra = 0;
+        ZHA_FOR_WORDS({
+            const bool keep = valid && bin_of(ev, M) == bstar && sel_key(ev, j) <= lo;
+            const unsigned bal = __ballot_sync(kFull, keep);
+            if (lane == 0 && bal) {
+                atomicOr(outw + wi, bal);
+                extra += __popc(bal);
+            }
+        })
+        extra = block_sum<unsigned long long>(extra, red_u);
+        if (threadIdx.x == 0) s_found = (int)extra;
     }
-    __syncthreads();
-    const unsigned long long kstar = s_kstar;
-
-    // pass 5: kept bitmap
-    unsigned long long cnt = 0;
-    for (int64_t wi = warp; wi < nwords; wi += nwarps) {
-        const int64_t j = wi * 32 + lane;
-        bool keep = false;
-        if (valid_at(j)) {
-            const float ev = e[j];
-            const int bn = bin_of(ev, M);
-            keep = bn < bstar || (bn == bstar && sel_key(ev, j) <= kstar);
-        }
-        const unsigned bal = __ballot_sync(kFull, keep);
-        if (lane == 0) {
-            outw[wi] = bal;
-            cnt += __popc(bal);
-        }
-    }
+#undef ZHA_FOR_WORDS
     cnt = block_sum<unsigned long long>(cnt, red_u);
-    if (threadIdx.x == 0) *kcount = (int32_t)cnt;
+    if (threadIdx.x == 0) *kcount = (int32_t)(cnt + (unsigned long long)s_found);
 }
 
 int score_blocks_x(int lane_blocks, int groups) {
