@@ -31,7 +31,7 @@ from hierarchical_tree_indexed_build_b200 import inputs  # noqa: E402
 
 METRIC = "ZHA decode queries/s at 256K & 1M ctx; achieved HBM GB/s vs peak"
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max SM clock
-TENSOR_KERNELS = {"k_score_tc": "tf32", "k_attn_tc": "bf16"}
+TENSOR_KERNELS = {"k_score_tc": "f16", "k_attn_tc": "bf16"}
 
 
 def parse():
@@ -58,14 +58,16 @@ def measured_peaks():
 
 
 def tensor_peak(dtype):
-    """Dense tensor peak for the kernel's MMA dtype: the measured bf16 burst figure, halved
-    for tf32 (kind::tf32 runs at half the bf16 rate)."""
+    """Dense tensor peak for the kernel's MMA dtype: the measured bf16 burst figure (fp16
+    runs at the bf16 rate, tf32 at half of it)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             bf16, src = json.load(f)["bf16_tflops"], "measured"
-    except Exception:
+    except (OSError, KeyError, ValueError):
         bf16, src = 1590.0, "fallback"
-    return (bf16 / 2 if dtype == "tf32" else bf16), "%s bf16 %s" % (src, "x 1/2 (tf32)" if dtype == "tf32" else "")
+    if dtype == "tf32":
+        return bf16 / 2, "%s bf16 x 1/2 (tf32)" % src
+    return bf16, "%s bf16%s" % (src, " (f16 runs at the bf16 rate)" if dtype == "f16" else "")
 
 
 class Clocks:

@@ -338,7 +338,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         s_cap = std::max<int64_t>(s_cap, (nseg_max + segs - 1) / segs);
     }
     w.lanes_cap = dec->lanes_cap;
-    w.es = (cap1 + 3) / 4 * 4;
+    w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
     w.us = cap1;
     w.s_cap = s_cap;
 
@@ -361,6 +361,10 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     off += up256((size_t)dec->groups_cap * w.uw * 4);
     const size_t part_off = off;
     off += up256((size_t)dec->lanes_cap * w.s_cap * (dec->d + 4) * 4);
+    const size_t lmax_off = off;
+    off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
+    const size_t lcnt_off = off;
+    off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
     const size_t ctr_off = off;
     off += up256((size_t)kCtrCount * 8);
     const size_t status_off = off;
@@ -381,6 +385,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.ucount = reinterpret_cast<int32_t*>(base + ucount_off);
     w.uword = reinterpret_cast<uint32_t*>(base + uword_off);
     w.part = reinterpret_cast<float*>(base + part_off);
+    w.lane_max = reinterpret_cast<uint32_t*>(base + lmax_off);
+    w.lane_cnt = reinterpret_cast<int32_t*>(base + lcnt_off);
     w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);
     w.status = reinterpret_cast<int32_t*>(base + status_off);
     dec->seq_dev = reinterpret_cast<SeqDev*>(base + seq_off);
@@ -460,6 +466,9 @@ extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, fl
         ZHA_CUDA(cudaMemsetAsync(dec->w.kept[l], 0, (size_t)b.n_lanes * dec->w.W[l] * 4, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.ctr, 0, (size_t)kCtrCount * 8, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.status, 0, 4, st));
+    // ordered-bits 0 is below every float; counts start at 0
+    ZHA_CUDA(cudaMemsetAsync(dec->w.lane_max, 0, (size_t)(kMaxL + 1) * dec->lanes_cap * 4, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.lane_cnt, 0, (size_t)(kMaxL + 1) * dec->lanes_cap * 4, st));
     const float scale = score_scale(dec->d);
     for (int it = 0; it < dec->Lmax; ++it) {
         if (it > 0) ZHA_CUDA(launch_union(b, dec->w, it, 0, st));

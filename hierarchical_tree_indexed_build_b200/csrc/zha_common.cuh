@@ -52,6 +52,8 @@ struct Work {
     int64_t uw;
     float* part;                     // [lanes_cap][s_cap][d+2] attention partials
     int64_t s_cap;
+    uint32_t* lane_max;              // [(kMaxL+1)][lanes_cap] frontier max score per lane (ordered bits)
+    int32_t* lane_cnt;               // [(kMaxL+1)][lanes_cap] frontier size per lane
     unsigned long long* ctr;         // kCtrCount counters
     int32_t* status;                 // device status word (0 = ok)
 };
@@ -75,10 +77,23 @@ __host__ __device__ inline int64_t lane_of(const Batch& b, int s, int g, int y) 
     return ((int64_t)s * b.n_q + i) * b.Hq + (int64_t)g * b.G + hh;
 }
 
+// Order-preserving map of a float to uint32 (atomicMax on the result is a float max).
+__host__ __device__ inline uint32_t ord_bits(float f) {
+    union { float f; uint32_t u; } c;
+    c.f = f;
+    return (c.u & 0x80000000u) ? ~c.u : (c.u | 0x80000000u);
+}
+__host__ __device__ inline float unord_bits(uint32_t o) {
+    union { float f; uint32_t u; } c;
+    c.u = (o & 0x80000000u) ? (o ^ 0x80000000u) : ~o;
+    return c.f;
+}
+
 // Device status bits.
 constexpr int32_t kStatusSelectFallbackLimit = 1;
 constexpr int32_t kStatusCapacity = 2;
 constexpr int32_t kStatusTimeout = 4;        // a bounded wait on the tensor-core pipeline gave up
+constexpr int32_t kStatusRange = 8;          // an entry of Q or of a summary exceeds the fp16 range
 
 // Split size (tokens) of the attention work for a call with n_gl lanes per group.
 inline __host__ __device__ int split_tokens(int n_gl) { return n_gl <= 64 ? 1024 : 4096; }

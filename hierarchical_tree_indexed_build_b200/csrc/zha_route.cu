@@ -255,6 +255,10 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
     const float* base = sq.rec[lev] + (int64_t)g * sq.cap[lev] * ns;
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     float* ex = w.e + x * w.es;
+    // the lane's kept set one level up decides which candidates are on its frontier
+    const uint32_t* Pb = top ? nullptr : w.kept[lev + 1] + x * w.W[lev + 1];
+    float fmax = -INFINITY;
+    int fcnt = 0;
     for (int64_t k = (int64_t)blockIdx.x * NPC + slot; k < nc; k += (int64_t)gridDim.x * NPC) {
         const int64_t j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
         const float* rec = base + j * ns;
@@ -274,31 +278,41 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
             dot += __shfl_xor_sync(kFull, dot, 2);
             best = fmaxf(best, fmaf(scale, dot, __ldg(rec + (int64_t)R * D + r)));
         }
-        if (lane_ok && q == 0) ex[j] = best;
+        if (lane_ok && q == 0) {
+            bool mb = true;
+            if (!top) {
+                const int64_t pj = j / C;
+                mb = (__ldg(Pb + (pj >> 5)) >> (pj & 31)) & 1u;
+            }
+            ex[j] = mb ? best : -INFINITY;
+            if (mb) {
+                fmax = fmaxf(fmax, best);
+                ++fcnt;
+            }
+        }
+    }
+    if (lane_ok && q == 0 && fcnt > 0) {
+        atomicMax(w.lane_max + (int64_t)lev * w.lanes_cap + x, ord_bits(fmax));
+        atomicAdd(w.lane_cnt + (int64_t)lev * w.lanes_cap + x, fcnt);
     }
 }
 
 // ----------------------------------------------------------------------------- select
 
 constexpr int kSelThreads = 512;
-constexpr int kNB = 4096;            // bins over (max e - e) * kBinScale
-constexpr float kBinScale = 128.0f;
-constexpr int kCap = 4096;           // boundary-bin candidates sorted in shared memory
-constexpr float kMassScale = 1099511627776.0f;   // 2^40: fixed-point masses, exact sums (<= 2^24 candidates)
+constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
+constexpr float kBinScale = 64.0f;
+constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
+constexpr int kUn = 4;               // 128-candidate blocks per warp in flight
+// 2^39: fixed-point masses; sums of <= 2^24 candidates stay below 2^63 and are exact
+constexpr float kMassScale = 549755813888.0f;
 
-__device__ __forceinline__ uint32_t ord_f32(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float unord_f32(uint32_t o) {
-    return __uint_as_float((o & 0x80000000u) ? (o ^ 0x80000000u) : ~o);
-}
 // Ascending key order == (e descending, node index ascending).
-__device__ __forceinline__ unsigned long long sel_key(float e, int64_t j) {
-    return ((unsigned long long)(~ord_f32(e)) << 32) | (unsigned long long)(uint32_t)j;
+__device__ __forceinline__ unsigned long long sel_key(float e, int j) {
+    return ((unsigned long long)(~ord_bits(e)) << 32) | (unsigned long long)(uint32_t)j;
 }
 __device__ __forceinline__ float key_score(unsigned long long k) {
-    return unord_f32(~(uint32_t)(k >> 32));
+    return unord_bits(~(uint32_t)(k >> 32));
 }
 __device__ __forceinline__ unsigned long long mass_of(float e, float M) {
     return (unsigned long long)(expf(e - M) * kMassScale);
@@ -308,13 +322,18 @@ __device__ __forceinline__ int bin_of(float e, float M) {
     return t >= (float)(kNB - 1) ? kNB - 1 : (int)t;
 }
 
-__global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it) {
+// One block per lane.  The scorer left, for every candidate of the lane's group (the
+// children of the group's union of kept nodes, or all top nodes), the plane estimate if
+// the candidate is on this lane's frontier and -inf otherwise, plus the lane's frontier
+// maximum M and size F.  Two passes over the candidates: a histogram of fixed-point masses
+// over bins of M - e, then the kept bits of the bins above the boundary bin and the
+// boundary bin's candidates, which are sorted by (e desc, j asc) to finish the prefix.
+__global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int it) {
     extern __shared__ unsigned long long sel_smem[];
-    unsigned long long* hist = sel_smem;                                    // [kNB]
-    unsigned long long* keys = hist + kNB;                                  // [kCap]
-    unsigned int* hcnt = reinterpret_cast<unsigned int*>(keys + kCap);      // [kNB]
+    unsigned long long* hist = sel_smem;   // [kNB]
+    unsigned long long* keys = hist + kNB; // [kCap]
     __shared__ unsigned long long red_u[33];
-    __shared__ float red_f[33];
+    __shared__ int red_i[33];
     __shared__ int s_bstar;
     __shared__ unsigned long long s_cumb;
     __shared__ unsigned int s_nkeys;
@@ -322,167 +341,186 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
 
     const int64_t x = blockIdx.x;
     const int s = (int)(x / ((int64_t)b.n_q * b.Hq));
+    const int g = (int)(x % b.Hq) / b.G;
+    const int grp = s * b.Hkv + g;
     const SeqDev& sq = b.seqs[s];
     const int lev = sq.L - it;
     if (lev < 1) return;
-    const int64_t nl = sq.n[lev];
     int32_t* kcount = w.kcount + (int64_t)lev * w.lanes_cap + x;
-    if (nl == 0) {
-        if (threadIdx.x == 0) *kcount = 0;
-        return;
-    }
-    const bool top = (lev == sq.L);
-    const int64_t C = sq.C;
-    const uint32_t* P = top ? nullptr : w.kept[lev + 1] + x * w.W[lev + 1];
-    const float* e = w.e + x * w.es;
-    uint32_t* outw = w.kept[lev] + x * w.W[lev];
-    const int64_t nwords = (nl + 31) / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    const int64_t np1 = top ? 0 : sq.n[lev + 1];   // complete parents
-
-    // Candidate j = 32 wi + lane: its score and whether it is on the lane's frontier (a child
-    // of a kept complete parent).  Both loads are issued unconditionally and independently so
-    // a warp keeps several words in flight; scores off the frontier are never used.
-    auto fetch = [&](int64_t wi, float& ev, bool& v) {
-        const int64_t j = wi * 32 + lane;
-        const bool in = j < nl;
-        const int64_t jj = in ? j : nl - 1;
-        ev = e[jj];
-        if (top) {
-            v = in;
-        } else {
-            const int64_t pj = jj / C;
-            const uint32_t pw = __ldg(P + (min(pj, np1 > 0 ? np1 - 1 : 0) >> 5));
-            v = in && pj < np1 && ((pw >> (pj & 31)) & 1u);
-        }
-    };
-    constexpr int kUn = 4;   // words per warp in flight
-#define ZHA_FOR_WORDS(BODY)                                                                  \
-    for (int64_t w0 = warp; w0 < nwords; w0 += kUn * nwarps) {                               \
-        float ev_[kUn];                                                                      \
-        bool v_[kUn];                                                                        \
-        _Pragma("unroll") for (int u = 0; u < kUn; ++u) {                                    \
-            const int64_t wi_ = w0 + (int64_t)u * nwarps;                                    \
-            v_[u] = false;                                                                   \
-            ev_[u] = 0.0f;                                                                   \
-            if (wi_ < nwords) fetch(wi_, ev_[u], v_[u]);                                     \
-        }                                                                                    \
-        _Pragma("unroll") for (int u = 0; u < kUn; ++u) {                                    \
-            const int64_t wi = w0 + (int64_t)u * nwarps;                                     \
-            if (wi >= nwords) break;                                                         \
-            const int64_t j = wi * 32 + lane;                                                \
-            const float ev = ev_[u];                                                         \
-            const bool valid = v_[u];                                                        \
-            BODY                                                                             \
-        }                                                                                    \
-    }
-
-    // pass 1: frontier max and size
-    float mloc = -INFINITY;
-    unsigned long long floc = 0;
-    ZHA_FOR_WORDS({
-        (void)j;
-        if (valid) {
-            mloc = fmaxf(mloc, ev);
-            ++floc;
-        }
-    })
-    const float M = block_max(mloc, red_f);
-    const unsigned long long F = block_sum<unsigned long long>(floc, red_u);
-    if (threadIdx.x == 0) atomicAdd(&w.ctr[kCtrLaneNodes + lev], F);
+    const int64_t F = w.lane_cnt[(int64_t)lev * w.lanes_cap + x];
+    if (threadIdx.x == 0) atomicAdd(&w.ctr[kCtrLaneNodes + lev], (unsigned long long)F);
     if (F == 0) {
         if (threadIdx.x == 0) *kcount = 0;
         return;
     }
-    if (b.p >= 1.0f) {
-        ZHA_FOR_WORDS({
-            (void)j;
-            (void)ev;
-            const unsigned bal = __ballot_sync(kFull, valid);
-            if (lane == 0) outw[wi] = bal;
-        })
-        if (threadIdx.x == 0) *kcount = (int32_t)F;
+    const float M = unord_bits(w.lane_max[(int64_t)lev * w.lanes_cap + x]);
+    const bool top = (lev == sq.L);
+    const int C = sq.C;
+    // candidate and node indices are < 2^24 (level-1 nodes are capped there): 32-bit math
+    const int nc = (int)(top ? sq.T : (int64_t)w.ucount[grp] * C);
+    const int32_t* ul = w.ulist + (int64_t)grp * w.us;
+    // candidates 4k..4k+3 are 4 consecutive, 4-aligned nodes
+    const bool contig = top || (C % 4 == 0);
+    const float* e = w.e + x * w.es;
+    uint32_t* outw = w.kept[lev] + x * w.W[lev];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int nblk = (nc + 127) / 128;
+
+    // candidate k -> node index
+    auto cand_j = [&](int k) -> int {
+        if (top) return k;
+        const uint32_t pk = (uint32_t)k / (uint32_t)C;
+        return __ldg(ul + pk) * C + (k - (int)pk * C);
+    };
+    // scores of candidates k0..k0+3 (k0 = 128 bk + 4 lane); -inf past the end
+    auto load = [&](int bk, float4& ev, int& j0) {
+        const int k0 = bk * 128 + 4 * lane;
+        ev = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        j0 = -1;
+        if (k0 >= nc) return;
+        j0 = cand_j(k0);
+        if (contig) {
+            ev = *reinterpret_cast<const float4*>(e + j0);   // rows are padded to 128 floats
+            if (k0 + 1 >= nc) ev.y = -INFINITY;
+            if (k0 + 2 >= nc) ev.z = -INFINITY;
+            if (k0 + 3 >= nc) ev.w = -INFINITY;
+        } else {
+            ev.x = e[j0];
+            if (k0 + 1 < nc) ev.y = e[cand_j(k0 + 1)];
+            if (k0 + 2 < nc) ev.z = e[cand_j(k0 + 2)];
+            if (k0 + 3 < nc) ev.w = e[cand_j(k0 + 3)];
+        }
+    };
+    auto jof = [&](int bk, int j0, int c) -> int {
+        return contig ? j0 + c : cand_j(bk * 128 + 4 * lane + c);
+    };
+    // every warp visits its blocks with kUn loads in flight; body(bk, scores[4], j0)
+    auto for_cands = [&](auto&& body) {
+        for (int b0 = warp; b0 < nblk; b0 += kUn * nwarps) {
+            float4 ev[kUn];
+            int j0[kUn];
+#pragma unroll
+            for (int u = 0; u < kUn; ++u) load(b0 + u * nwarps, ev[u], j0[u]);
+#pragma unroll
+            for (int u = 0; u < kUn; ++u) {
+                const int bk = b0 + u * nwarps;
+                if (bk >= nblk) break;
+                body(bk, ev[u], j0[u]);
+            }
+        }
+    };
+    // kept bits of candidates k0..k0+3 (nibble) into the bitmap: one plain store per
+    // 32-candidate word when the warp's 8-lane group covers a whole aligned word (the
+    // bitmap starts zeroed), else atomics
+    auto put_bits = [&](int bk, uint32_t nib, int j0) {
+        if (contig) {
+            const int jf = __shfl_sync(kFull, j0, lane & ~7);
+            const int jl = __shfl_sync(kFull, j0, lane | 7);
+            uint32_t wv = nib << (4 * (lane & 7));
+            wv |= __shfl_xor_sync(kFull, wv, 1);
+            wv |= __shfl_xor_sync(kFull, wv, 2);
+            wv |= __shfl_xor_sync(kFull, wv, 4);
+            if (jf >= 0 && (jf & 31) == 0 && jl == jf + 28) {
+                if ((lane & 7) == 0 && wv) outw[jf >> 5] = wv;
+            } else if (nib) {
+                atomicOr(outw + (j0 >> 5), nib << (j0 & 31));
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if ((nib >> c) & 1u) {
+                    const int j = jof(bk, j0, c);
+                    atomicOr(outw + (j >> 5), 1u << (j & 31));
+                }
+        }
+    };
+
+    int bstar = kNB;               // bins < bstar are kept whole
+    unsigned long long need = 0;   // mass still needed from the boundary bin
+    if (b.p < 1.0f) {
+        // pass 1: fixed-point masses into bins of (M - e)
+        for (int i = threadIdx.x; i < kNB; i += blockDim.x) hist[i] = 0ull;
+        if (threadIdx.x == 0) s_nkeys = 0;
+        __syncthreads();
+        for_cands([&](int bk, const float4 ev4, int j0) {
+        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (v[c] > -INFINITY) atomicAdd(&hist[bin_of(v[c], M)], mass_of(v[c], M));
+        });
+        __syncthreads();
+        unsigned long long zloc = 0;
+        for (int i = threadIdx.x; i < kNB; i += blockDim.x) zloc += hist[i];
+        const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
+        unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
+        if (target < 1ull) target = 1ull;
+        if (target > Z) target = Z;
+        // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
+        if (warp == 0) {
+            constexpr int per = kNB / 32;
+            unsigned long long ls = 0;
+#pragma unroll 4
+            for (int k = 0; k < per; ++k) ls += hist[lane * per + k];
+            unsigned long long incl = ls;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long t = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const unsigned long long excl = incl - ls;
+            const unsigned bal = __ballot_sync(kFull, excl < target && target <= incl);
+            const int src = bal ? __ffs(bal) - 1 : 31;
+            if (lane == src) {
+                unsigned long long cum = excl;
+                int bs = lane * per + per - 1;
+#pragma unroll 1
+                for (int k = 0; k < per; ++k) {
+                    const int bb = lane * per + k;
+                    if (cum + hist[bb] >= target) {
+                        bs = bb;
+                        break;
+                    }
+                    cum += hist[bb];
+                }
+                s_bstar = bs;
+                s_cumb = cum;
+            }
+        }
+        __syncthreads();
+        bstar = s_bstar;
+        need = target - s_cumb;
+    }
+
+    // pass 2: kept bits of the bins above the boundary; boundary-bin candidates collected
+    unsigned long long cnt = 0;
+    for_cands([&](int bk, const float4 ev4, int j0) {
+        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+        uint32_t nib = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (!(v[c] > -INFINITY)) continue;
+            const int bn = bin_of(v[c], M);
+            if (bn < bstar) {
+                nib |= 1u << c;
+            } else if (bn == bstar) {
+                const unsigned idx = atomicAdd(&s_nkeys, 1u);
+                if (idx < (unsigned)kCap) keys[idx] = sel_key(v[c], jof(bk, j0, c));
+            }
+        }
+        cnt += __popc(nib);
+        put_bits(bk, nib, j0);
+    });
+    cnt = block_sum<unsigned long long>(cnt, red_u);
+    if (bstar == kNB) {
+        if (threadIdx.x == 0) *kcount = (int32_t)cnt;
         return;
     }
-
-    // pass 2: fixed-point masses, total, histogram over bins of (M - e)
-    for (int i = threadIdx.x; i < kNB; i += blockDim.x) {
-        hist[i] = 0ull;
-        hcnt[i] = 0u;
-    }
-    __syncthreads();
-    unsigned long long zloc = 0;
-    ZHA_FOR_WORDS({
-        (void)j;
-        if (valid) {
-            const unsigned long long u = mass_of(ev, M);
-            zloc += u;
-            const int bn = bin_of(ev, M);
-            atomicAdd(&hist[bn], u);
-            atomicAdd(&hcnt[bn], 1u);
-        }
-    })
-    const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
-    unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
-    if (target < 1ull) target = 1ull;
-    if (target > Z) target = Z;
-
-    // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
-    if (warp == 0) {
-        constexpr int per = kNB / 32;
-        unsigned long long ls = 0;
-        for (int k = 0; k < per; ++k) ls += hist[lane * per + k];
-        unsigned long long incl = ls;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long t = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const unsigned long long excl = incl - ls;
-        const unsigned bal = __ballot_sync(kFull, excl < target && target <= incl);
-        const int src = bal ? __ffs(bal) - 1 : 31;
-        if (lane == src) {
-            unsigned long long cum = excl;
-            int bs = lane * per + per - 1;
-            for (int k = 0; k < per; ++k) {
-                const int bb = lane * per + k;
-                if (cum + hist[bb] >= target) {
-                    bs = bb;
-                    break;
-                }
-                cum += hist[bb];
-            }
-            s_bstar = bs;
-            s_cumb = cum;
-        }
-        if (threadIdx.x == 0) s_nkeys = 0;
-    }
-    __syncthreads();
-    const int bstar = s_bstar;
-    const unsigned long long need = target - s_cumb;
-    const unsigned nb = hcnt[bstar];
-    const bool collect = nb <= (unsigned)kCap;
-
-    // pass 3: kept bitmap for bins above the boundary; boundary-bin candidates collected
-    unsigned long long cnt = 0;
-    ZHA_FOR_WORDS({
-        bool keep = false;
-        if (valid) {
-            const int bn = bin_of(ev, M);
-            keep = bn < bstar;
-            if (bn == bstar && collect) keys[atomicAdd(&s_nkeys, 1u)] = sel_key(ev, j);
-        }
-        const unsigned bal = __ballot_sync(kFull, keep);
-        if (lane == 0) {
-            outw[wi] = bal;
-            cnt += __popc(bal);
-        }
-    })
     __syncthreads();
 
-    if (collect) {
+    const unsigned nkeys = s_nkeys;
+    if (nkeys <= (unsigned)kCap) {
         // sort the boundary bin by (e desc, j asc) and take the prefix reaching the target
-        const int n = (int)s_nkeys;
+        const int n = (int)nkeys;
         int npow = 1;
         while (npow < n) npow <<= 1;
         for (int i = threadIdx.x; i < npow; i += blockDim.x)
@@ -518,10 +556,8 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
                 break;
             }
         }
-        __syncthreads();
-        found = block_min_t<int>(found, reinterpret_cast<int*>(red_f));
+        found = block_min_t<int>(found, red_i);
         if (found >= n) found = n - 1;
-        // set the bits of the boundary prefix (the words were written in pass 3)
         for (int i = threadIdx.x; i <= found; i += blockDim.x) {
             const uint32_t jk = (uint32_t)keys[i];
             atomicOr(outw + (jk >> 5), 1u << (jk & 31));
@@ -530,22 +566,29 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
     } else {
         // rare: too many candidates in one bin - bisection on the exact key order, then a pass
         unsigned long long klo = ~0ull, khi = 0ull;
-        ZHA_FOR_WORDS({
-            if (valid && bin_of(ev, M) == bstar) {
-                const unsigned long long kk = sel_key(ev, j);
-                klo = kk < klo ? kk : klo;
-                khi = kk > khi ? kk : khi;
-            }
-        })
+        for_cands([&](int bk, const float4 ev4, int j0) {
+        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (v[c] > -INFINITY && bin_of(v[c], M) == bstar) {
+                    const unsigned long long kk = sel_key(v[c], jof(bk, j0, c));
+                    klo = kk < klo ? kk : klo;
+                    khi = kk > khi ? kk : khi;
+                }
+        });
         unsigned long long lo = block_min_t<unsigned long long>(klo, red_u);
         unsigned long long hi = block_max_t<unsigned long long>(khi, red_u);
         int iters = 0;
         while (lo < hi && iters < 70) {
             const unsigned long long mid = lo + (hi - lo) / 2;
             unsigned long long acc = 0;
-            ZHA_FOR_WORDS({
-                if (valid && bin_of(ev, M) == bstar && sel_key(ev, j) <= mid) acc += mass_of(ev, M);
-            })
+            for_cands([&](int bk, const float4 ev4, int j0) {
+        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (v[c] > -INFINITY && bin_of(v[c], M) == bstar && sel_key(v[c], jof(bk, j0, c)) <= mid)
+                        acc += mass_of(v[c], M);
+            });
             acc = block_sum<unsigned long long>(acc, red_u);
             if (acc >= need) hi = mid;
             else lo = mid + 1;
@@ -553,19 +596,22 @@ __global__ void __launch_bounds__(kSelThreads) k_select(Batch b, Work w, int it)
         }
         if (threadIdx.x == 0 && iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
         unsigned long long extra = 0;
-        ZHA_FOR_WORDS({
-            const bool keep = valid && bin_of(ev, M) == bstar && sel_key(ev, j) <= lo;
-            const unsigned bal = __ballot_sync(kFull, keep);
-            if (lane == 0 && bal) {
-                atomicOr(outw + wi, bal);
-                extra += __popc(bal);
-            }
-        })
+        for_cands([&](int bk, const float4 ev4, int j0) {
+        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (v[c] > -INFINITY && bin_of(v[c], M) == bstar) {
+                    const int j = jof(bk, j0, c);
+                    if (sel_key(v[c], j) <= lo) {
+                        atomicOr(outw + (j >> 5), 1u << (j & 31));
+                        ++extra;
+                    }
+                }
+        });
         extra = block_sum<unsigned long long>(extra, red_u);
         if (threadIdx.x == 0) s_found = (int)extra;
     }
-#undef ZHA_FOR_WORDS
-    cnt = block_sum<unsigned long long>(cnt, red_u);
+    __syncthreads();
     if (threadIdx.x == 0) *kcount = (int32_t)(cnt + (unsigned long long)s_found);
 }
 
@@ -603,7 +649,7 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
 }
 
 cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st) {
-    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8 + (size_t)kNB * 4;
+    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8;
     cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     ProfScope ps_("k_select", st);
     k_select<<<b.n_lanes, kSelThreads, smem, st>>>(b, w, it);

@@ -2,21 +2,27 @@
 //
 // Same quantity as k_score (fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的:
 // 取这些平面的最大值; wqu.guru, section "Building the tree"): for every lane of a
-// (sequence, KV head) group and every candidate node j,
-//     e_j = max_r ( s q.m_r(j) + b_r(j) ).
-// When a group holds many lanes (many query tokens x GQA heads) this is a dense
-// contraction D[lane][(node, r)] = sum_k Q[lane][k] m_r(j)[k], run here as
-// tcgen05.mma kind::tf32 with M = 128 lanes, N = 8 nodes x 16 planes, K = d, fp32
-// accumulators in tensor memory.
+// (sequence, KV head) group and every candidate node j on the lane's frontier,
+//     e_j = max_r ( s q.m_r(j) + b_r(j) ),
+// and -inf for candidates off the lane's frontier (children of nodes other lanes kept).
+// When a group holds many lanes (query tokens x GQA heads) this is a dense contraction
+// D[lane][(node, r)] = sum_k Q[lane][k] m_r(j)[k], run here as tcgen05.mma kind::f16 with
+// M = 128 lanes, N = 8 nodes x 16 planes, K = d, f32 accumulators in tensor memory.
 //
-// Precision: Q is bf16, hence exact in tf32.  The f32 summary m is split into
-// hi = m with its 13 low mantissa bits cleared (exact tf32) and lo = m - hi (exact in
-// f32); two MMA passes accumulate Q.hi + Q.lo, leaving a relative error of about 2^-22
-// on m (the truncation of lo) - float32-grade scores.
+// Precision: Q is bf16, which fp16 holds exactly for magnitudes in [2^-17, 65504).  The
+// f32 summary m is split into two fp16 terms m = hi + lo (lo the fp16 rounding of m - hi),
+// so two MMA passes accumulate Q.m with an error of at most 2^-22 |m| + 2^-25 per
+// element: float32-grade scores.  An entry of Q or m of magnitude >= 65504 does not fit;
+// the kernel then sets kStatusRange (the CUDA-core scorer has no such limit).
 //
-// Shared-memory operands use the canonical K-major 128-byte-swizzle layout: per K block
-// of 32 f32, rows are 128 bytes apart, the 16-byte chunk c of row r sits at chunk
-// c ^ (r % 8), 8-row groups are 1024 bytes apart (the descriptor's stride byte offset).
+// Pipeline (one CTA per SM, persistent over its node tiles):
+//   warps 0-7   producers: load a node tile (f32), split into the two fp16 planes, store
+//               them in a 128-byte-swizzled K-major shared-memory stage (2 stages);
+//   warps 8-11  epilogue: tensor memory -> max over planes + b -> scores; lane 0 of warp 8
+//               also issues the MMAs of the next tile into the other TMEM accumulator.
+// Shared-memory operand layout: per K block of 64 bf16, rows are 128 bytes apart, the
+// 16-byte chunk c of row r sits at chunk c ^ (r % 8), 8-row groups 1024 bytes apart.
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "zha_common.cuh"
@@ -28,14 +34,17 @@ namespace zha {
 namespace {
 
 constexpr int kTileM = 128;          // lanes per tile (MMA M)
-constexpr int kTileN = 64;           // rows (node, plane) per tile (MMA N)
+constexpr int kTileN = 128;          // rows (node, plane) per tile (MMA N)
 constexpr int kR = 16;               // planes per node on this path
 constexpr int kNodes = kTileN / kR;  // nodes per tile
-constexpr int kProducers = 256;      // warps 0-7: load, split, stage
-constexpr int kEpilogue = 128;       // warps 8-11: TMEM -> scores; lane 0 of warp 8 issues the MMAs
+constexpr int kProducers = 256;      // warps 0-7
+constexpr int kEpilogue = 128;       // warps 8-11
 constexpr int kThreads = kProducers + kEpilogue;
-constexpr int kMmaWarp = kProducers / 32;   // also allocates tensor memory
-constexpr int kRing = 3;             // node tiles whose loads each producer keeps in flight
+constexpr int kMmaWarp = kProducers / 32;   // first epilogue warp: issues MMAs, owns TMEM
+constexpr int kRing = 2;             // node tiles whose loads each producer keeps in flight
+constexpr int kChunk = kProducers / kNodes;   // tiles whose node ids are staged at once
+constexpr int kPlanes = 2;           // fp16 terms of m
+constexpr float kHalfMax = 65504.0f; // largest finite fp16
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -53,15 +62,14 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: kind::tf32, f32 accumulate, A and B K-major, M x N.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kTileN >> 3) << 17) |
-                            ((uint32_t)(kTileM >> 4) << 24);
+// Instruction descriptor: kind::f16 with fp16 A/B, f32 accumulate, both K-major, M x N.
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
 
-__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t acc) {
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(acc));
 }
@@ -111,23 +119,34 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Byte offset of (row, 16-byte chunk c of K block kb) in a [KB][rows][128 B] tile.
-__device__ __forceinline__ uint32_t swz(int kb, int rows, int row, int c) {
-    return (uint32_t)(kb * (rows * 128) + row * 128 + ((c ^ (row & 7)) << 4));
+// Byte offset of element d (16-bit) of row `row` in a K-major tile of 128-row, 128-byte blocks.
+__device__ __forceinline__ uint32_t swz16(int row, int d) {
+    const int kb = d >> 6, c = (d & 63) >> 3;
+    return (uint32_t)(kb * (128 * 128) + row * 128 + ((c ^ (row & 7)) << 4) + (d & 7) * 2);
+}
+
+// m = hi + lo, hi the fp16 rounding of m and lo that of m - hi; two elements per word.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int it, float scale) {
-    constexpr int KB = D / 32;                        // 128-byte K blocks
+    constexpr int KB = D / 64;                        // 128-byte K blocks of 16-bit elements
     constexpr int A_BYTES = KB * kTileM * 128;
-    constexpr int B_BYTES = KB * kTileN * 128;        // one plane of one stage
+    constexpr int P_BYTES = KB * kTileN * 128;        // one fp16 plane of one stage
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sA = base;
-    unsigned char* sB0 = base + A_BYTES;                                  // [2 stages][hi, lo][B_BYTES]
-    float* sBv = reinterpret_cast<float*>(sB0 + 4 * B_BYTES);            // [2][kTileN] b values
+    unsigned char* sB0 = base + A_BYTES;                                  // [2 stages][2 planes][P_BYTES]
+    float* sBv = reinterpret_cast<float*>(sB0 + 2 * kPlanes * P_BYTES);   // [2][kTileN] b values
     int64_t* sJ = reinterpret_cast<int64_t*>(sBv + 2 * kTileN);          // [2][kNodes] node ids (-1: none)
+    int32_t* sNode = reinterpret_cast<int32_t*>(sJ + 2 * kNodes);        // [2][kChunk * kNodes] staged ids
     __shared__ __align__(8) uint64_t bar_full[2], bar_acc_full[2], bar_acc_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -163,19 +182,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
         asm volatile("fence.mbarrier_init.release.cluster;");
         abort_sh = 0;
     }
-    // A: the tile's query rows as f32 (exact), zero rows past the group's lanes.
-    for (int i = tid; i < kTileM * (D / 4); i += kThreads) {
-        const int row = i / (D / 4), c4 = i % (D / 4);
+    // A: the tile's query rows (bf16 -> fp16, exact in range), zero rows past the group's lanes.
+    float amax = 0.0f;
+    for (int i = tid; i < kTileM * (D / 8); i += kThreads) {
+        const int row = i / (D / 8), c16 = i % (D / 8);
         const int y = y0 + row;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (y < b.n_gl) {
-            const uint2 u = __ldg(reinterpret_cast<const uint2*>(b.Q + lane_of(b, s, g, y) * D) + c4);
-            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-            const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-            v = make_float4(a0.x, a0.y, a1.x, a1.y);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (y < b.n_gl) v = __ldg(reinterpret_cast<const uint4*>(b.Q + lane_of(b, s, g, y) * D) + c16);
+        uint32_t hv[4];
+        const uint32_t* bv = &v.x;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(bv + t));
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            const __half2 h = __floats2half2_rn(f.x, f.y);
+            hv[t] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        *reinterpret_cast<float4*>(sA + swz(c4 / 8, kTileM, row, c4 % 8)) = v;
+        *reinterpret_cast<uint4*>(sA + swz16(row, c16 * 8)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
+    if (!(amax < kHalfMax)) atomicOr(w.status, kStatusRange);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -192,24 +217,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
     };
 
     if (warp < kProducers / 32) {
-        // ---------------- producers: rows of node tiles -> tf32 hi / f32 lo, swizzled.
-        // Each thread keeps the loads of kRing tiles in flight (register ring, static slots).
+        // ---------------- producers
         constexpr int kRowStep = kProducers / (D / 4);
-        constexpr int kU = kTileN / kRowStep;
+        constexpr int kU = kTileN / kRowStep;         // float4 per thread per tile
         const int c4 = tid % (D / 4);
         const int row0 = tid / (D / 4);
+        float mmax = 0.0f;   // largest |m| this thread split
+        // Node ids of chunk c (tiles [c kChunk, (c+1) kChunk) of this block) into sNode[c & 1]:
+        // one independent load per producer thread, so no tile waits on a dependent load.
+        auto fill_chunk = [&](int64_t c) {
+            const int64_t i = c * kChunk + tid / kNodes;
+            int32_t j = -1;
+            if (i < nt) j = (int32_t)node_of(blockIdx.x + i * gridDim.x, tid % kNodes);
+            sNode[(c & 1) * kProducers + tid] = j;
+        };
+        auto node_at = [&](int64_t i, int nl) -> int64_t {
+            return sNode[((i / kChunk) & 1) * kProducers + (i % kChunk) * kNodes + nl];
+        };
         auto prefetch = [&](int64_t i, float4 (&pre)[kU], float& preb, int64_t& prej) {
             if (i >= nt) return;
-            const int64_t t = blockIdx.x + i * gridDim.x;
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int row = row0 + u * kRowStep;
-                const int64_t j = node_of(t, row / kR);
+                const int64_t j = node_at(i, row / kR);
                 pre[u] = j >= 0 ? __ldg(reinterpret_cast<const float4*>(recb + j * ns + (int64_t)(row % kR) * D) + c4)
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             if (tid < kTileN) {
-                prej = node_of(t, tid / kR);
+                prej = node_at(i, tid / kR);
                 preb = prej >= 0 ? __ldg(recb + prej * ns + (int64_t)kR * D + tid % kR) : 0.0f;
             }
         };
@@ -217,26 +252,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
         auto step = [&](int64_t i, float4 (&pre)[kU], float& preb, int64_t& prej) -> bool {
             if (i >= nt) return false;
             const int st = (int)(i & 1);
-            // stage st (and its b / node ids) is free once the epilogue of tile i-2 is done
-            if (i >= 2 && !mbar_wait(smem_u32(&bar_acc_empty[st]), (uint32_t)(((i >> 1) - 1) & 1))) {
+            // stage st (and its b / node ids) is free once the epilogue of tile i-2 is done.
+            // After an abort the producers keep stepping without waiting, so that all of them
+            // reach the same named barriers.
+            if (i >= 2 && !abort_sh && !mbar_wait(smem_u32(&bar_acc_empty[st]), (uint32_t)(((i >> 1) - 1) & 1))) {
                 atomicOr(w.status, kStatusTimeout);
                 abort_sh = 1;
             }
-            if (abort_sh) return false;
-            unsigned char* hiB = sB0 + (2 * st) * B_BYTES;
-            unsigned char* loB = hiB + B_BYTES;
+            unsigned char* pl = sB0 + (size_t)(kPlanes * st) * P_BYTES;
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int row = row0 + u * kRowStep;
                 const float4 m = pre[u];
-                float4 hi, lo;
-                hi.x = __uint_as_float(__float_as_uint(m.x) & 0xFFFFE000u); lo.x = m.x - hi.x;
-                hi.y = __uint_as_float(__float_as_uint(m.y) & 0xFFFFE000u); lo.y = m.y - hi.y;
-                hi.z = __uint_as_float(__float_as_uint(m.z) & 0xFFFFE000u); lo.z = m.z - hi.z;
-                hi.w = __uint_as_float(__float_as_uint(m.w) & 0xFFFFE000u); lo.w = m.w - hi.w;
-                const uint32_t off = swz(c4 / 8, kTileN, row, c4 % 8);
-                *reinterpret_cast<float4*>(hiB + off) = hi;
-                *reinterpret_cast<float4*>(loB + off) = lo;
+                mmax = fmaxf(mmax, fmaxf(fmaxf(fabsf(m.x), fabsf(m.y)), fmaxf(fabsf(m.z), fabsf(m.w))));
+                uint32_t h0, l0, h1, l1;
+                split2(m.x, m.y, h0, l0);
+                split2(m.z, m.w, h1, l1);
+                const uint32_t off = swz16(row, c4 * 4);
+                *reinterpret_cast<uint2*>(pl + off) = make_uint2(h0, h1);
+                *reinterpret_cast<uint2*>(pl + P_BYTES + off) = make_uint2(l0, l1);
             }
             if (tid < kTileN) {
                 sBv[st * kTileN + tid] = preb;
@@ -244,20 +278,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(smem_u32(&bar_full[st]));
+            // tile i + kRing may open the next chunk: stage its node ids one chunk ahead
+            if ((i + kRing) % kChunk == 0 && i + kRing < nt) {
+                asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");   // old ids of that buffer consumed
+                fill_chunk((i + kRing) / kChunk + 1);
+            }
+            if ((i + kRing) % kChunk == 0)
+                asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");   // new ids visible
             prefetch(i + kRing, pre, preb, prej);
             return true;
         };
-        float4 p0[kU], p1[kU], p2[kU];
-        float b0 = 0.f, b1 = 0.f, b2 = 0.f;
-        int64_t j0 = -1, j1 = -1, j2 = -1;
+        fill_chunk(0);
+        fill_chunk(1);
+        asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");
+        float4 p0[kU], p1[kU];
+        float b0 = 0.f, b1 = 0.f;
+        int64_t j0 = -1, j1 = -1;
         prefetch(0, p0, b0, j0);
         prefetch(1, p1, b1, j1);
-        prefetch(2, p2, b2, j2);
         for (int64_t i = 0; i < nt; i += kRing) {
             if (!step(i, p0, b0, j0)) break;
             if (!step(i + 1, p1, b1, j1)) break;
-            if (!step(i + 2, p2, b2, j2)) break;
         }
+        if (!(mmax < kHalfMax)) atomicOr(w.status, kStatusRange);
     } else {
         // ---------------- epilogue: scores of tile i from accumulator i % 2.  Lane 0 of the
         // first epilogue warp issues tile i+1's MMAs before this warp drains tile i.
@@ -267,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
         const bool ok = y < b.n_gl;
         const int64_t x = lane_of(b, s, g, ok ? y : 0);
         float* ex = w.e + x * w.es;
+        // the lane's kept set one level up decides which candidates are on its frontier
+        const uint32_t* Pb = top ? nullptr : w.kept[lev + 1] + x * w.W[lev + 1];
+        float fmax = -INFINITY;
+        int fcnt = 0;
         const bool issuer = warp == kMmaWarp && lane == 0;
         const uint32_t a0 = smem_u32(sA);
         auto issue = [&](int64_t i) {
@@ -280,17 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
             if (abort_sh) return;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t d = tmem + (uint32_t)(st * kTileN);
-            const uint32_t h0 = smem_u32(sB0 + (2 * st) * B_BYTES), l0 = h0 + B_BYTES;
+            const uint32_t pl0 = smem_u32(sB0 + (size_t)(kPlanes * st) * P_BYTES);
 #pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
-                const uint32_t b0 = pass == 0 ? h0 : l0;
+            for (int pass = 0; pass < kPlanes; ++pass)
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_tf32(d, umma_desc(a0 + kb * (kTileM * 128) + kk * 32),
-                                 umma_desc(b0 + kb * (kTileN * 128) + kk * 32), (pass | kb | kk) ? 1u : 0u);
-            }
+                        mma_f16(d, umma_desc(a0 + kb * (kTileM * 128) + kk * 32),
+                                 umma_desc(pl0 + pass * P_BYTES + kb * (kTileN * 128) + kk * 32),
+                                 (pass | kb | kk) ? 1u : 0u);
             mma_commit(smem_u32(&bar_acc_full[st]));
         };
         if (issuer) issue(0);
@@ -302,8 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
                 atomicOr(w.status, kStatusTimeout);
                 abort_sh = 1;
             }
-            if (abort_sh) break;
+            if (__any_sync(0xffffffffu, abort_sh != 0)) break;   // warp-uniform: tcgen05.ld below is collective
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            uint32_t member = 0;
+#pragma unroll
+            for (int nl = 0; nl < kNodes; ++nl) {
+                const int64_t j = sJ[st * kNodes + nl];
+                bool mb = j >= 0;
+                if (mb && !top) {
+                    const int64_t pj = j / C;
+                    mb = (__ldg(Pb + (pj >> 5)) >> (pj & 31)) & 1u;
+                }
+                member |= (mb ? 1u : 0u) << nl;
+            }
 #pragma unroll
             for (int nl = 0; nl < kNodes; ++nl) {
                 float v[16];
@@ -312,10 +369,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
 #pragma unroll
                 for (int r = 0; r < kR; ++r) best = fmaxf(best, fmaf(scale, v[r], sBv[st * kTileN + nl * kR + r]));
                 const int64_t j = sJ[st * kNodes + nl];
-                if (ok && j >= 0) ex[j] = best;
+                const bool mb = (member >> nl) & 1u;
+                if (ok && j >= 0) ex[j] = mb ? best : -INFINITY;
+                if (mb) {
+                    fmax = fmaxf(fmax, best);
+                    ++fcnt;
+                }
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             mbar_arrive(smem_u32(&bar_acc_empty[st]));
+        }
+        if (ok && fcnt > 0) {
+            atomicMax(w.lane_max + (int64_t)lev * w.lanes_cap + x, ord_bits(fmax));
+            atomicAdd(w.lane_cnt + (int64_t)lev * w.lanes_cap + x, fcnt);
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -328,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_score_tc(Batch b, Work w, int i
 }  // namespace
 
 size_t score_tc_smem(int d) {
-    return (size_t)(d / 32) * 128 * (kTileM + 4 * kTileN) + 2 * kTileN * 4 + 2 * kNodes * 8 + 1024;
+    return (size_t)(d / 64) * 128 * 128 * (1 + 2 * kPlanes) + 2 * kTileN * 4 + 2 * kNodes * 8 + 2 * kProducers * 4 +
+           1024;
 }
 
 cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {

@@ -132,8 +132,12 @@ zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* c
  * rounding).  ZHA_KERNELS_AUTO picks the tensor cores (tcgen05) when a (sequence, KV
  * head) group has >= 64 lanes - for scoring only if every tree has R = 16 - and the CUDA
  * cores otherwise; SIMT and TENSOR force one kind.
- *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::tf32 with hi+lo passes
- *          (ZHA_ERR_ARG for TENSOR unless every tree has R = 16)
+ *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::f16 with Q in fp16 and
+ *          each summary split into fp16 hi + lo passes (ZHA_ERR_ARG for TENSOR unless
+ *          every tree has R = 16).  The tensor path needs every entry of Q and of the
+ *          cache's keys below 65504 in magnitude (the fp16 range); otherwise it sets
+ *          bit 8 of the device status word (see zha_decoder_stats) and its plane
+ *          estimates are not valid - select SIMT for such data.
  *   attn   exact attention: CUDA-core split-KV, or tcgen05 kind::f16 (S = Q K^T exact
  *          products, P split into bf16 hi + lo for P V) */
 typedef enum zha_kernels { ZHA_KERNELS_AUTO = 0, ZHA_KERNELS_SIMT = 1, ZHA_KERNELS_TENSOR = 2 } zha_kernels;
@@ -182,7 +186,10 @@ int64_t zha_decoder_words(const zha_decoder* dec, int32_t level);
 /* Work counters of the last zha_route / zha_sparse_attn (synchronises `stream`):
  * nodes scored per level as the union over each (sequence, KV head) group of lanes and
  * as the per-lane sum, attended tokens (union per group and per-lane sum), and the
- * device status word (0 = ok). */
+ * device status word (0 = ok; bit 1: the top-p select ran out of bisection steps,
+ * bit 4: a tensor-core wait gave up after 2 s, bit 8: an input outside the fp16 range
+ * reached the tensor-core scorer).
+ * Returns ZHA_ERR_DEVICE when the status word is not 0. */
 typedef struct zha_decode_stats {
     int64_t union_nodes[ZHA_MAX_LEVELS];      /* index l-1 */
     int64_t lane_nodes[ZHA_MAX_LEVELS];

@@ -235,7 +235,8 @@ def test_error_paths_on_device():
 @needs_cuda
 @pytest.mark.parametrize("n_q", [1, 8, 64])
 def test_tensor_core_and_cuda_core_scoring_agree(n_q):
-    """The tcgen05 scorer (tf32 hi + lo passes) and the fp32 CUDA-core scorer route the
+    """The tcgen05 scorer (fp16 Q, summaries split into fp16 hi + lo passes) and the fp32
+    CUDA-core scorer route the
     64K deep workload to the same kept sets (up to logged ties) and the same outputs; the
     tensor-core result is also checked against the oracle."""
     wl = inputs.deep_64k(n_q=n_q)
@@ -256,6 +257,29 @@ def test_tensor_core_and_cuda_core_scoring_agree(n_q):
     qs = list(range(min(n_q, 4)))
     rep, e1, e2, _ = TL.check_decode(seq, seq.n_tokens, Q[0], 0.95, b.out[0], b.kept[0], qs)
     _report("tensor n_q=%d" % n_q, rep, e1, e2)
+
+
+@needs_cuda
+def test_tensor_core_scoring_flags_inputs_outside_fp16_range():
+    """A query entry beyond the fp16 range makes the tensor-core scorer raise status bit 8
+    (its estimates are then not valid); the CUDA-core scorer takes the same input."""
+    import ctypes
+    wl = inputs.deep_64k(n_q=64)
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0].clone()
+    Q[0, 3, 5, 7] = 1.0e5                          # bf16 holds it, fp16 does not
+    Qd = Q.cuda()
+    for path, want in ((zha.ZHA_KERNELS_TENSOR, 8), (zha.ZHA_KERNELS_SIMT, 0)):
+        dec = zha.Decoder([tree], 64)
+        dec.set_kernels(score=path, attn=zha.ZHA_KERNELS_SIMT)
+        dec.route(Qd, 0.95)
+        torch.cuda.synchronize()
+        st = zha.DecodeStats()
+        rc = zha.lib().zha_decoder_stats(dec.handle, ctypes.byref(st), 0)
+        assert (st.status & 8) == want
+        assert rc == (zha.ZHA_ERR_DEVICE if want else zha.ZHA_OK)
+        dec.close()
 
 
 @needs_cuda
