@@ -337,6 +337,12 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         const int64_t segs = segs_per_split(1, t->g.C);
         s_cap = std::max<int64_t>(s_cap, (nseg_max + segs - 1) / segs);
     }
+    // union parents of a scored level sit at level >= 2
+    int64_t cap2 = 1;
+    for (auto* t : dec->trees)
+        if (t->g.L >= 2) cap2 = std::max<int64_t>(cap2, t->cap[2]);
+    w.ms = cap2;
+    w.mwords = (max_queries * dec->G + 31) / 32;
     w.lanes_cap = dec->lanes_cap;
     w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
     w.us = cap1;
@@ -361,6 +367,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     off += up256((size_t)dec->groups_cap * w.uw * 4);
     const size_t part_off = off;
     off += up256((size_t)dec->lanes_cap * w.s_cap * (dec->d + 4) * 4);
+    const size_t memb_off = off;
+    off += up256((size_t)dec->groups_cap * w.ms * w.mwords * 4);
     const size_t lmax_off = off;
     off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
     const size_t lcnt_off = off;
@@ -385,6 +393,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.ucount = reinterpret_cast<int32_t*>(base + ucount_off);
     w.uword = reinterpret_cast<uint32_t*>(base + uword_off);
     w.part = reinterpret_cast<float*>(base + part_off);
+    w.memb = reinterpret_cast<uint32_t*>(base + memb_off);
     w.lane_max = reinterpret_cast<uint32_t*>(base + lmax_off);
     w.lane_cnt = reinterpret_cast<int32_t*>(base + lcnt_off);
     w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);

@@ -52,6 +52,9 @@ struct Work {
     int64_t uw;
     float* part;                     // [lanes_cap][s_cap][d+2] attention partials
     int64_t s_cap;
+    uint32_t* memb;                  // [groups_cap][ms][mwords] union parents' lane masks (tensor scorer)
+    int64_t ms;
+    int32_t mwords;
     uint32_t* lane_max;              // [(kMaxL+1)][lanes_cap] frontier max score per lane (ordered bits)
     int32_t* lane_cnt;               // [(kMaxL+1)][lanes_cap] frontier size per lane
     unsigned long long* ctr;         // kCtrCount counters

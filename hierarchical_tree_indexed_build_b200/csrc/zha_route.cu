@@ -37,12 +37,6 @@ __device__ __forceinline__ T warp_sum(T v) {
     return v;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
-}
-
 // Block-wide reductions; `red` holds >= 32 elements; all threads get the result.
 template <typename T>
 __device__ T block_sum(T v, T* red) {
@@ -54,16 +48,6 @@ __device__ T block_sum(T v, T* red) {
     T t = (lane < nw) ? red[lane] : T(0);
     t = warp_sum(t);
     return t;
-}
-
-__device__ float block_max(float v, float* red) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-    v = warp_max(v);
-    __syncthreads();
-    if (lane == 0) red[wid] = v;
-    __syncthreads();
-    float t = (lane < nw) ? red[lane] : -INFINITY;
-    return warp_max(t);
 }
 
 template <typename T>

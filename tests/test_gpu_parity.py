@@ -233,7 +233,7 @@ def test_error_paths_on_device():
 
 
 @needs_cuda
-@pytest.mark.parametrize("n_q", [1, 8, 64])
+@pytest.mark.parametrize("n_q", [1, 8, 20, 48, 64])
 def test_tensor_core_and_cuda_core_scoring_agree(n_q):
     """The tcgen05 scorer (fp16 Q, summaries split into fp16 hi + lo passes) and the fp32
     CUDA-core scorer route the
