@@ -136,6 +136,21 @@ __device__ __forceinline__ void reset_smem(float* st, int stride) {
     for (int k = 0; k < D / 4; ++k) st[(2 + k) * stride] = 0.0f;
 }
 
+// Key rows of a worker's span are staged in shared memory by cp.async, kStages groups of
+// kTok tokens in flight, so the sequential per-token update reads K at shared-memory
+// latency instead of waiting on global loads.
+constexpr int kTok = 8;
+constexpr int kStages = 3;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Streams the C^k_emit tokens of one level-k_emit node per worker and emits the summaries of
 // every node of levels 1..k_emit beneath it.  Level-1 state lives in registers, levels
 // 2..k_emit in shared memory ([level][field][thread]).
@@ -145,9 +160,10 @@ __global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
     const int wt = 4 * a.R;
     const int wpb = blockDim.x / wt;
     const int tid = threadIdx.x;
-    const int r = (tid % wt) >> 2;
+    const int wk = tid / wt, wl = tid % wt;          // worker in block, thread in worker
+    const int r = wl >> 2;
     const int q = tid & 3;
-    int64_t widx = (int64_t)blockIdx.x * wpb + tid / wt;
+    int64_t widx = (int64_t)blockIdx.x * wpb + wk;
     const int64_t total = (int64_t)a.Hkv * a.nu;
     const bool active = widx < total;
     if (!active) widx = total - 1;
@@ -161,67 +177,105 @@ __global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
     const int nst = a.k_emit - 1;   // shared-memory levels (2..k_emit)
     const int stride = blockDim.x;
     for (int l = 0; l < nst; ++l) reset_smem<D>(smem_state + (int64_t)l * (D / 4 + 2) * stride + tid, stride);
+    // staged key rows: [worker][stage][token][D] bf16 after the level states
+    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem_state + (int64_t)nst * (D / 4 + 2) * stride) +
+                        (int64_t)wk * kStages * kTok * D;
 
     int64_t span_emit = 1;
     for (int l = 0; l < a.k_emit; ++l) span_emit *= C;
     const int64_t t0 = u * span_emit;
     const __nv_bfloat16* Kg = a.K + ((int64_t)g * a.ld + t0) * D;
+    const int ngrp = (int)((span_emit + kTok - 1) / kTok);
+    constexpr int kChunks = kTok * D * 2 / 16;       // 16-byte pieces of one token group
+    auto issue = [&](int grp) {
+        if (grp < ngrp) {
+            __nv_bfloat16* dst = sK + (grp % kStages) * kTok * D;
+            const __nv_bfloat16* src = Kg + (int64_t)grp * kTok * D;
+            const int64_t rest = span_emit - (int64_t)grp * kTok;
+            const int64_t ntk = rest < kTok ? rest : kTok;
+            for (int c = wl; c < kChunks; c += wt)
+                if (c / (D * 2 / 16) < ntk) cp_async16(dst + c * 8, src + c * 8);
+        }
+        cp_async_commit();   // one group per call on every thread keeps the counts aligned
+    };
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
 
     float mx = -INFINITY, z = 0.0f, acc[D / 4];
 #pragma unroll
     for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
 
-    float kv[D / 4], kn[D / 4];
-    load_row_bf16<D>(Kg, q, kn);
     int left = C;   // tokens left in the current level-1 chunk
-    for (int64_t tt = 0; tt < span_emit; ++tt) {
+    for (int grp = 0; grp < ngrp; ++grp) {
+        issue(grp + kStages - 1);
+        cp_async_wait<kStages - 1>();
+        __syncthreads();
+        const __nv_bfloat16* kb = sK + (grp % kStages) * kTok * D;
+        const int64_t rest = span_emit - (int64_t)grp * kTok;
+        const int ntk = (int)(rest < kTok ? rest : kTok);
+        for (int tk = 0; tk < ntk; ++tk) {
+            const int64_t tt = (int64_t)grp * kTok + tk;
+            float kv[D / 4];
+            {
+                const uint2* p = reinterpret_cast<const uint2*>(kb + tk * D);
 #pragma unroll
-        for (int k = 0; k < D / 4; ++k) kv[k] = kn[k];
-        if (tt + 1 < span_emit) load_row_bf16<D>(Kg + (tt + 1) * D, q, kn);
-        float dot = 0.0f;
+                for (int i = 0; i < D / 16; ++i) {
+                    const uint2 uu = p[4 * i + q];
+                    const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.x));
+                    const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.y));
+                    kv[4 * i + 0] = x0.x;
+                    kv[4 * i + 1] = x0.y;
+                    kv[4 * i + 2] = x1.x;
+                    kv[4 * i + 3] = x1.y;
+                }
+            }
+            float dot = 0.0f;
 #pragma unroll
-        for (int k = 0; k < D / 4; ++k) dot = fmaf(qv[k], kv[k], dot);
-        const float sc = a.scale * quad_sum(dot);
-        const float mn = fmaxf(mx, sc);
-        const float c = expf(mx - mn);
-        const float w = expf(sc - mn);
-        z = fmaf(z, c, w);
+            for (int k = 0; k < D / 4; ++k) dot = fmaf(qv[k], kv[k], dot);
+            const float sc = a.scale * quad_sum(dot);
+            const float mn = fmaxf(mx, sc);
+            const float c = expf(mx - mn);
+            const float wgt = expf(sc - mn);
+            z = fmaf(z, c, wgt);
 #pragma unroll
-        for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], c, w * kv[k]);
-        mx = mn;
-        if (--left == 0) {
-            left = C;
-            const int64_t t = t0 + tt;
-            const int64_t j1 = t / C;
-            float m1[D / 4];
-            const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
-                                               a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
-                                               a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
-                                               active, m1);
-            if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
-            mx = -INFINITY;
-            z = 0.0f;
+            for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], c, wgt * kv[k]);
+            mx = mn;
+            if (--left == 0) {
+                left = C;
+                const int64_t t = t0 + tt;
+                const int64_t j1 = t / C;
+                float m1[D / 4];
+                const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
+                                                   a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
+                                                   a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
+                                                   active, m1);
+                if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
+                mx = -INFINITY;
+                z = 0.0f;
 #pragma unroll
-            for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
-            // cascade completed ancestors (levels 2..k_emit)
-            int64_t span = C;
-            for (int l = 2; l <= a.k_emit; ++l) {
-                span *= C;
-                if ((tt + 1) % span != 0) break;
-                float* st = smem_state + (int64_t)(l - 2) * (D / 4 + 2) * stride + tid;
-                float smx, sz, sacc[D / 4], ml[D / 4];
-                load_state<D>(st, stride, smx, sz, sacc);
-                const int64_t jl = t / span;
-                const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
-                                                   a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
-                                                   a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
-                                                   active, ml);
-                if (l < a.k_emit)
-                    fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
-                reset_smem<D>(st, stride);
+                for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
+                // cascade completed ancestors (levels 2..k_emit)
+                int64_t span = C;
+                for (int l = 2; l <= a.k_emit; ++l) {
+                    span *= C;
+                    if ((tt + 1) % span != 0) break;
+                    float* st = smem_state + (int64_t)(l - 2) * (D / 4 + 2) * stride + tid;
+                    float smx, sz, sacc[D / 4], ml[D / 4];
+                    load_state<D>(st, stride, smx, sz, sacc);
+                    const int64_t jl = t / span;
+                    const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
+                                                       a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
+                                                       a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
+                                                       active, ml);
+                    if (l < a.k_emit)
+                        fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
+                    reset_smem<D>(st, stride);
+                }
             }
         }
+        __syncthreads();   // stage grp % kStages is refilled by the next iteration's issue
     }
+    cp_async_wait<0>();
 }
 
 // Merges the C children (level l-1) of each parent node P in [p0, p0+np) at level l:
@@ -269,7 +323,8 @@ cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st) {
     const int wpb = workers_per_block(a.R);
     const int threads = wpb * 4 * a.R;
     const int64_t blocks = ((int64_t)a.Hkv * a.nu + wpb - 1) / wpb;
-    const size_t smem = (size_t)(a.k_emit - 1) * (d / 4 + 2) * threads * sizeof(float);
+    const size_t smem = (size_t)(a.k_emit - 1) * (d / 4 + 2) * threads * sizeof(float) +
+                        (size_t)wpb * kStages * kTok * d * 2;
     ProfScope ps_("k_build_stream", st);
     if (d == 128) {
         cudaFuncSetAttribute(k_build_stream<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
