@@ -8,6 +8,8 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "zha_common.cuh"
 #include "zha_launch.h"
 
@@ -40,6 +42,27 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 float score_scale(int d) { return (float)(1.0 / sqrt((double)d)); }
 
+// TMA map over one level's fp16 planes: (dim, plane r, hi/lo, node over all KV heads),
+// boxes of 64 dims x R planes of one node, 128-byte swizzle (the MMA operand layout).
+bool encode_plane_map(CUtensorMap* map, const float* rec, int d, int R, int64_t nodes, int ns) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return false;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)R, 2, (cuuint64_t)nodes};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)R * d * 2, (cuuint64_t)ns * 4};
+    const cuuint32_t box[4] = {64, (cuuint32_t)R, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<float*>(rec), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 struct zha_tree {
@@ -51,6 +74,7 @@ struct zha_tree {
     float* rec[kMaxL + 1];
     float* lse[kMaxL + 1];
     __nv_bfloat16* qref;
+    int32_t* rflag;          // device word: a summary left the fp16 range
     void* block;
     size_t bytes;
     int device;
@@ -116,6 +140,8 @@ extern "C" zha_status zha_tree_create(const zha_geometry* g, zha_tree** out) {
     }
     const size_t qref_off = off;
     off += up256((size_t)g->n_kv_heads * g->R * g->d * 2);
+    const size_t rflag_off = off;
+    off += up256(4);
     cudaGetDevice(&t->device);
     cudaError_t e = cudaMalloc(&t->block, off);
     if (e != cudaSuccess) {
@@ -129,6 +155,8 @@ extern "C" zha_status zha_tree_create(const zha_geometry* g, zha_tree** out) {
         t->lse[l] = reinterpret_cast<float*>(base + lse_off[l]);
     }
     t->qref = reinterpret_cast<__nv_bfloat16*>(base + qref_off);
+    t->rflag = reinterpret_cast<int32_t*>(base + rflag_off);
+    cudaMemset(t->rflag, 0, 4);
     *out = t;
     return ZHA_OK;
 }
@@ -161,6 +189,7 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
     ba.K = static_cast<const __nv_bfloat16*>(K);
     ba.ld = g.capacity;
     ba.qref = t->qref;
+    ba.rflag = t->rflag;
     ba.Hkv = g.n_kv_heads;
     ba.R = g.R;
     ba.C = C;
@@ -176,6 +205,7 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
         MergeArgs ma;
         memset(&ma, 0, sizeof(ma));
         ma.qref = t->qref;
+        ma.rflag = t->rflag;
         ma.Hkv = g.n_kv_heads;
         ma.R = g.R;
         ma.C = C;
@@ -241,6 +271,7 @@ extern "C" zha_status zha_build_tree(zha_tree* t, const void* K, int64_t n_token
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     ZHA_CUDA(cudaMemcpyAsync(t->qref, q_ref, (size_t)t->g.n_kv_heads * t->g.R * t->g.d * 2,
                              cudaMemcpyDeviceToDevice, st));
+    ZHA_CUDA(cudaMemsetAsync(t->rflag, 0, 4, st));
     zha_status s = run_levels(t, K, 0, n_tokens, st);
     if (s != ZHA_OK) return s;
     t->n_tokens = n_tokens;
@@ -270,12 +301,9 @@ extern "C" zha_status zha_tree_export(const zha_tree* t, int32_t level, float* m
     const int64_t nl = t->n_tokens / ipow(g.C, level);
     if (nl == 0) return ZHA_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m) ZHA_CUDA(launch_export_m(t->rec[level], t->cap[level], t->ns, g.n_kv_heads, g.R, g.d, nl, m, st));
     for (int h = 0; h < g.n_kv_heads; ++h) {
         const float* src = t->rec[level] + (int64_t)h * t->cap[level] * t->ns;
-        if (m)
-            ZHA_CUDA(cudaMemcpy2DAsync(m + (int64_t)h * nl * g.R * g.d, (size_t)g.R * g.d * 4, src,
-                                       (size_t)t->ns * 4, (size_t)g.R * g.d * 4, (size_t)nl,
-                                       cudaMemcpyDeviceToDevice, st));
         if (b)
             ZHA_CUDA(cudaMemcpy2DAsync(b + (int64_t)h * nl * g.R, (size_t)g.R * 4, src + (int64_t)g.R * g.d,
                                        (size_t)t->ns * 4, (size_t)g.R * 4, (size_t)nl,
@@ -342,7 +370,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     for (auto* t : dec->trees)
         if (t->g.L >= 2) cap2 = std::max<int64_t>(cap2, t->cap[2]);
     w.ms = cap2;
-    w.mwords = (max_queries * dec->G + 31) / 32;
+    w.mwords = (max_queries * dec->G + 255) / 256 * 8;
     w.lanes_cap = dec->lanes_cap;
     w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
     w.us = cap1;
@@ -373,6 +401,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
     const size_t lcnt_off = off;
     off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
+    const size_t tmap_off = off;
+    off += up256((size_t)n_seq * (kMaxL + 1) * sizeof(CUtensorMap));
     const size_t ctr_off = off;
     off += up256((size_t)kCtrCount * 8);
     const size_t status_off = off;
@@ -400,6 +430,24 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.status = reinterpret_cast<int32_t*>(base + status_off);
     dec->seq_dev = reinterpret_cast<SeqDev*>(base + seq_off);
     dec->seq_host.resize(n_seq);
+    // TMA maps of the trees' fp16 planes, one per (sequence, level), for the tensor scorer
+    w.tmaps = nullptr;
+    if (dec->all_r16) {
+        std::vector<CUtensorMap> maps((size_t)n_seq * (kMaxL + 1));
+        memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+        bool ok = true;
+        for (int s = 0; s < n_seq && ok; ++s) {
+            const zha_tree* t = dec->trees[s];
+            for (int l = 1; l <= t->g.L && ok; ++l)
+                ok = encode_plane_map(&maps[(size_t)s * (kMaxL + 1) + l], t->rec[l], t->g.d, t->g.R,
+                                      (int64_t)t->g.n_kv_heads * t->cap[l], t->ns);
+        }
+        if (ok) {
+            CUtensorMap* dst = reinterpret_cast<CUtensorMap*>(base + tmap_off);
+            cudaMemcpy(dst, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
+            w.tmaps = dst;
+        }
+    }
     cudaMemset(w.ctr, 0, (size_t)kCtrCount * 8);
     cudaMemset(w.status, 0, 4);
     *out = dec;
@@ -434,6 +482,7 @@ static zha_status fill_seqs(zha_decoder* dec, const void* const* K, const void* 
             sd.cap[l] = t->cap[l];
             sd.rec[l] = t->rec[l];
         }
+        sd.rflag = t->rflag;
         if (K) sd.K = static_cast<const __nv_bfloat16*>(K[s]);
         if (V) sd.V = static_cast<const __nv_bfloat16*>(V[s]);
     }
@@ -531,6 +580,8 @@ extern "C" zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, i
     if (!ok(score) || !ok(attn)) return fail(ZHA_ERR_ARG, "unknown kernel choice");
     if (score == ZHA_KERNELS_TENSOR && !dec->all_r16)
         return fail(ZHA_ERR_ARG, "the tensor-core scorer needs R = 16 in every tree");
+    if (score == ZHA_KERNELS_TENSOR && !dec->w.tmaps)
+        return fail(ZHA_ERR_CUDA, "the tensor-core scorer's TMA maps could not be encoded");
     dec->score_path = score;
     dec->attn_path = attn;
     return ZHA_OK;

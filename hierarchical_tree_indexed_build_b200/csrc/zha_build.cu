@@ -14,6 +14,8 @@
 // unnormalised online softmax (mx, z, acc[]) with acc = sum_t exp(a_t - mx) k_t.
 #include <math.h>
 
+#include <algorithm>
+
 #include "zha_common.cuh"
 #include "zha_launch.h"
 #include "zha_profile.h"
@@ -39,19 +41,6 @@ __device__ __forceinline__ void load_row_bf16(const __nv_bfloat16* row, int q, f
     }
 }
 
-template <int D>
-__device__ __forceinline__ void load_row_f32(const float* row, int q, float (&v)[D / 4]) {
-    const float4* p = reinterpret_cast<const float4*>(row);
-#pragma unroll
-    for (int i = 0; i < D / 16; ++i) {
-        const float4 u = __ldg(p + 4 * i + q);
-        v[4 * i + 0] = u.x;
-        v[4 * i + 1] = u.y;
-        v[4 * i + 2] = u.z;
-        v[4 * i + 3] = u.w;
-    }
-}
-
 // Sum over the 4 quarter-threads of a row.
 __device__ __forceinline__ float quad_sum(float v) {
     v += __shfl_xor_sync(kFull, v, 1);
@@ -59,32 +48,61 @@ __device__ __forceinline__ float quad_sum(float v) {
     return v;
 }
 
+// m values of plane r held by thread quarter q (dims 16 i + 4 q + c) of a stored record.
+template <int D>
+__device__ __forceinline__ void load_row_m(const float* rec, int R, int r, int q, float (&v)[D / 4]) {
+    const __half* h = reinterpret_cast<const __half*>(rec);
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+        const uint2 hi = __ldg(reinterpret_cast<const uint2*>(h + (int64_t)r * D + 16 * i + 4 * q));
+        const uint2 lo = __ldg(reinterpret_cast<const uint2*>(h + (int64_t)R * D + (int64_t)r * D + 16 * i + 4 * q));
+        const float2 x = m_decode2(hi.x, lo.x), y = m_decode2(hi.y, lo.y);
+        v[4 * i + 0] = x.x;
+        v[4 * i + 1] = x.y;
+        v[4 * i + 2] = y.x;
+        v[4 * i + 3] = y.y;
+    }
+}
+
 // Turn a running state into the stored summary of one node and write it:
-// m_r = acc / z, lse_r = mx + log z, b_r = lse_r - s q_r.m_r.  Returns lse_r; m_r is left
-// in `m` so the parent can fold exactly the stored values.
+// m_r = acc / z (stored as fp16 hi + lo planes), lse_r = mx + log z, b_r = lse_r - s q_r.m_r
+// with the stored m.  Returns lse_r; the stored m (decoded) is left in `m` so the parent
+// folds exactly what a merge from the record would read.
 template <int D>
 __device__ __forceinline__ float finalize_store(float mx, float z, const float (&acc)[D / 4],
                                                 const float (&qv)[D / 4], float scale, float* rec,
-                                                float* lse, int r, int q, int R, bool store,
+                                                float* lse, int r, int q, int R, bool store, int32_t* rflag,
                                                 float (&m)[D / 4]) {
     const float inv = 1.0f / z;
     float qm = 0.0f;
+    bool bad = false;
+    __half* hp = reinterpret_cast<__half*>(rec);
 #pragma unroll
-    for (int k = 0; k < D / 4; ++k) {
-        m[k] = acc[k] * inv;
-        qm = fmaf(qv[k], m[k], qm);
+    for (int i = 0; i < D / 16; ++i) {
+        float a[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            a[c] = acc[4 * i + c] * inv;
+            bad |= !(fabsf(a[c]) < 65504.0f);
+        }
+        uint32_t h0, l0, h1, l1;
+        m_encode2(a[0], a[1], h0, l0, m[4 * i], m[4 * i + 1]);
+        m_encode2(a[2], a[3], h1, l1, m[4 * i + 2], m[4 * i + 3]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qm = fmaf(qv[4 * i + c], m[4 * i + c], qm);
+        if (store) {
+            *reinterpret_cast<uint2*>(hp + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(h0, h1);
+            *reinterpret_cast<uint2*>(hp + (int64_t)R * D + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(l0, l1);
+        }
     }
     qm = quad_sum(qm);
     const float l = mx + logf(z);
     if (store) {
-        float4* dst = reinterpret_cast<float4*>(rec + (int64_t)r * D);
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i)
-            dst[4 * i + q] = make_float4(m[4 * i], m[4 * i + 1], m[4 * i + 2], m[4 * i + 3]);
         if (q == 0) {
             rec[(int64_t)R * D + r] = fmaf(-scale, qm, l);
             lse[r] = l;
         }
+        if (bad) atomicOr(rflag, 1);
     }
     return l;
 }
@@ -248,7 +266,7 @@ __global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
                 const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
                                                    a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
                                                    a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
-                                                   active, m1);
+                                                   active, a.rflag, m1);
                 if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
                 mx = -INFINITY;
                 z = 0.0f;
@@ -266,7 +284,7 @@ __global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
                     const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
                                                        a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
                                                        a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
-                                                       active, ml);
+                                                       active, a.rflag, ml);
                     if (l < a.k_emit)
                         fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
                     reset_smem<D>(st, stride);
@@ -303,12 +321,26 @@ __global__ void __launch_bounds__(128) k_merge(MergeArgs a) {
 #pragma unroll
     for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
     for (int c = 0; c < a.C; ++c) {
-        load_row_f32<D>(crec + (int64_t)c * a.ns + (int64_t)r * D, q, mc);
+        load_row_m<D>(crec + (int64_t)c * a.ns, a.R, r, q, mc);
         const float lc = __ldg(clse + (int64_t)c * a.R + r);
         fold_child<D>(mx, z, acc, lc, mc);
     }
     finalize_store<D>(mx, z, acc, qv, a.scale, a.rec + ((int64_t)g * a.cap + P) * a.ns,
-                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, mo);
+                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, a.rflag, mo);
+}
+
+// Decodes the m planes of nodes [0, n) of every KV head into f32 [Hkv][n][R][d].
+__global__ void k_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
+                           float* m) {
+    const int64_t per = (int64_t)R * d / 4;   // float4 per node
+    const int64_t total = (int64_t)Hkv * n * per;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t node = t / per, e4 = t % per;
+        const int64_t h = node / n, j = node % n;
+        const int r = (int)(e4 * 4 / d), k = (int)(e4 * 4 % d);
+        const float4 v = m_load4(rec + (h * cap + j) * ns, R, d, r, k);
+        reinterpret_cast<float4*>(m)[t] = v;
+    }
 }
 
 int workers_per_block(int R) {
@@ -317,6 +349,15 @@ int workers_per_block(int R) {
 }
 
 }  // namespace
+
+cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
+                            float* m, cudaStream_t st) {
+    const int64_t total = (int64_t)Hkv * n * R * d / 4;
+    if (total <= 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148 * 16);
+    k_export_m<<<(unsigned)blocks, 256, 0, st>>>(rec, cap, ns, Hkv, R, d, n, m);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st) {
     if (a.nu <= 0) return cudaSuccess;

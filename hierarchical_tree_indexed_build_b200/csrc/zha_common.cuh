@@ -1,7 +1,9 @@
 // zha_common.cuh - device-side tables and helpers shared by the libzha kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,7 +27,8 @@ struct SeqDev {
     int64_t ld;                      // K/V rows per KV head (capacity)
     int64_t n[kMaxL + 1];            // complete nodes per level (index = level)
     int64_t cap[kMaxL + 1];          // node capacity per level
-    const float* rec[kMaxL + 1];     // [Hkv][cap_l][ns]
+    const float* rec[kMaxL + 1];     // [Hkv][cap_l][ns] node records (layout below)
+    const int32_t* rflag;            // tree's range flag: a summary left the fp16 range
     const __nv_bfloat16* K;          // [Hkv][ld][d]
     const __nv_bfloat16* V;
 };
@@ -54,7 +57,8 @@ struct Work {
     int64_t s_cap;
     uint32_t* memb;                  // [groups_cap][ms][mwords] union parents' lane masks (tensor scorer)
     int64_t ms;
-    int32_t mwords;
+    int32_t mwords;                  // a multiple of 8 covering every 256-lane pair of a group
+    const CUtensorMap* tmaps;        // [n_seq][kMaxL + 1] fp16 plane maps of the trees' levels (or null)
     uint32_t* lane_max;              // [(kMaxL+1)][lanes_cap] frontier max score per lane (ordered bits)
     int32_t* lane_cnt;               // [(kMaxL+1)][lanes_cap] frontier size per lane
     unsigned long long* ctr;         // kCtrCount counters
@@ -78,6 +82,34 @@ struct Batch {
 __host__ __device__ inline int64_t lane_of(const Batch& b, int s, int g, int y) {
     const int i = y / b.G, hh = y % b.G;
     return ((int64_t)s * b.n_q + i) * b.Hq + (int64_t)g * b.G + hh;
+}
+
+// Node record (ns floats): the R reference-query means m_r are stored as two fp16 planes,
+// hi [R][d] = fp16(m) then lo [R][d] = fp16(m - hi), followed by b [R] (f32).  hi + lo
+// recovers m within 2^-22 |m| + 2^-25 (exactly representable in f32), and the planes are
+// the tensor cores' operand format.  |m| must stay below 65504.
+__device__ __forceinline__ void m_encode2(float a, float b, uint32_t& hi, uint32_t& lo, float& da, float& db) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+    const float2 lf = __half22float2(l);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+    da = hf.x + lf.x;
+    db = hf.y + lf.y;
+}
+__device__ __forceinline__ float2 m_decode2(uint32_t hi, uint32_t lo) {
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+    const float2 lf = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+    return make_float2(hf.x + lf.x, hf.y + lf.y);
+}
+// Four consecutive m values (dims k..k+3 of plane r) of a record from its two planes.
+__device__ __forceinline__ float4 m_load4(const float* rec, int R, int D, int r, int k) {
+    const __half* h = reinterpret_cast<const __half*>(rec);
+    const uint2 a = *reinterpret_cast<const uint2*>(h + (int64_t)r * D + k);
+    const uint2 c = *reinterpret_cast<const uint2*>(h + (int64_t)R * D + (int64_t)r * D + k);
+    const float2 x = m_decode2(a.x, c.x), y = m_decode2(a.y, c.y);
+    return make_float4(x.x, x.y, y.x, y.y);
 }
 
 // Order-preserving map of a float to uint32 (atomicMax on the result is a float max).

@@ -15,6 +15,7 @@ struct BuildArgs {
     const __nv_bfloat16* K;      // [Hkv][ld][d]
     int64_t ld;
     const __nv_bfloat16* qref;   // [Hkv][R][d]
+    int32_t* rflag;              // set when a summary leaves the fp16 range
     int32_t Hkv, R, C, ns, k_emit;
     int64_t u0, nu;
     float scale;
@@ -26,6 +27,7 @@ struct BuildArgs {
 // Merge: parents [p0, p0+np) of one level from their C children.
 struct MergeArgs {
     const __nv_bfloat16* qref;
+    int32_t* rflag;
     int32_t Hkv, R, C, ns;
     int64_t p0, np;
     float scale;
@@ -39,6 +41,9 @@ struct MergeArgs {
 
 cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st);
 cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st);
+// m of nodes [0, n) of every KV head of one level, decoded to f32 [Hkv][n][R][d].
+cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
+                            float* m, cudaStream_t st);
 
 // Decode (routing + attention).  `it` is the level iteration: sequence s works on level
 // L_s - it.  mode 0 of the union kernel prepares routing iteration it (union of the kept

@@ -210,8 +210,10 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
     const bool top = (lev == sq.L);
     const int C = sq.C;
     const int64_t nc = top ? sq.T : (int64_t)w.ucount[grp] * C;
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
+        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+    }
     if (nc == 0) return;
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int NPC = 8 / WB;
@@ -246,13 +248,17 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
     for (int64_t k = (int64_t)blockIdx.x * NPC + slot; k < nc; k += (int64_t)gridDim.x * NPC) {
         const int64_t j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
         const float* rec = base + j * ns;
+        const __half* rh = reinterpret_cast<const __half*>(rec);
         float best = -INFINITY;
         for (int r = 0; r < R; ++r) {
-            const float4* row = reinterpret_cast<const float4*>(rec + (int64_t)r * D);
+            const uint2* hrow = reinterpret_cast<const uint2*>(rh + (int64_t)r * D);
+            const uint2* lrow = reinterpret_cast<const uint2*>(rh + (int64_t)R * D + (int64_t)r * D);
             float dot = 0.0f;
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) {
-                const float4 m = __ldg(row + 4 * i + q);
+                const uint2 hv = __ldg(hrow + 4 * i + q), lv = __ldg(lrow + 4 * i + q);
+                const float2 m01 = m_decode2(hv.x, lv.x), m23 = m_decode2(hv.y, lv.y);
+                const float4 m = make_float4(m01.x, m01.y, m23.x, m23.y);
                 dot = fmaf(qv[4 * i], m.x, dot);
                 dot = fmaf(qv[4 * i + 1], m.y, dot);
                 dot = fmaf(qv[4 * i + 2], m.z, dot);
@@ -288,8 +294,7 @@ constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
 constexpr int kUn = 4;               // 128-candidate blocks per warp in flight
-// 2^39: fixed-point masses; sums of <= 2^24 candidates stay below 2^63 and are exact
-constexpr float kMassScale = 549755813888.0f;
+// masses are fixed point with 2^39 for exp(0); sums of <= 2^24 candidates stay below 2^63
 
 // Ascending key order == (e descending, node index ascending).
 __device__ __forceinline__ unsigned long long sel_key(float e, int j) {
@@ -298,13 +303,32 @@ __device__ __forceinline__ unsigned long long sel_key(float e, int j) {
 __device__ __forceinline__ float key_score(unsigned long long k) {
     return unord_bits(~(uint32_t)(k >> 32));
 }
-__device__ __forceinline__ unsigned long long mass_of(float e, float M) {
-    return (unsigned long long)(expf(e - M) * kMassScale);
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
-__device__ __forceinline__ int bin_of(float e, float M) {
-    const float t = (M - e) * kBinScale;
-    return t >= (float)(kNB - 1) ? kNB - 1 : (int)t;
-}
+// The cut's arithmetic is shared by every pass and kept off the quarter-rate conversion
+// unit: one ex2 per candidate, the rest on the FMA and integer pipes.
+struct SelMath {
+    float nl2M;     // -M log2(e)
+    float m64;      // M kBinScale
+    // fixed-point mass floor(exp(e - M) 2^39), read from the bits of the float exp(e - M)
+    __device__ __forceinline__ unsigned long long mass(float e) const {
+        const float f = ex2_approx(fmaf(e, 1.4426950408889634f, nl2M));   // in [0, 1]
+        const uint32_t u = __float_as_uint(f);
+        const int ex = (int)(u >> 23);                                        // f >= 0
+        const uint32_t mant = (u & 0x7fffffu) | 0x800000u;
+        const int sh = ex - 111;                                              // 2^39 / 2^23 = 2^16 at ex = 127
+        if (ex == 0) return 0ull;
+        return sh >= 0 ? ((unsigned long long)mant << sh) : (unsigned long long)(mant >> min(-sh, 31));
+    }
+    // bin = round((M - e) kBinScale), clamped to kNB - 1 (magic-number rounding, no conversion)
+    __device__ __forceinline__ int bin(float e) const {
+        const float t = fminf(fmaf(e, -kBinScale, m64), (float)(kNB - 1));
+        return __float_as_int(t + 8388608.0f) - 0x4B000000;
+    }
+};
 
 // One block per lane.  The scorer left, for every candidate of the lane's group (the
 // children of the group's union of kept nodes, or all top nodes), the plane estimate if
@@ -338,6 +362,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         return;
     }
     const float M = unord_bits(w.lane_max[(int64_t)lev * w.lanes_cap + x]);
+    SelMath sm;
+    sm.nl2M = -M * 1.4426950408889634f;
+    sm.m64 = M * kBinScale;
     const bool top = (lev == sq.L);
     const int C = sq.C;
     // candidate and node indices are < 2^24 (level-1 nodes are capped there): 32-bit math
@@ -350,9 +377,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int nblk = (nc + 127) / 128;
 
-    // candidate k -> node index
+    // candidate k -> node index (shifts when C is a power of two)
+    const int cs = (C & (C - 1)) == 0 ? __ffs(C) - 1 : -1;
     auto cand_j = [&](int k) -> int {
         if (top) return k;
+        if (cs >= 0) return (__ldg(ul + (k >> cs)) << cs) + (k & (C - 1));
         const uint32_t pk = (uint32_t)k / (uint32_t)C;
         return __ldg(ul + pk) * C + (k - (int)pk * C);
     };
@@ -430,7 +459,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                if (v[c] > -INFINITY) atomicAdd(&hist[bin_of(v[c], M)], mass_of(v[c], M));
+                if (v[c] > -INFINITY) atomicAdd(&hist[sm.bin(v[c])], sm.mass(v[c]));
         });
         __syncthreads();
         unsigned long long zloc = 0;
@@ -483,7 +512,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             if (!(v[c] > -INFINITY)) continue;
-            const int bn = bin_of(v[c], M);
+            const int bn = sm.bin(v[c]);
             if (bn < bstar) {
                 nib |= 1u << c;
             } else if (bn == bstar) {
@@ -529,12 +558,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const int per = (n + blockDim.x - 1) / blockDim.x;
         const int i0 = threadIdx.x * per;
         unsigned long long run = 0;
-        for (int i = i0; i < min(n, i0 + per); ++i) run += mass_of(key_score(keys[i]), M);
+        for (int i = i0; i < min(n, i0 + per); ++i) run += sm.mass(key_score(keys[i]));
         unsigned long long tot;
         unsigned long long cum = block_excl_scan<unsigned long long>(run, red_u, tot);
         int found = n;
         for (int i = i0; i < min(n, i0 + per); ++i) {
-            cum += mass_of(key_score(keys[i]), M);
+            cum += sm.mass(key_score(keys[i]));
             if (cum >= need) {
                 found = i;
                 break;
@@ -554,7 +583,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                if (v[c] > -INFINITY && bin_of(v[c], M) == bstar) {
+                if (v[c] > -INFINITY && sm.bin(v[c]) == bstar) {
                     const unsigned long long kk = sel_key(v[c], jof(bk, j0, c));
                     klo = kk < klo ? kk : klo;
                     khi = kk > khi ? kk : khi;
@@ -570,8 +599,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    if (v[c] > -INFINITY && bin_of(v[c], M) == bstar && sel_key(v[c], jof(bk, j0, c)) <= mid)
-                        acc += mass_of(v[c], M);
+                    if (v[c] > -INFINITY && sm.bin(v[c]) == bstar && sel_key(v[c], jof(bk, j0, c)) <= mid)
+                        acc += sm.mass(v[c]);
             });
             acc = block_sum<unsigned long long>(acc, red_u);
             if (acc >= need) hi = mid;
@@ -584,7 +613,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                if (v[c] > -INFINITY && bin_of(v[c], M) == bstar) {
+                if (v[c] > -INFINITY && sm.bin(v[c]) == bstar) {
                     const int j = jof(bk, j0, c);
                     if (sel_key(v[c], j) <= lo) {
                         atomicOr(outw + (j >> 5), 1u << (j & 31));
@@ -619,7 +648,8 @@ cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaSt
 }
 
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
-    const bool tc = b.all_r16 && (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
+    const bool tc = b.all_r16 && w.tmaps &&
+                    (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
     if (tc) return launch_score_tc(b, w, it, scale, st);
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);

@@ -10,22 +10,25 @@
 // M = 128 lanes, N = 8 nodes x 16 planes, K = d, f32 accumulators in tensor memory.
 //
 // Precision: Q is bf16, which fp16 holds exactly for magnitudes in [2^-17, 65504).  The
-// f32 summary m is split into two fp16 terms m = hi + lo (lo the fp16 rounding of m - hi),
-// so two MMA passes accumulate Q.m with an error of at most 2^-22 |m| + 2^-25 per
-// element: float32-grade scores.  An entry of Q or m of magnitude >= 65504 does not fit;
-// the kernel then sets kStatusRange (the CUDA-core scorer has no such limit).
+// tree stores each summary m as two fp16 planes m = hi + lo (lo the fp16 rounding of
+// m - hi), so two MMA passes accumulate Q.m exactly as the f32 scorer would see the stored
+// m: float32-grade scores.  A query entry of magnitude >= 65504 does not fit; the kernel
+// then sets kStatusRange (as does a tree whose summaries left the fp16 range).
 //
-// Pipeline (one CTA per SM, persistent over its node tiles; LT = 1 or 2 lane tiles of 128
-// lanes per CTA share every node tile, so one read of a node serves 128 LT lanes):
-//   warps 0-7   producers: load a node tile (f32, one tile in flight in registers), split it
-//               into the two fp16 planes and store them in a 128-byte-swizzled K-major
-//               shared-memory stage (2 stages), with the tile's b values, node ids and the
-//               frontier-membership words of the CTA's lanes;
-//   warps 8..   epilogue, 4 per lane tile: tensor memory -> max over planes + b -> scores;
-//               lane 0 of warp 8 also issues the MMAs into one of two TMEM accumulators per
-//               lane tile (the next tile's as soon as its operands are staged).
-// Shared-memory operand layout: per K block of 64 fp16, rows are 128 bytes apart, the
-// 16-byte chunk c of row r sits at chunk c ^ (r % 8), 8-row groups 1024 bytes apart.
+// Pipeline (one CTA per SM, persistent over its node tiles of 8 nodes; LT = 1 or 2 lane
+// tiles of 128 lanes per CTA share every node tile):
+//   warp 0      loader: TMA copies of each node's two fp16 planes (boxes of 64 dims x 16
+//               planes, 128-byte swizzled by the copy engine into the MMA operand layout),
+//               plus bulk copies of the node's b values and of the CTA lanes' membership
+//               words, into one of 3 shared-memory stages;
+//   warp 1      MMA issuer: per lane tile, 2 planes x d/16 tcgen05.mma kind::f16 with the
+//               query tile (A) in tensor memory and the node tile (B) in shared memory;
+//   warps 2..   epilogue, 4 per lane tile: tensor memory -> max over planes + b -> scores.
+// With A in tensor memory an MMA reads only its B rows from shared memory.  Each lane tile
+// has one accumulator; while one lane tile's epilogue drains, the other's MMAs run (with
+// LT = 1 the accumulator is double-buffered instead).
+// Tensor memory: accumulators at columns 0 and 128, the queries of lane tile t at columns
+// 256 + t d/2 (two fp16 of a row per 32-bit column).
 //
 // Frontier membership comes from k_member: for every union parent u of the level above
 // and every 32 lanes of the group, one word whose bit t says whether lane 32 w + t kept u
@@ -47,9 +50,6 @@ constexpr int kTileM = 128;          // lanes per tile (MMA M)
 constexpr int kTileN = 128;          // rows (node, plane) per tile (MMA N)
 constexpr int kR = 16;               // planes per node on this path
 constexpr int kNodes = kTileN / kR;  // nodes per tile
-constexpr int kProducers = 256;      // warps 0-7
-constexpr int kMmaWarp = kProducers / 32;   // first epilogue warp: issues MMAs, owns TMEM
-constexpr int kChunk = kProducers / kNodes;   // tiles whose node ids are staged at once
 constexpr int kPlanes = 2;           // fp16 terms of m
 constexpr float kHalfMax = 65504.0f; // largest finite fp16
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
@@ -72,13 +72,27 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
 // Instruction descriptor: kind::f16 with fp16 A/B, f32 accumulate, both K-major, M x N.
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
 
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t acc) {
+// D (tensor memory) = or += A (tensor memory) x B (shared memory descriptor)
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
         :
-        : "r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(acc));
+        : "r"(tmem_d), "r"(tmem_a), "l"(b), "r"(kIdesc), "r"(acc));
+}
+
+// Writes 32 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :
+        : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
@@ -114,19 +128,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     }
 }
 
-// Non-blocking probe: has the phase with the given parity completed?
-__device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
     asm volatile(
@@ -140,21 +141,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Byte offset of element d (16-bit) of row `row` in a K-major tile of 128-row, 128-byte blocks.
-__device__ __forceinline__ uint32_t swz16(int row, int d) {
-    const int kb = d >> 6, c = (d & 63) >> 3;
-    return (uint32_t)(kb * (128 * 128) + row * 128 + ((c ^ (row & 7)) << 4) + (d & 7) * 2);
-}
-
-// m = hi + lo, hi the fp16 rounding of m and lo that of m - hi; two elements per word.
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const __half2 h = __floats2half2_rn(a, b);
-    const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
-    hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // Lanes' kept bits of the level above, transposed: memb[grp][u][w] bit t = lane 32 w + t
@@ -199,24 +185,44 @@ __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it) {
     }
 }
 
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        :
+        : "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :
+                 : "r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
+constexpr int kStages = 3;           // shared-memory stages of node tiles
+
 template <int D, int LT>
-__global__ void __launch_bounds__(kProducers + 128 * LT, 1) k_score_tc(Batch b, Work w, int it, float scale) {
-    constexpr int kThreads = kProducers + 128 * LT;
+__global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, int it, float scale) {
     constexpr int kEpilogue = 128 * LT;
     constexpr int kLW = 4 * LT;                       // 32-lane membership words per CTA
-    constexpr int KB = D / 64;                        // 128-byte K blocks of 16-bit elements
-    constexpr int A_BYTES = KB * kTileM * 128;        // one lane tile
+    constexpr int KB = D / 64;                        // 128-byte K blocks of fp16
     constexpr int P_BYTES = KB * kTileN * 128;        // one fp16 plane of one stage
+    constexpr int STAGE = kPlanes * P_BYTES;
+    constexpr uint32_t kColA = 256;                   // queries; accumulators at 0 and 128
+    constexpr uint32_t kCols = 512;
+    constexpr uint32_t kNodeBytes = kPlanes * KB * 16 * 128;   // both planes of one node
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* sA = base;                                             // [LT][A_BYTES]
-    unsigned char* sB0 = base + LT * A_BYTES;                             // [2 stages][2 planes][P_BYTES]
-    float* sBv = reinterpret_cast<float*>(sB0 + 2 * kPlanes * P_BYTES);   // [2][kTileN] b values
-    uint32_t* sMask = reinterpret_cast<uint32_t*>(sBv + 2 * kTileN);     // [2][kLW][kNodes] membership
-    int32_t* sJ = reinterpret_cast<int32_t*>(sMask + 2 * kLW * kNodes);  // [2][kNodes] node ids (-1: none)
-    int32_t* sNode = sJ + 2 * kNodes;                                     // [2][kChunk * kNodes] staged ids
-    __shared__ __align__(8) uint64_t bar_full[2], bar_acc_full[2], bar_acc_empty[2];
+    unsigned char* sB0 = base;                                             // [kStages][2 planes][P_BYTES]
+    float* sBv = reinterpret_cast<float*>(sB0 + kStages * STAGE);          // [kStages][kNodes][16] b values
+    uint32_t* sMask = reinterpret_cast<uint32_t*>(sBv + kStages * kTileN); // [kStages][kNodes][kLW] membership
+    int32_t* sJ = reinterpret_cast<int32_t*>(sMask + kStages * kNodes * kLW);   // [kStages][kNodes] node ids
+    __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages], bar_acc_full[2], bar_acc_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     volatile int& abort_sh = abort_flag;              // set by any role whose wait gave up
@@ -229,239 +235,217 @@ __global__ void __launch_bounds__(kProducers + 128 * LT, 1) k_score_tc(Batch b, 
     const bool top = (lev == sq.L);
     const int C = sq.C;
     const int nc = (int)(top ? sq.T : (int64_t)w.ucount[grp] * C);   // < 2^31: level-1 nodes <= 2^24
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
+        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+    }
     const int ntiles = (nc + kNodes - 1) / kNodes;
     if ((int)blockIdx.x >= ntiles) return;          // whole block leaves before any barrier
     const int nt = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;   // tiles of this block
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int y0 = blockIdx.y * (kTileM * LT);
-    const uint32_t ncols = 2 * kTileN * LT;           // two accumulators per lane tile
 
-    if (warp == kMmaWarp) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
-                     "r"(ncols));
+                     "r"(kCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(&bar_full[i]), 1);
+            mbar_init(smem_u32(&bar_empty[i]), kEpilogue);
+        }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bar_full[i]), kProducers);
             mbar_init(smem_u32(&bar_acc_full[i]), 1);
-            mbar_init(smem_u32(&bar_acc_empty[i]), kEpilogue);
+            mbar_init(smem_u32(&bar_acc_empty[i]), kTileM);   // one lane tile drains a slot
         }
         asm volatile("fence.mbarrier_init.release.cluster;");
         abort_sh = 0;
     }
-    // A: the CTA's query rows (bf16 -> fp16, exact in range), zero rows past the group's lanes.
-    float amax = 0.0f;
-    for (int i = tid; i < LT * kTileM * (D / 8); i += kThreads) {
-        const int row = i / (D / 8), c16 = i % (D / 8);
-        const int y = y0 + row;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (y < b.n_gl) v = __ldg(reinterpret_cast<const uint4*>(b.Q + lane_of(b, s, g, y) * D) + c16);
-        uint32_t hv[4];
-        const uint32_t* bv = &v.x;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(bv + t));
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            const __half2 h = __floats2half2_rn(f.x, f.y);
-            hv[t] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        *reinterpret_cast<uint4*>(sA + (row / kTileM) * A_BYTES + swz16(row % kTileM, c16 * 8)) =
-            make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    if (!(amax < kHalfMax)) atomicOr(w.status, kStatusRange);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_base_sh;
 
-    const int64_t ns = sq.ns;
-    const float* recb = sq.rec[lev] + (int64_t)g * sq.cap[lev] * ns;
-    const int32_t* ul = w.ulist + (int64_t)grp * w.us;
-    const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.y * kLW;
-
-    if (warp < kProducers / 32) {
-        // ---------------- producers
-        constexpr int kRowStep = kProducers / (D / 4);
-        constexpr int kU = kTileN / kRowStep;         // float4 per thread per tile
-        const int c4 = tid % (D / 4);
-        const int row0 = tid / (D / 4);
-        float mmax = 0.0f;                            // largest |m| this thread split
-        const int lane_words = (b.n_gl + 31) / 32;
-        // candidate k of the group -> node index (or -1 past the end)
-        auto node_of = [&](int k) -> int {
-            if (k >= nc) return -1;
-            if (top) return k;
-            const uint32_t pk = (uint32_t)k / (uint32_t)C;
-            return __ldg(ul + pk) * C + (k - (int)pk * C);
-        };
-        // Node ids of chunk c (tiles [c kChunk, (c+1) kChunk) of this block) into sNode[c & 1]:
-        // one independent load per producer thread, so no tile waits on a dependent load.
-        auto fill_chunk = [&](int c) {
-            const int i = c * kChunk + tid / kNodes;
-            int j = -1;
-            if (i < nt) j = node_of((blockIdx.x + i * gridDim.x) * kNodes + tid % kNodes);
-            sNode[(c & 1) * kProducers + tid] = j;
-        };
-        auto node_at = [&](int i, int nl) -> int {
-            return sNode[((i / kChunk) & 1) * kProducers + (i % kChunk) * kNodes + nl];
-        };
-        float4 pre[kU];
-        float preb = 0.f;
-        int prej = -1;
-        uint32_t prem = 0;
-        auto prefetch = [&](int i) {
+    // epilogue thread <-> one lane row of the CTA (TMEM lane quarter = warp % 4)
+    const int ew = warp - 2;
+    const int lt = ew >> 2, quad = warp & 3;
+    const int row = lt * kTileM + quad * 32 + lane;
+    const uint32_t tlane = (uint32_t)(quad * 32) << 16;
+    if (warp >= 2) {
+        // A: this lane's query row (bf16 -> fp16, exact in range) into tensor memory; zero
+        // rows past the group's lanes
+        const int y = y0 + row;
+        const uint4* qp = reinterpret_cast<const uint4*>(b.Q + lane_of(b, s, g, y < b.n_gl ? y : 0) * D);
+        float amax = 0.0f;
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int row = row0 + u * kRowStep;
-                const int j = node_at(i, row / kR);
-                pre[u] = j >= 0 ? __ldg(reinterpret_cast<const float4*>(recb + (int64_t)j * ns + (row % kR) * D) + c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            if (tid < kTileN) {
-                prej = node_at(i, tid / kR);
-                preb = prej >= 0 ? __ldg(recb + (int64_t)prej * ns + kR * D + tid % kR) : 0.0f;
-            }
-            if (tid < kLW * kNodes) {
-                // membership word (node tid / kLW, lane word tid % kLW) of tile i
-                const int k = (blockIdx.x + i * gridDim.x) * kNodes + tid / kLW;
-                const bool wok = (int)blockIdx.y * kLW + tid % kLW < lane_words;   // words past the group's lanes: 0
-                prem = (k >= nc || !wok) ? 0u : top ? 0xffffffffu : __ldg(memb + (int64_t)(k / C) * w.mwords + tid % kLW);
-            }
-        };
-        fill_chunk(0);
-        fill_chunk(1);
-        asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");
-        prefetch(0);
-        for (int i = 0; i < nt; ++i) {
-            const int st = i & 1;
-            // stage st (and its metadata) is free once the epilogue of tile i-2 is done.
-            // After an abort the producers keep stepping without waiting, so that all of them
-            // reach the same named barriers.
-            if (i >= 2 && !abort_sh && !mbar_wait(smem_u32(&bar_acc_empty[st]), (uint32_t)(((i >> 1) - 1) & 1))) {
-                atomicOr(w.status, kStatusTimeout);
-                abort_sh = 1;
-            }
-            unsigned char* pl = sB0 + (size_t)(kPlanes * st) * P_BYTES;
+        for (int h = 0; h < D / 64; ++h) {
+            uint32_t hv[32];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int row = row0 + u * kRowStep;
-                const float4 m = pre[u];
-                mmax = fmaxf(mmax, fmaxf(fmaxf(fabsf(m.x), fabsf(m.y)), fmaxf(fabsf(m.z), fabsf(m.w))));
-                uint32_t h0, l0, h1, l1;
-                split2(m.x, m.y, h0, l0);
-                split2(m.z, m.w, h1, l1);
-                const uint32_t off = swz16(row, c4 * 4);
-                *reinterpret_cast<uint2*>(pl + off) = make_uint2(h0, h1);
-                *reinterpret_cast<uint2*>(pl + P_BYTES + off) = make_uint2(l0, l1);
+            for (int c = 0; c < 8; ++c) {
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (y < b.n_gl) v = __ldg(qp + h * 8 + c);
+                const uint32_t* bv = &v.x;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(bv + t));
+                    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                    const __half2 hh = __floats2half2_rn(f.x, f.y);
+                    hv[c * 4 + t] = *reinterpret_cast<const uint32_t*>(&hh);
+                }
             }
-            if (tid < kTileN) {
-                sBv[st * kTileN + tid] = preb;
-                if (tid % kR == 0) sJ[st * kNodes + tid / kR] = prej;
-            }
-            if (tid < kLW * kNodes) sMask[st * kLW * kNodes + (tid % kLW) * kNodes + tid / kLW] = prem;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(smem_u32(&bar_full[st]));
-            // tile i + 1 may open the next chunk: stage its node ids one chunk ahead
-            if ((i + 1) % kChunk == 0 && i + 1 < nt) {
-                asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");   // old ids of that buffer consumed
-                fill_chunk((i + 1) / kChunk + 1);
-            }
-            if ((i + 1) % kChunk == 0)
-                asm volatile("bar.sync 1, %0;" ::"n"(kProducers) : "memory");   // new ids visible
-            if (i + 1 < nt) prefetch(i + 1);
+            tmem_st32(tmem + tlane + kColA + (uint32_t)(lt * (D / 2) + h * 32), hv);
         }
-        if (!(mmax < kHalfMax)) atomicOr(w.status, kStatusRange);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        if (!(amax < kHalfMax)) atomicOr(w.status, kStatusRange);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+    if (warp == 0) {
+        // ---------------- loader.  Lanes compute the node ids of 4 tiles at a time (one
+        // candidate each), a batch ahead of use; lane 0 issues the copies.
+        const CUtensorMap* map = w.tmaps + (int64_t)s * (kMaxL + 1) + lev;
+        asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+        const float* recb = sq.rec[lev];
+        const int64_t node0 = (int64_t)g * sq.cap[lev];               // first node of this KV head
+        const int32_t* ul = w.ulist + (int64_t)grp * w.us;
+        const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.y * kLW;
+        auto ids = [&](int i0, int& j, int& u) {
+            const int t = i0 + lane / kNodes;
+            j = -1;
+            u = 0;
+            if (t < nt) {
+                const int k = (blockIdx.x + t * gridDim.x) * kNodes + lane % kNodes;
+                if (k < nc) {
+                    if (top) {
+                        j = k;
+                    } else {
+                        u = (int)((uint32_t)k / (uint32_t)C);
+                        j = __ldg(ul + u) * C + (k - u * C);
+                    }
+                }
+            }
+        };
+        int jc, uc, jn, un;
+        ids(0, jc, uc);
+        int issued = 0;
+        bool stop = false;
+        for (int i0 = 0; i0 < nt && !stop; i0 += 4) {
+            ids(i0 + 4, jn, un);                      // next batch, in flight while this one issues
+            for (int t = 0; t < 4 && i0 + t < nt; ++t) {
+                const int i = i0 + t, st = i % kStages;
+                const int src = lane < kNodes ? t * kNodes + lane : 0;
+                const int jj = __shfl_sync(0xffffffffu, jc, src);   // lanes 0..7: node nl = lane
+                const int uu = __shfl_sync(0xffffffffu, uc, src);
+                if (lane == 0 && i >= kStages && !abort_sh &&
+                    !mbar_wait(smem_u32(&bar_empty[st]), (uint32_t)(((i / kStages) - 1) & 1))) {
+                    atomicOr(w.status, kStatusTimeout);
+                    abort_sh = 1;
+                }
+                if (__any_sync(0xffffffffu, abort_sh != 0)) {
+                    stop = true;
+                    break;
+                }
+                const uint32_t valid = __ballot_sync(0xffffffffu, lane < kNodes && jj >= 0);
+                if (lane < kNodes) sJ[st * kNodes + lane] = jj;
+                const uint32_t fb = smem_u32(&bar_full[st]);
+                __syncwarp();
+                if (lane == 0) {
+                    // the stage's only arrival, with the bytes every copy below will deliver
+                    mbar_expect_tx(fb, (uint32_t)__popc(valid) * (kNodeBytes + kR * 4 + (top ? 0 : kLW * 4)));
+                    const uint32_t sb = smem_u32(sB0 + (size_t)st * STAGE);
+                    for (int nl = 0; nl < kNodes; ++nl) {
+                        if (!((valid >> nl) & 1u)) continue;
+                        const int j = sJ[st * kNodes + nl];
+#pragma unroll
+                        for (int pl = 0; pl < kPlanes; ++pl)
+#pragma unroll
+                            for (int kb = 0; kb < KB; ++kb)
+                                tma_load_4d(sb + pl * P_BYTES + kb * (kTileN * 128) + nl * (kR * 128), map, kb * 64, 0,
+                                            pl, (int)(node0 + j), fb);
+                        bulk_load(smem_u32(sBv + st * kTileN + nl * kR), recb + (node0 + j) * sq.ns + kR * D, kR * 4, fb);
+                    }
+                }
+                __syncwarp();
+                // membership words of node nl = lane: row of its union parent uu
+                if (!top && lane < kNodes && ((valid >> lane) & 1u))
+                    bulk_load(smem_u32(sMask + (st * kNodes + lane) * kLW), memb + (int64_t)uu * w.mwords, kLW * 4, fb);
+                __syncwarp();
+                issued = i + 1;
+            }
+            jc = jn;
+            uc = un;
+        }
+        // copies still in flight must land before the block ends
+        if (lane == 0)
+            for (int i = max(0, issued - kStages); i < issued; ++i)
+                mbar_wait(smem_u32(&bar_full[i % kStages]), (uint32_t)((i / kStages) & 1));
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (lane 0)
+        if (lane == 0) {
+            const int jobs = nt * LT;
+            for (int q = 0; q < jobs && !abort_sh; ++q) {
+                const int i = q / LT, t = q % LT, st = i % kStages, slot = q & 1;
+                bool okw = true;
+                if (t == 0) okw = mbar_wait(smem_u32(&bar_full[st]), (uint32_t)((i / kStages) & 1));
+                if (okw && q >= 2) okw = mbar_wait(smem_u32(&bar_acc_empty[slot]), (uint32_t)(((q >> 1) - 1) & 1));
+                if (!okw) {
+                    atomicOr(w.status, kStatusTimeout);
+                    abort_sh = 1;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t d = tmem + (uint32_t)(slot * kTileN);
+                const uint32_t ta = tmem + kColA + (uint32_t)(t * (D / 2));
+                const uint64_t db = umma_desc(smem_u32(sB0 + (size_t)st * STAGE));
+#pragma unroll 1
+                for (int pk = 0; pk < kPlanes * KB; ++pk) {
+                    const int pass = pk / KB, kb = pk % KB;
+                    const uint64_t b1 = db + (uint64_t)((pass * P_BYTES + kb * (kTileN * 128)) >> 4);
+                    const uint32_t a1 = ta + (uint32_t)(kb * 32);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(d, a1 + (uint32_t)(kk * 8), b1 + (uint64_t)(kk * 2), (pk | kk) ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&bar_acc_full[slot]));
+            }
+        }
+        __syncwarp();
     } else {
-        // ---------------- epilogue: scores of tile i from accumulator i % 2 of each lane tile.
-        // Lane 0 of the first epilogue warp also issues the MMAs: tile i+1's before this
-        // warp drains tile i when its operands are already staged, else right after the
-        // drain, so the epilogue never waits on the producers while an accumulator is full.
-        const int ew = warp - kProducers / 32;
-        const int lt = ew >> 2, quad = warp & 3;      // TMEM lane quarter = warp % 4
-        const int row = lt * kTileM + quad * 32 + lane;
+        // ---------------- epilogue
         const int y = y0 + row;
         const bool ok = y < b.n_gl;
         const int64_t x = lane_of(b, s, g, ok ? y : 0);
         float* ex = w.e + x * w.es;
         float fmax = -INFINITY;
         int fcnt = 0;
-        const bool issuer = warp == kMmaWarp && lane == 0;
-        auto issue = [&](int i) {
-            const int st = i & 1;
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t pl0 = smem_u32(sB0 + (size_t)(kPlanes * st) * P_BYTES);
-            // descriptors advance by the operand offset in 16-byte units (start-address field);
-            // loops kept rolled so the compiler does not hold every descriptor in registers
-#pragma unroll 1
-            for (int t = 0; t < LT; ++t) {
-                const uint32_t d = tmem + (uint32_t)((t * 2 + st) * kTileN);
-                const uint64_t da = umma_desc(smem_u32(sA + t * A_BYTES));
-                const uint64_t db = umma_desc(pl0);
-#pragma unroll 1
-                for (int pk = 0; pk < kPlanes * KB; ++pk) {
-                    const int pass = pk / KB, kb = pk % KB;
-                    const uint64_t a1 = da + (uint64_t)((kb * (kTileM * 128)) >> 4);
-                    const uint64_t b1 = db + (uint64_t)((pass * P_BYTES + kb * (kTileN * 128)) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(d, a1 + (uint64_t)(kk * 2), b1 + (uint64_t)(kk * 2), (pk | kk) ? 1u : 0u);
-                }
-            }
-            mma_commit(smem_u32(&bar_acc_full[st]));
-        };
-        // operands of tile i staged and its accumulators drained (by tile i-2's epilogue)
-        auto ready = [&](int i) -> bool {
-            const int st = i & 1;
-            if (!mbar_test(smem_u32(&bar_full[st]), (uint32_t)((i >> 1) & 1))) return false;
-            return i < 2 || mbar_test(smem_u32(&bar_acc_empty[st]), (uint32_t)(((i >> 1) - 1) & 1));
-        };
-        auto issue_blocking = [&](int i) {
-            const int st = i & 1;
-            bool okw = mbar_wait(smem_u32(&bar_full[st]), (uint32_t)((i >> 1) & 1));
-            if (okw && i >= 2) okw = mbar_wait(smem_u32(&bar_acc_empty[st]), (uint32_t)(((i >> 1) - 1) & 1));
-            if (!okw) {
-                atomicOr(w.status, kStatusTimeout);
-                abort_sh = 1;
-            }
-            if (!abort_sh) issue(i);
-        };
-        if (issuer) issue_blocking(0);
         for (int i = 0; i < nt; ++i) {
-            bool issued_next = false;
-            if (issuer && i + 1 < nt && !abort_sh && ready(i + 1)) {
-                issue(i + 1);
-                issued_next = true;
-            }
-            __syncwarp();
-            const int st = i & 1;
-            if (!mbar_wait(smem_u32(&bar_acc_full[st]), (uint32_t)((i >> 1) & 1))) {
+            const int st = i % kStages, q = i * LT + lt, slot = q & 1;
+            if (!mbar_wait(smem_u32(&bar_acc_full[slot]), (uint32_t)((q >> 1) & 1))) {
                 atomicOr(w.status, kStatusTimeout);
                 abort_sh = 1;
             }
             if (__any_sync(0xffffffffu, abort_sh != 0)) break;   // warp-uniform: tcgen05.ld below is collective
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // the stage's metadata stays valid until this epilogue releases it: copy it out
+            // the stage (node ids, b, membership) is complete: its full barrier has fired
+            mbar_wait(smem_u32(&bar_full[st]), (uint32_t)((i / kStages) & 1));
             int jv[kNodes];
-#pragma unroll
-            for (int nl = 0; nl < kNodes; ++nl) jv[nl] = sJ[st * kNodes + nl];
             uint32_t member = 0;
-            {
-                const uint4* mk = reinterpret_cast<const uint4*>(sMask + st * kLW * kNodes + (row >> 5) * kNodes);
-                const uint4 m0 = mk[0], m1 = mk[1];
-                const uint32_t mws[kNodes] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-                for (int nl = 0; nl < kNodes; ++nl) member |= ((mws[nl] >> lane) & 1u) << nl;
+            for (int nl = 0; nl < kNodes; ++nl) {
+                jv[nl] = sJ[st * kNodes + nl];
+                const bool mb = jv[nl] >= 0 && (top || ((sMask[(st * kNodes + nl) * kLW + (row >> 5)] >> lane) & 1u));
+                member |= (mb ? 1u : 0u) << nl;
             }
             const float4* bv4 = reinterpret_cast<const float4*>(sBv + st * kTileN);
             float best[kNodes];
 #pragma unroll
             for (int pr = 0; pr < kNodes / 2; ++pr) {
                 float v[32];
-                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((lt * 2 + st) * kTileN + pr * 2 * kR), v);
+                tmem_ld32(tmem + tlane + (uint32_t)(slot * kTileN + pr * 2 * kR), v);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     float bb = -INFINITY;
@@ -477,8 +461,8 @@ __global__ void __launch_bounds__(kProducers + 128 * LT, 1) k_score_tc(Batch b, 
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            mbar_arrive(smem_u32(&bar_acc_empty[st]));
-            if (issuer && i + 1 < nt && !issued_next) issue_blocking(i + 1);
+            mbar_arrive(smem_u32(&bar_acc_empty[slot]));
+            mbar_arrive(smem_u32(&bar_empty[st]));
             // scores out: -inf off the frontier; 16-byte stores where 4 nodes are consecutive
 #pragma unroll
             for (int nl = 0; nl < kNodes; ++nl) {
@@ -512,8 +496,8 @@ __global__ void __launch_bounds__(kProducers + 128 * LT, 1) k_score_tc(Batch b, 
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (warp == kMmaWarp)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
 }
 
 template <int D, int LT>
@@ -523,15 +507,15 @@ cudaError_t launch_tc(const Batch& b, const Work& w, int it, float scale, cudaSt
     dim3 grid(nb, pairs, b.n_groups);
     const size_t smem = score_tc_smem_lt(D, LT);
     cudaFuncSetAttribute(k_score_tc<D, LT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_score_tc<D, LT><<<grid, kProducers + 128 * LT, smem, st>>>(b, w, it, scale);
+    k_score_tc<D, LT><<<grid, 64 + 128 * LT, smem, st>>>(b, w, it, scale);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t score_tc_smem_lt(int d, int lt) {
-    return (size_t)(d / 64) * 128 * 128 * (lt + 2 * kPlanes) + 2 * kTileN * 4 + 2 * 4 * lt * kNodes * 4 +
-           2 * kNodes * 4 + 2 * kProducers * 4 + 1024;
+    return (size_t)kStages * kPlanes * (d / 64) * kTileN * 128 + (size_t)kStages * kTileN * 4 +
+           (size_t)kStages * kNodes * 4 * lt * 4 + (size_t)kStages * kNodes * 4 + 1024;
 }
 
 size_t score_tc_smem(int d) { return score_tc_smem_lt(d, 2); }
