@@ -42,9 +42,12 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 float score_scale(int d) { return (float)(1.0 / sqrt((double)d)); }
 
-// TMA map over one level's fp16 planes: (dim, plane r, hi/lo, node over all KV heads),
-// boxes of 64 dims x R planes of one node, 128-byte swizzle (the MMA operand layout).
-bool encode_plane_map(CUtensorMap* map, const float* rec, int d, int R, int64_t nodes, int ns) {
+// TMA maps of one level (fp16 planes viewed as (dim, plane r, hi/lo, node over all KV
+// heads), 128-byte swizzle = the MMA operand layout; b viewed as (r, node)):
+//   maps[0] planes, boxes of 64 dims x R planes x 1 node
+//   maps[1] planes, boxes of 64 dims x R planes x 4 nodes
+//   maps[2] b, boxes of R values x 4 nodes
+bool encode_level_maps(CUtensorMap* maps, const float* rec, int d, int R, int64_t nodes, int ns) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
@@ -56,11 +59,21 @@ bool encode_plane_map(CUtensorMap* map, const float* rec, int d, int R, int64_t 
     }
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)R, 2, (cuuint64_t)nodes};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)R * d * 2, (cuuint64_t)ns * 4};
-    const cuuint32_t box[4] = {64, (cuuint32_t)R, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<float*>(rec), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    for (int k = 0; k < 2; ++k) {
+        const cuuint32_t box[4] = {64, (cuuint32_t)R, 1, k == 0 ? 1u : 4u};
+        if (encode(&maps[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<float*>(rec), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    const cuuint64_t bdims[2] = {(cuuint64_t)R, (cuuint64_t)nodes};
+    const cuuint64_t bstrides[1] = {(cuuint64_t)ns * 4};
+    const cuuint32_t bbox[2] = {(cuuint32_t)R, 4};
+    const cuuint32_t bestr[2] = {1, 1};
+    return encode(&maps[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(rec) + (int64_t)R * d, bdims,
+                  bstrides, bbox, bestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -365,11 +378,9 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         const int64_t segs = segs_per_split(1, t->g.C);
         s_cap = std::max<int64_t>(s_cap, (nseg_max + segs - 1) / segs);
     }
-    // union parents of a scored level sit at level >= 2
-    int64_t cap2 = 1;
-    for (auto* t : dec->trees)
-        if (t->g.L >= 2) cap2 = std::max<int64_t>(cap2, t->cap[2]);
-    w.ms = cap2;
+    // union lists whose lane masks are transposed: parents of a scored level (level >= 2)
+    // and the kept level-1 chunks attention gathers
+    w.ms = cap1;
     w.mwords = (max_queries * dec->G + 255) / 256 * 8;
     w.lanes_cap = dec->lanes_cap;
     w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
@@ -402,7 +413,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     const size_t lcnt_off = off;
     off += up256((size_t)(kMaxL + 1) * dec->lanes_cap * 4);
     const size_t tmap_off = off;
-    off += up256((size_t)n_seq * (kMaxL + 1) * sizeof(CUtensorMap));
+    off += up256((size_t)n_seq * (kMaxL + 1) * kMapsPerLevel * sizeof(CUtensorMap));
     const size_t ctr_off = off;
     off += up256((size_t)kCtrCount * 8);
     const size_t status_off = off;
@@ -433,14 +444,14 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     // TMA maps of the trees' fp16 planes, one per (sequence, level), for the tensor scorer
     w.tmaps = nullptr;
     if (dec->all_r16) {
-        std::vector<CUtensorMap> maps((size_t)n_seq * (kMaxL + 1));
+        std::vector<CUtensorMap> maps((size_t)n_seq * (kMaxL + 1) * kMapsPerLevel);
         memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
         bool ok = true;
         for (int s = 0; s < n_seq && ok; ++s) {
             const zha_tree* t = dec->trees[s];
             for (int l = 1; l <= t->g.L && ok; ++l)
-                ok = encode_plane_map(&maps[(size_t)s * (kMaxL + 1) + l], t->rec[l], t->g.d, t->g.R,
-                                      (int64_t)t->g.n_kv_heads * t->cap[l], t->ns);
+                ok = encode_level_maps(&maps[((size_t)s * (kMaxL + 1) + l) * kMapsPerLevel], t->rec[l], t->g.d, t->g.R,
+                                       (int64_t)t->g.n_kv_heads * t->cap[l], t->ns);
         }
         if (ok) {
             CUtensorMap* dst = reinterpret_cast<CUtensorMap*>(base + tmap_off);

@@ -7,7 +7,8 @@
 // A_x = {0} U tokens of the level-1 chunks x kept U tail.  Used when a group holds many
 // lanes, so that a tile of 128 lanes x 128 token positions is a dense contraction:
 //   S = Q K^T      tcgen05.mma kind::f16 (bf16 x bf16 products are exact, f32 accumulate)
-//   P = exp(s S - m) on the lanes' own positions (0 elsewhere), split P = P_hi + P_lo (bf16)
+//   P = exp(s S - m) on the lanes' own positions (0 elsewhere), split P = P_hi + P_lo (bf16,
+//   each rounded to 8 significant bits by an integer add on its bits)
 //   O += P_hi V + P_lo V   (P carries ~2^-17 relative error; V is exact)
 // O stays in tensor memory for the whole split; the running max m is raised lazily (only
 // when a tile's max exceeds it by more than 8, then O and the sum are rescaled), so most
@@ -36,6 +37,12 @@ constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tenso
 constexpr int kBlock = kRows * 128;   // bytes of one 128-byte-wide block of 128 rows
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
@@ -134,10 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     unsigned char* sPh = sV0 + 2 * KBD * kBlock;            // 2 blocks
     unsigned char* sPl = sPh + 2 * kBlock;                  // 2 blocks
     int32_t* s_tok0 = reinterpret_cast<int32_t*>(sPl + 2 * kBlock);  // [2][kPos] token (-1: none)
-    int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: chunk id, -1 all, -2 none
+    int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: union index, -1 all, -2 none
     uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_slot0 + 2 * kPos);   // [2][kPos] slot of each position
     uint32_t* s_valid0 = reinterpret_cast<uint32_t*>(s_pslot0 + 2 * kPos); // [2][kPos/32] positions with a token
-    float* s_xmax = reinterpret_cast<float*>(s_valid0 + 2 * (kPos / 32));  // [2][kRows] tile max per half
+    uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][kPos][4] lane masks per slot
+    float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [2][kRows] tile max per half
     float* s_xsum = s_xmax + 2 * kRows;                                     // [2][kRows] row sums per half
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_sh;
@@ -192,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int y = y0 + row;
     const bool y_ok = y < b.n_gl;
     const int64_t x = lane_of(b, s, g, y_ok ? y : 0);
-    const uint32_t* kb1 = w.kept[1] + x * w.W[1];
     const uint32_t lane_t = (uint32_t)((warp & 3) * 32) << 16;
     float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in both warps of a row
 
@@ -204,35 +211,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 
     // Tokens of tile p0 into buffer st (threads 0..127, one position each): sink segment
     // (position 0 only), kept chunks, tail.  Also the slot table: slot k of the tile is the
-    // k-th segment it touches; s_slot holds its chunk id (-1: every lane, -2: none) and
-    // s_pslot the slot of each position; s_valid marks positions holding a token.
+    // k-th segment it touches; s_slot holds the segment's index in the group's union list
+    // (-1: every lane, -2: none), s_mw the 32-lane membership words of the CTA's 128 lanes
+    // for that union chunk, s_pslot the slot of each position; s_valid marks positions
+    // holding a token.  Positions and tokens fit 32 bits (caches hold < 2^31 rows).
+    const int cs = (C & (C - 1)) == 0 ? __ffs((int)C) - 1 : -1;   // shift for power-of-two C
+    const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.y * 4;
     auto resolve = [&](int64_t p0, int st) {
         if (tid < kPos) {
-            const int64_t pp = p0 + tid;
+            const int pp = (int)p0 + tid;
+            const int segl = cs >= 0 ? (pp >> cs) : pp / (int)C;     // segment within the split
+            const int off = pp - segl * (int)C;
             int32_t tok = -1, code = -2;
             if (pp < npos) {
-                const int64_t seg = sg0 + pp / C, off = pp % C;
+                const int64_t seg = sg0 + segl;
                 if (has_sink && seg == 0) {
                     code = -1;
                     if (off == 0) tok = 0;
                 } else {
-                    const int64_t k = seg - has_sink;
+                    const int k = (int)(seg - has_sink);
                     if (k < nu) {
-                        const int64_t j = ul[k];
-                        const int64_t t = j * C + off;
-                        code = (int32_t)j;
-                        if (t != 0) tok = (int32_t)t;
+                        const int t = ul[k] * (int)C + off;
+                        code = k;
+                        if (t != 0) tok = t;
                     } else {
-                        const int64_t t = tail0 + (k - nu) * C + off;
+                        const int64_t t = tail0 + (int64_t)(k - nu) * C + off;
                         code = -1;
                         if (t < N) tok = (int32_t)t;
                     }
                 }
             }
-            const int slot = (int)((p0 + tid) / C - p0 / C);
+            const int p0s = cs >= 0 ? ((int)p0 >> cs) : (int)p0 / (int)C;
+            const int slot = segl - p0s;
             s_tok0[st * kPos + tid] = tok;
             s_pslot0[st * kPos + tid] = (uint8_t)slot;
-            if (tid == 0 || (p0 + tid) % C == 0) s_slot0[st * kPos + slot] = code;
+            if (tid == 0 || off == 0) {
+                s_slot0[st * kPos + slot] = code;
+                // lane masks land asynchronously with the tile's K/V gather (same commit
+                // group, waited at the top of the tile that uses them); zero-filled if none
+                const uint32_t* src = memb + (int64_t)(code >= 0 ? code : 0) * w.mwords;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(s_mw0 + (st * kPos + slot) * 4)),
+                             "l"(src), "r"(code >= 0 ? 16u : 0u)
+                             : "memory");
+            }
             const unsigned vb = __ballot_sync(0xffffffffu, tok >= 0);
             if (lane == 0) s_valid0[st * (kPos / 32) + warp] = vb;
         }
@@ -279,29 +300,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         }
         __syncwarp();
 
-        // This row's membership on its half of the tile: one bitmap load per chunk slot,
-        // all independent, expanded to positions through the slot index.
+        // This row's membership on its half of the tile, slot by slot from the staged lane
+        // masks: a slot covers a run of consecutive positions.
         uint64_t mem = 0;
         {
-            const uint8_t* ps = s_pslot0 + st * kPos + half * kHalf;
-            const int k0 = ps[0], k1 = ps[kHalf - 1];
-            uint64_t slotbits = 0;
-            for (int kb = k0; kb <= k1; kb += 16) {
-                uint32_t wv[16];
-                int32_t code[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    code[i] = kb + i <= k1 ? s_slot0[st * kPos + kb + i] : -2;
-                    wv[i] = code[i] >= 0 ? __ldg(kb1 + (code[i] >> 5)) : 0u;
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t bit = code[i] == -1 ? 1u : (code[i] >= 0 ? (wv[i] >> (code[i] & 31)) & 1u : 0u);
-                    slotbits |= (uint64_t)bit << (kb + i - k0);
+            const uint8_t* ps = s_pslot0 + st * kPos;
+            const int hs = half * kHalf;
+            const int k0 = ps[hs], k1 = ps[hs + kHalf - 1];
+            const int lw = row >> 5, bit = row & 31;
+            // slot k spans positions [k C - o0, (k+1) C - o0) of the tile, o0 = p0 mod C
+            const int o0 = (int)(p0 % C);
+            for (int k = k0; k <= k1; ++k) {
+                const int32_t code = s_slot0[st * kPos + k];
+                const bool in = code == -1 || (code >= 0 && ((s_mw0[(st * kPos + k) * 4 + lw] >> bit) & 1u));
+                if (in) {
+                    const int a = max(k * (int)C - o0, hs) - hs, e = min((k + 1) * (int)C - o0, hs + kHalf) - hs;
+                    const uint64_t hi_mask = e >= 64 ? ~0ull : ((1ull << e) - 1ull);
+                    mem |= hi_mask & ~((1ull << a) - 1ull);
                 }
             }
-#pragma unroll 8
-            for (int i = 0; i < kHalf; ++i) mem |= ((slotbits >> (ps[i] - k0)) & 1ull) << i;
             const uint32_t* vw = s_valid0 + st * (kPos / 32) + half * 2;
             mem &= (uint64_t)vw[0] | ((uint64_t)vw[1] << 32);
             if (!y_ok) mem = 0;
@@ -360,17 +377,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             uint32_t hi[8], lo[8];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
-                const float e0 = exp2f(fmaf(sl, v[i], -ml));
-                const float e1 = exp2f(fmaf(sl, v[i + 1], -ml));
+                const float e0 = ex2_approx(fmaf(sl, v[i], -ml));
+                const float e1 = ex2_approx(fmaf(sl, v[i + 1], -ml));
                 const float p0v = ((mem >> (c * 16 + i)) & 1ull) ? e0 : 0.0f;
                 const float p1v = ((mem >> (c * 16 + i + 1)) & 1ull) ? e1 : 0.0f;
                 lsum += p0v;
                 lsum += p1v;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0v, p1v);
-                const float2 hf = __bfloat1622float2(h);
-                const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0v - hf.x, p1v - hf.y);
-                hi[i / 2] = *reinterpret_cast<const uint32_t*>(&h);
-                lo[i / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+                // bf16 hi = p rounded to 8 significant bits (integer add on the bits), lo =
+                // the exact remainder rounded likewise; packed by byte permutes, so the split
+                // stays off the conversion unit
+                const uint32_t h0 = (__float_as_uint(p0v) + 0x8000u) & 0xffff0000u;
+                const uint32_t h1 = (__float_as_uint(p1v) + 0x8000u) & 0xffff0000u;
+                const uint32_t l0 = __float_as_uint(p0v - __uint_as_float(h0)) + 0x8000u;
+                const uint32_t l1 = __float_as_uint(p1v - __uint_as_float(h1)) + 0x8000u;
+                hi[i / 2] = __byte_perm(h0, h1, 0x7632);
+                lo[i / 2] = __byte_perm(l0, l1, 0x7632);
             }
             // positions 64 half + 16 c .. +15 are 16-byte chunks 8 half + 2c, +1 of this row
             const int c16 = half * 8 + 2 * c;
@@ -397,19 +418,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                              idesc_bf16(D, 1), (first_pv && pass == 0 && ks == 0) ? 0u : 1u);
                 }
             }
-            commit(su32(&mbar));
+            // no commit: the next tile's S commit tracks these MMAs too (a commit covers every
+            // earlier tcgen05 operation of the issuing thread), so P V overlaps the next
+            // tile's gather wait, slot table and membership
         }
         __syncwarp();
-        if (!wait_phase(su32(&mbar), phase) && lane == 0) {
-            atomicOr(w.status, kStatusTimeout);
-            abort_sh = 1;
-        }
-        phase ^= 1;
         first_pv = false;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        __syncthreads();
         if (abort_sh) break;
     }
+    // the last P V: one more commit, then O is final
+    if (tid == 0) commit(su32(&mbar));
+    __syncwarp();
+    if (!wait_phase(su32(&mbar), phase) && lane == 0) {
+        atomicOr(w.status, kStatusTimeout);
+        abort_sh = 1;
+    }
+    phase ^= 1;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     // partial (o, m, l) of every lane row of the tile: each warp writes its half of o
     s_xsum[half * kRows + row] = lsum;
@@ -444,12 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
     return (size_t)(4 * kbd + 4) * kBlock + 2 * kPos * 4 + 2 * kPos * 4 + 2 * kPos + 2 * (kPos / 32) * 4 +
-           4 * kRows * 4 + 1024;
+           2 * kPos * 4 * 4 + 4 * kRows * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
     if (max_splits <= 0) return cudaSuccess;
     ProfScope ps_("k_attn_tc", st);
+    cudaError_t e = launch_member(b, w, 0, 1, st);   // lane masks of the kept level-1 chunks
+    if (e != cudaSuccess) return e;
     const int lane_tiles = (b.n_gl + kRows - 1) / kRows;
     dim3 grid((unsigned)max_splits, lane_tiles, b.n_groups);
     const size_t smem = attn_tc_smem(b.d);

@@ -33,6 +33,8 @@ struct SeqDev {
     const __nv_bfloat16* V;
 };
 
+constexpr int kMapsPerLevel = 3;     // planes by 1 node, planes by 4 nodes, b by 4 nodes
+
 // Counter slots (unsigned long long).
 constexpr int kCtrUnionNodes = 0;              // + level
 constexpr int kCtrLaneNodes = kMaxL + 1;       // + level
@@ -58,7 +60,7 @@ struct Work {
     uint32_t* memb;                  // [groups_cap][ms][mwords] union parents' lane masks (tensor scorer)
     int64_t ms;
     int32_t mwords;                  // a multiple of 8 covering every 256-lane pair of a group
-    const CUtensorMap* tmaps;        // [n_seq][kMaxL + 1] fp16 plane maps of the trees' levels (or null)
+    const CUtensorMap* tmaps;        // [n_seq][kMaxL + 1][kMapsPerLevel] TMA maps of the trees' levels (or null)
     uint32_t* lane_max;              // [(kMaxL+1)][lanes_cap] frontier max score per lane (ordered bits)
     int32_t* lane_cnt;               // [(kMaxL+1)][lanes_cap] frontier size per lane
     unsigned long long* ctr;         // kCtrCount counters

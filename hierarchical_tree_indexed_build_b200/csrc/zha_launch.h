@@ -50,6 +50,9 @@ cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t H
 // sets of level L_s - it + 1); mode 1 prepares attention (union of level-1 kept sets).
 cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaStream_t st);
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
+// Transposed lane masks of a union level (mode 0: parents of iteration it's candidates;
+// mode 1: kept level-1 chunks) into w.memb.
+cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaStream_t st);
 cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
 // Lanes per group from which the automatic choice scores on tensor cores.
 constexpr int kTensorScoreMinLanes = 64;

@@ -148,6 +148,7 @@ extern "C" zha_status zha_sparse_attn_static(const void* K, const void* V, int64
     b.n_groups = Hkv;
     b.Q = static_cast<const __nv_bfloat16*>(Q);
     b.p = 1.0f;
+    b.attn_path = 1;   // CUDA-core attention: it reads the kept bitmaps directly, no lane masks
 
     const float scale = (float)(1.0 / sqrt((double)d));
     if (launch_union(b, w, 0, 1, st) != cudaSuccess || launch_attn(b, w, splits, scale, st) != cudaSuccess ||

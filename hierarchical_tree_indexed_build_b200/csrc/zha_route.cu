@@ -293,7 +293,7 @@ constexpr int kSelThreads = 512;
 constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
-constexpr int kUn = 4;               // 128-candidate blocks per warp in flight
+constexpr int kUn = 2;               // 128-candidate blocks per warp in flight
 // masses are fixed point with 2^39 for exp(0); sums of <= 2^24 candidates stay below 2^63
 
 // Ascending key order == (e descending, node index ascending).
@@ -390,14 +390,21 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const int k0 = bk * 128 + 4 * lane;
         ev = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         j0 = -1;
+        if (contig) {
+            // predicated, not branched: lanes past the end read node 0 and mask it
+            const bool in = k0 < nc;
+            const int jj = cand_j(in ? k0 : 0);
+            const float4 x = *reinterpret_cast<const float4*>(e + jj);   // rows are padded to 128 floats
+            j0 = in ? jj : -1;
+            ev.x = in ? x.x : -INFINITY;
+            ev.y = k0 + 1 < nc ? x.y : -INFINITY;
+            ev.z = k0 + 2 < nc ? x.z : -INFINITY;
+            ev.w = k0 + 3 < nc ? x.w : -INFINITY;
+            return;
+        }
         if (k0 >= nc) return;
         j0 = cand_j(k0);
-        if (contig) {
-            ev = *reinterpret_cast<const float4*>(e + j0);   // rows are padded to 128 floats
-            if (k0 + 1 >= nc) ev.y = -INFINITY;
-            if (k0 + 2 >= nc) ev.z = -INFINITY;
-            if (k0 + 3 >= nc) ev.w = -INFINITY;
-        } else {
+        {
             ev.x = e[j0];
             if (k0 + 1 < nc) ev.y = e[cand_j(k0 + 1)];
             if (k0 + 2 < nc) ev.z = e[cand_j(k0 + 2)];
@@ -433,11 +440,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             wv |= __shfl_xor_sync(kFull, wv, 1);
             wv |= __shfl_xor_sync(kFull, wv, 2);
             wv |= __shfl_xor_sync(kFull, wv, 4);
-            if (jf >= 0 && (jf & 31) == 0 && jl == jf + 28) {
-                if ((lane & 7) == 0 && wv) outw[jf >> 5] = wv;
-            } else if (nib) {
-                atomicOr(outw + (j0 >> 5), nib << (j0 & 31));
-            }
+            const bool whole = jf >= 0 && (jf & 31) == 0 && jl == jf + 28;
+            if (whole && (lane & 7) == 0 && wv) outw[jf >> 5] = wv;
+            if (!whole && nib) atomicOr(outw + (j0 >> 5), nib << (j0 & 31));
         } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -456,10 +461,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         if (threadIdx.x == 0) s_nkeys = 0;
         __syncthreads();
         for_cands([&](int bk, const float4 ev4, int j0) {
-        const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+            const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+            // -inf (off the frontier) gives mass 0 and the last bin: computed without branches,
+            // only the atomic is predicated
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                if (v[c] > -INFINITY) atomicAdd(&hist[sm.bin(v[c])], sm.mass(v[c]));
+            for (int c = 0; c < 4; ++c) {
+                const unsigned long long ms = sm.mass(v[c]);
+                const int bn = sm.bin(v[c]);
+                if (ms) atomicAdd(&hist[bn], ms);
+            }
         });
         __syncthreads();
         unsigned long long zloc = 0;
@@ -508,17 +518,33 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     unsigned long long cnt = 0;
     for_cands([&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
-        uint32_t nib = 0;
+        uint32_t nib = 0, col = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            if (!(v[c] > -INFINITY)) continue;
+            const bool ok = v[c] > -INFINITY;
             const int bn = sm.bin(v[c]);
-            if (bn < bstar) {
-                nib |= 1u << c;
-            } else if (bn == bstar) {
-                const unsigned idx = atomicAdd(&s_nkeys, 1u);
-                if (idx < (unsigned)kCap) keys[idx] = sel_key(v[c], jof(bk, j0, c));
+            nib |= (ok && bn < bstar ? 1u : 0u) << c;
+            col |= (ok && bn == bstar ? 1u : 0u) << c;
+        }
+        // boundary-bin candidates: one shared-memory atomic per warp reserves their slots
+        if (__any_sync(kFull, col != 0)) {
+            const int mine = __popc(col);
+            int incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += t;
             }
+            unsigned base0 = 0;
+            if (lane == 31) base0 = atomicAdd(&s_nkeys, (unsigned)incl);
+            base0 = __shfl_sync(kFull, base0, 31);
+            unsigned idx = base0 + (unsigned)(incl - mine);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if ((col >> c) & 1u) {
+                    if (idx < (unsigned)kCap) keys[idx] = sel_key(v[c], jof(bk, j0, c));
+                    ++idx;
+                }
         }
         cnt += __popc(nib);
         put_bits(bk, nib, j0);

@@ -17,10 +17,10 @@
 //
 // Pipeline (one CTA per SM, persistent over its node tiles of 8 nodes; LT = 1 or 2 lane
 // tiles of 128 lanes per CTA share every node tile):
-//   warp 0      loader: TMA copies of each node's two fp16 planes (boxes of 64 dims x 16
-//               planes, 128-byte swizzled by the copy engine into the MMA operand layout),
-//               plus bulk copies of the node's b values and of the CTA lanes' membership
-//               words, into one of 3 shared-memory stages;
+//   warp 0      loader: TMA copies of the nodes' two fp16 planes (boxes of 64 dims x 16
+//               planes x 4 consecutive nodes, 128-byte swizzled by the copy engine into the
+//               MMA operand layout; 1-node boxes when C is not a multiple of 4), of their b
+//               values, and of the CTA lanes' membership words, into one of 3 stages;
 //   warp 1      MMA issuer: per lane tile, 2 planes x d/16 tcgen05.mma kind::f16 with the
 //               query tile (A) in tensor memory and the node tile (B) in shared memory;
 //   warps 2..   epilogue, 4 per lane tile: tensor memory -> max over planes + b -> scores.
@@ -143,15 +143,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Lanes' kept bits of the level above, transposed: memb[grp][u][w] bit t = lane 32 w + t
-// kept union parent u.  Grid (parent chunks, lane words, groups); a warp covers 32 parents.
-__global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it) {
+// Lanes' kept bits of one level, transposed over the group's union list of that level:
+// memb[grp][u][w] bit t = lane 32 w + t kept union node u.  Mode 0: the level above the one
+// routing iteration `it` scores (its nodes are the candidates' parents); mode 1: level 1
+// (the chunks attention gathers).  Grid (chunks, lane words, groups); a warp covers 32 nodes.
+__global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mode) {
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
     const SeqDev& sq = b.seqs[s];
-    const int lev = sq.L - it;
-    if (lev < 1 || lev == sq.L) return;           // top level: no parents
-    const int pl = lev + 1;
+    int pl;
+    if (mode == 0) {
+        const int lev = sq.L - it;
+        if (lev < 1 || lev == sq.L) return;       // top level: no parents
+        pl = lev + 1;
+    } else {
+        if (sq.T == 0) return;                    // dense attention: no union
+        pl = 1;
+    }
     const int nu = w.ucount[grp];
     const int lw = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int y = lw * 32 + lane;
@@ -191,6 +199,13 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
         :
         : "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :
+        : "r"(dst), "l"(map), "r"(x), "r"(y), "r"(mbar)
         : "memory");
 }
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
@@ -244,6 +259,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     const int nt = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;   // tiles of this block
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int y0 = blockIdx.y * (kTileM * LT);
+    const bool runs = top || (C % 4 == 0);
 
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
@@ -306,8 +322,13 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     if (warp == 0) {
         // ---------------- loader.  Lanes compute the node ids of 4 tiles at a time (one
         // candidate each), a batch ahead of use; lane 0 issues the copies.
-        const CUtensorMap* map = w.tmaps + (int64_t)s * (kMaxL + 1) + lev;
-        asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+        const CUtensorMap* maps = w.tmaps + ((int64_t)s * (kMaxL + 1) + lev) * kMapsPerLevel;
+#pragma unroll
+        for (int k = 0; k < kMapsPerLevel; ++k)
+            asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(maps + k) : "memory");
+        // candidates come in aligned runs of 4 consecutive nodes with one parent when C % 4 == 0
+        // (and at the top level): one 4-node box per plane and K block, one for b, one
+        // membership row per run
         const float* recb = sq.rec[lev];
         const int64_t node0 = (int64_t)g * sq.cap[lev];               // first node of this KV head
         const int32_t* ul = w.ulist + (int64_t)grp * w.us;
@@ -348,28 +369,33 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                     stop = true;
                     break;
                 }
-                const uint32_t valid = __ballot_sync(0xffffffffu, lane < kNodes && jj >= 0);
+                uint32_t valid = __ballot_sync(0xffffffffu, lane < kNodes && jj >= 0);
+                if (runs) valid &= 0x11u;                  // a run is loaded whole from its first node
                 if (lane < kNodes) sJ[st * kNodes + lane] = jj;
                 const uint32_t fb = smem_u32(&bar_full[st]);
                 __syncwarp();
                 if (lane == 0) {
                     // the stage's only arrival, with the bytes every copy below will deliver
-                    mbar_expect_tx(fb, (uint32_t)__popc(valid) * (kNodeBytes + kR * 4 + (top ? 0 : kLW * 4)));
+                    const uint32_t per = runs ? 4 * kNodeBytes + 4 * kR * 4 : kNodeBytes + kR * 4;
+                    mbar_expect_tx(fb, (uint32_t)__popc(valid) * (per + (top ? 0 : kLW * 4)));
                     const uint32_t sb = smem_u32(sB0 + (size_t)st * STAGE);
                     for (int nl = 0; nl < kNodes; ++nl) {
                         if (!((valid >> nl) & 1u)) continue;
-                        const int j = sJ[st * kNodes + nl];
+                        const int wn = (int)(node0 + sJ[st * kNodes + nl]);
 #pragma unroll
                         for (int pl = 0; pl < kPlanes; ++pl)
 #pragma unroll
                             for (int kb = 0; kb < KB; ++kb)
-                                tma_load_4d(sb + pl * P_BYTES + kb * (kTileN * 128) + nl * (kR * 128), map, kb * 64, 0,
-                                            pl, (int)(node0 + j), fb);
-                        bulk_load(smem_u32(sBv + st * kTileN + nl * kR), recb + (node0 + j) * sq.ns + kR * D, kR * 4, fb);
+                                tma_load_4d(sb + pl * P_BYTES + kb * (kTileN * 128) + nl * (kR * 128), maps + (runs ? 1 : 0),
+                                            kb * 64, 0, pl, wn, fb);
+                        if (runs)
+                            tma_load_2d(smem_u32(sBv + st * kTileN + nl * kR), maps + 2, 0, wn, fb);
+                        else
+                            bulk_load(smem_u32(sBv + st * kTileN + nl * kR), recb + (int64_t)wn * sq.ns + kR * D, kR * 4, fb);
                     }
                 }
                 __syncwarp();
-                // membership words of node nl = lane: row of its union parent uu
+                // membership words of node (or run) nl = lane: row of its union parent uu
                 if (!top && lane < kNodes && ((valid >> lane) & 1u))
                     bulk_load(smem_u32(sMask + (st * kNodes + lane) * kLW), memb + (int64_t)uu * w.mwords, kLW * 4, fb);
                 __syncwarp();
@@ -437,7 +463,8 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
 #pragma unroll
             for (int nl = 0; nl < kNodes; ++nl) {
                 jv[nl] = sJ[st * kNodes + nl];
-                const bool mb = jv[nl] >= 0 && (top || ((sMask[(st * kNodes + nl) * kLW + (row >> 5)] >> lane) & 1u));
+                const int ms = runs ? (nl & ~3) : nl;   // a run's nodes share their parent's row
+                const bool mb = jv[nl] >= 0 && (top || ((sMask[(st * kNodes + ms) * kLW + (row >> 5)] >> lane) & 1u));
                 member |= (mb ? 1u : 0u) << nl;
             }
             const float4* bv4 = reinterpret_cast<const float4*>(sBv + st * kTileN);
@@ -520,14 +547,20 @@ size_t score_tc_smem_lt(int d, int lt) {
 
 size_t score_tc_smem(int d) { return score_tc_smem_lt(d, 2); }
 
+cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaStream_t st) {
+    const int lw = (b.n_gl + 31) / 32;
+    int nbm = (int)((w.ms + 255) / 256);
+    nbm = nbm < 1 ? 1 : (nbm > 148 ? 148 : nbm);
+    k_member<<<dim3(nbm, lw, b.n_groups), 256, 0, st>>>(b, w, it, mode);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
     ProfScope ps_("k_score_tc", st);
     if (it > 0) {
         // membership words of the group's union parents (the level above the scored one)
-        const int lw = (b.n_gl + 31) / 32;
-        int nbm = (int)((w.ms + 255) / 256);
-        nbm = nbm < 1 ? 1 : (nbm > 148 ? 148 : nbm);
-        k_member<<<dim3(nbm, lw, b.n_groups), 256, 0, st>>>(b, w, it);
+        const cudaError_t e = launch_member(b, w, it, 0, st);
+        if (e != cudaSuccess) return e;
     }
     const int lane_tiles = (b.n_gl + kTileM - 1) / kTileM;
     if (lane_tiles >= 2) {
