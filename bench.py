@@ -226,7 +226,7 @@ def run_ours(args, rank, world, dev):
 
     # decode-only throughput and union bytes of the decode
     dec_ms = sum(v[1] for k, v in prof.items()
-                 if k in ("k_union", "k_score", "k_score_tc", "k_select", "k_attn", "k_attn_tc", "k_combine")) / args.steps
+                 if k in ("k_union", "k_member", "k_score", "k_score_tc", "k_select", "k_attn", "k_attn_tc", "k_combine")) / args.steps
     union_bytes = sum(st.union_nodes) * st.node_bytes + st.union_tokens * 4 * g.d
     stages = {k: round(v[1] / args.steps, 4) for k, v in sorted(prof.items())}
     res = {

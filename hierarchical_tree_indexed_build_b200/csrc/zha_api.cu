@@ -369,7 +369,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         int64_t W = 1;
         for (auto* t : dec->trees)
             if (l <= t->g.L) W = std::max<int64_t>(W, (t->cap[l] + 31) / 32);
-        w.W[l] = W;
+        w.W[l] = (W + 7) / 8 * 8;   // rows of whole 32-byte segments (vector reads of 256-node spans)
     }
     for (auto* t : dec->trees) {
         cap1 = std::max<int64_t>(cap1, t->cap[1]);
@@ -384,7 +384,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.mwords = (max_queries * dec->G + 255) / 256 * 8;
     w.lanes_cap = dec->lanes_cap;
     w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
-    w.us = cap1;
+    w.us = (cap1 + 7) / 8 * 8 + 8;   // union lists: room for 16-byte-rounded bulk reads past the end
     w.s_cap = s_cap;
 
     size_t off = 0;

@@ -474,9 +474,9 @@ size_t attn_tc_smem(int d) {
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
     if (max_splits <= 0) return cudaSuccess;
-    ProfScope ps_("k_attn_tc", st);
     cudaError_t e = launch_member(b, w, 0, 1, st);   // lane masks of the kept level-1 chunks
     if (e != cudaSuccess) return e;
+    ProfScope ps_("k_attn_tc", st);
     const int lane_tiles = (b.n_gl + kRows - 1) / kRows;
     dim3 grid((unsigned)max_splits, lane_tiles, b.n_groups);
     const size_t smem = attn_tc_smem(b.d);

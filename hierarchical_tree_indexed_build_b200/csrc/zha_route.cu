@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
                 const int64_t pj = j / C;
                 mb = (__ldg(Pb + (pj >> 5)) >> (pj & 31)) & 1u;
             }
-            ex[j] = mb ? best : -INFINITY;
+            ex[k] = mb ? best : -INFINITY;   // candidate order
             if (mb) {
                 fmax = fmaxf(fmax, best);
                 ++fcnt;
@@ -293,7 +293,13 @@ constexpr int kSelThreads = 512;
 constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
-constexpr int kUn = 2;               // 128-candidate blocks per warp in flight
+constexpr int kUn = 2;               // 128-candidate blocks per warp in flight (gather path)
+constexpr int kPD = 6;               // per-thread prefetch ring depth (cp.async)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 // masses are fixed point with 2^39 for exp(0); sums of <= 2^24 candidates stay below 2^63
 
 // Ascending key order == (e descending, node index ascending).
@@ -331,15 +337,22 @@ struct SelMath {
 };
 
 // One block per lane.  The scorer left, for every candidate of the lane's group (the
-// children of the group's union of kept nodes, or all top nodes), the plane estimate if
-// the candidate is on this lane's frontier and -inf otherwise, plus the lane's frontier
-// maximum M and size F.  Two passes over the candidates: a histogram of fixed-point masses
+// children of the group's union of kept nodes, or all top nodes) in candidate order, the
+// plane estimate if the candidate is on this lane's frontier and -inf otherwise, plus the
+// lane's frontier maximum M and size F.  Two passes over the candidates: a histogram of fixed-point masses
 // over bins of M - e, then the kept bits of the bins above the boundary bin and the
 // boundary bin's candidates, which are sorted by (e desc, j asc) to finish the prefix.
 __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int it) {
     extern __shared__ unsigned long long sel_smem[];
-    unsigned long long* hist = sel_smem;   // [kNB]
-    unsigned long long* keys = hist + kNB; // [kCap]
+    // bin masses as two 32-bit words (shared-memory 64-bit atomics are several times slower):
+    // hlo accumulates the low words, hhi the high words and every wrap of hlo, so a bin's
+    // exact 64-bit mass is hhi 2^32 + hlo
+    uint32_t* hlo = reinterpret_cast<uint32_t*>(sel_smem);   // [kNB]
+    uint32_t* hhi = hlo + kNB;                                // [kNB]
+    unsigned long long* keys = sel_smem + kNB;                // [kCap]
+    float4* pref = reinterpret_cast<float4*>(keys + kCap);   // [threads][kPD] prefetched scores
+    int32_t* prefj = reinterpret_cast<int32_t*>(pref + (size_t)kSelThreads * kPD);   // [threads][kPD] union entries
+    auto hist = [&](int i) -> unsigned long long { return ((unsigned long long)hhi[i] << 32) | hlo[i]; };
     __shared__ unsigned long long red_u[33];
     __shared__ int red_i[33];
     __shared__ int s_bstar;
@@ -368,7 +381,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     const bool top = (lev == sq.L);
     const int C = sq.C;
     // candidate and node indices are < 2^24 (level-1 nodes are capped there): 32-bit math
-    const int nc = (int)(top ? sq.T : (int64_t)w.ucount[grp] * C);
+    const int nu = top ? 0 : w.ucount[grp];
+    const int nc = top ? (int)sq.T : nu * C;
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     // candidates 4k..4k+3 are 4 consecutive, 4-aligned nodes
     const bool contig = top || (C % 4 == 0);
@@ -385,42 +399,82 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         const uint32_t pk = (uint32_t)k / (uint32_t)C;
         return __ldg(ul + pk) * C + (k - (int)pk * C);
     };
-    // scores of candidates k0..k0+3 (k0 = 128 bk + 4 lane); -inf past the end
-    auto load = [&](int bk, float4& ev, int& j0) {
+    // scores of candidates k0..k0+3 (k0 = 128 bk + 4 lane), stored in candidate order by the
+    // scorer; -inf past the end.  With need_j, also the node index of candidate k0 (of the
+    // 4 consecutive nodes when contig), loaded independently of the scores.
+    auto load = [&](int bk, float4& ev, int& j0, bool need_j) {
         const int k0 = bk * 128 + 4 * lane;
-        ev = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        j0 = -1;
-        if (contig) {
-            // predicated, not branched: lanes past the end read node 0 and mask it
-            const bool in = k0 < nc;
-            const int jj = cand_j(in ? k0 : 0);
-            const float4 x = *reinterpret_cast<const float4*>(e + jj);   // rows are padded to 128 floats
-            j0 = in ? jj : -1;
-            ev.x = in ? x.x : -INFINITY;
-            ev.y = k0 + 1 < nc ? x.y : -INFINITY;
-            ev.z = k0 + 2 < nc ? x.z : -INFINITY;
-            ev.w = k0 + 3 < nc ? x.w : -INFINITY;
-            return;
-        }
-        if (k0 >= nc) return;
-        j0 = cand_j(k0);
-        {
-            ev.x = e[j0];
-            if (k0 + 1 < nc) ev.y = e[cand_j(k0 + 1)];
-            if (k0 + 2 < nc) ev.z = e[cand_j(k0 + 2)];
-            if (k0 + 3 < nc) ev.w = e[cand_j(k0 + 3)];
-        }
+        const bool in = k0 < nc;
+        const float4 xv = *reinterpret_cast<const float4*>(e + (in ? k0 : 0));   // rows padded to 128
+        j0 = (need_j && in) ? cand_j(k0) : -1;
+        ev.x = in ? xv.x : -INFINITY;
+        ev.y = k0 + 1 < nc ? xv.y : -INFINITY;
+        ev.z = k0 + 2 < nc ? xv.z : -INFINITY;
+        ev.w = k0 + 3 < nc ? xv.w : -INFINITY;
     };
     auto jof = [&](int bk, int j0, int c) -> int {
         return contig ? j0 + c : cand_j(bk * 128 + 4 * lane + c);
     };
     // every warp visits its blocks with kUn loads in flight; body(bk, scores[4], j0)
-    auto for_cands = [&](auto&& body) {
+    // Contiguous layouts: every thread prefetches its own float4 of scores (and, when node
+    // ids are needed, its union-list entry) kPD - 1 iterations ahead with cp.async into a
+    // private shared-memory ring; it reads back only what it copied, so no barrier is needed.
+    auto stream = [&](bool need_j, auto&& body) {
+        float4* my = pref + (size_t)threadIdx.x * kPD;
+        int32_t* myj = prefj + (size_t)threadIdx.x * kPD;
+        const int niter = warp < nblk ? (nblk - warp + nwarps - 1) / nwarps : 0;   // uniform in a warp
+        const bool want_u = need_j && !top;
+        auto issue = [&](int t) {
+            const int k0 = (warp + t * nwarps) * 128 + 4 * lane;
+            const bool in = t < niter && k0 < nc;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(my + t % kPD)),
+                         "l"(e + (in ? k0 : 0)), "r"(in ? 16u : 0u)
+                         : "memory");
+            if (want_u) {
+                const int uk = in ? (cs >= 0 ? (k0 >> cs) : k0 / C) : 0;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(myj + t % kPD)),
+                             "l"(ul + uk), "r"(in ? 4u : 0u)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+#pragma unroll
+        for (int t = 0; t < kPD - 1; ++t) issue(t);
+        for (int t = 0; t < niter; ++t) {
+            issue(t + kPD - 1);
+            asm volatile("cp.async.wait_group %0;" ::"n"(kPD - 1) : "memory");
+            const int bk = warp + t * nwarps;
+            const int k0 = bk * 128 + 4 * lane;
+            const float4 xv = my[t % kPD];
+            float4 ev;
+            ev.x = k0 < nc ? xv.x : -INFINITY;
+            ev.y = k0 + 1 < nc ? xv.y : -INFINITY;
+            ev.z = k0 + 2 < nc ? xv.z : -INFINITY;
+            ev.w = k0 + 3 < nc ? xv.w : -INFINITY;
+            int j0 = -1;
+            if (need_j && k0 < nc) {
+                if (top) {
+                    j0 = k0;
+                } else {
+                    const int pj = myj[t % kPD];
+                    const int uk = cs >= 0 ? (k0 >> cs) : k0 / C;
+                    j0 = cs >= 0 ? (pj << cs) + (k0 & (C - 1)) : pj * C + (k0 - uk * C);
+                }
+            }
+            body(bk, ev, j0);
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+    };
+    auto for_cands = [&](bool need_j, auto&& body) {
+        if (contig) {
+            stream(need_j, body);
+            return;
+        }
         for (int b0 = warp; b0 < nblk; b0 += kUn * nwarps) {
             float4 ev[kUn];
             int j0[kUn];
 #pragma unroll
-            for (int u = 0; u < kUn; ++u) load(b0 + u * nwarps, ev[u], j0[u]);
+            for (int u = 0; u < kUn; ++u) load(b0 + u * nwarps, ev[u], j0[u], need_j);
 #pragma unroll
             for (int u = 0; u < kUn; ++u) {
                 const int bk = b0 + u * nwarps;
@@ -457,10 +511,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     unsigned long long need = 0;   // mass still needed from the boundary bin
     if (b.p < 1.0f) {
         // pass 1: fixed-point masses into bins of (M - e)
-        for (int i = threadIdx.x; i < kNB; i += blockDim.x) hist[i] = 0ull;
+        for (int i = threadIdx.x; i < kNB; i += blockDim.x) {
+            hlo[i] = 0u;
+            hhi[i] = 0u;
+        }
         if (threadIdx.x == 0) s_nkeys = 0;
         __syncthreads();
-        for_cands([&](int bk, const float4 ev4, int j0) {
+        for_cands(false, [&](int bk, const float4 ev4, int j0) {
             const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
             // -inf (off the frontier) gives mass 0 and the last bin: computed without branches,
             // only the atomic is predicated
@@ -468,12 +525,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             for (int c = 0; c < 4; ++c) {
                 const unsigned long long ms = sm.mass(v[c]);
                 const int bn = sm.bin(v[c]);
-                if (ms) atomicAdd(&hist[bn], ms);
+                if (ms) {
+                    const uint32_t lo = (uint32_t)ms, hi = (uint32_t)(ms >> 32);
+                    const uint32_t old = atomicAdd(&hlo[bn], lo);
+                    const uint32_t carry = old + lo < old ? 1u : 0u;
+                    if (hi + carry) atomicAdd(&hhi[bn], hi + carry);
+                }
             }
         });
         __syncthreads();
         unsigned long long zloc = 0;
-        for (int i = threadIdx.x; i < kNB; i += blockDim.x) zloc += hist[i];
+        for (int i = threadIdx.x; i < kNB; i += blockDim.x) zloc += hist(i);
         const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
         unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
         if (target < 1ull) target = 1ull;
@@ -483,7 +545,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             constexpr int per = kNB / 32;
             unsigned long long ls = 0;
 #pragma unroll 4
-            for (int k = 0; k < per; ++k) ls += hist[lane * per + k];
+            for (int k = 0; k < per; ++k) ls += hist(lane * per + k);
             unsigned long long incl = ls;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -499,11 +561,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
 #pragma unroll 1
                 for (int k = 0; k < per; ++k) {
                     const int bb = lane * per + k;
-                    if (cum + hist[bb] >= target) {
+                    if (cum + hist(bb) >= target) {
                         bs = bb;
                         break;
                     }
-                    cum += hist[bb];
+                    cum += hist(bb);
                 }
                 s_bstar = bs;
                 s_cumb = cum;
@@ -516,7 +578,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
 
     // pass 2: kept bits of the bins above the boundary; boundary-bin candidates collected
     unsigned long long cnt = 0;
-    for_cands([&](int bk, const float4 ev4, int j0) {
+    for_cands(true, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
         uint32_t nib = 0, col = 0;
 #pragma unroll
@@ -605,7 +667,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     } else {
         // rare: too many candidates in one bin - bisection on the exact key order, then a pass
         unsigned long long klo = ~0ull, khi = 0ull;
-        for_cands([&](int bk, const float4 ev4, int j0) {
+        for_cands(true, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -621,7 +683,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         while (lo < hi && iters < 70) {
             const unsigned long long mid = lo + (hi - lo) / 2;
             unsigned long long acc = 0;
-            for_cands([&](int bk, const float4 ev4, int j0) {
+            for_cands(true, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
@@ -635,7 +697,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         }
         if (threadIdx.x == 0 && iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
         unsigned long long extra = 0;
-        for_cands([&](int bk, const float4 ev4, int j0) {
+        for_cands(true, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -689,7 +751,7 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
 }
 
 cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st) {
-    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8;
+    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8 + (size_t)kSelThreads * kPD * (16 + 4);
     cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     ProfScope ps_("k_select", st);
     k_select<<<b.n_lanes, kSelThreads, smem, st>>>(b, w, it);

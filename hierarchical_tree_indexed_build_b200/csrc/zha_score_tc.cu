@@ -146,50 +146,95 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // Lanes' kept bits of one level, transposed over the group's union list of that level:
 // memb[grp][u][w] bit t = lane 32 w + t kept union node u.  Mode 0: the level above the one
 // routing iteration `it` scores (its nodes are the candidates' parents); mode 1: level 1
-// (the chunks attention gathers).  Grid (chunks, lane words, groups); a warp covers 32 nodes.
+// (the chunks attention gathers).  A block transposes a tile of 256 union entries x 256
+// lanes (8 lane words): where the tile's entries are 256 consecutive nodes (a dense stretch
+// of the union), each lane reads the 9 bitmap words covering them and realigns them by
+// funnel shifts, warps transpose 32 x 32 bit blocks with ballots through shared memory, and
+// each entry's 8 words are written as one 32-byte segment; other tiles go entry by entry.
+// Grid (tiles, lane-word groups of 8, groups), 256 threads.
 __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mode) {
+    __shared__ uint32_t T[256][9];                    // [lane][node word], padded
+    __shared__ __align__(16) uint32_t O[256][8];      // [entry][lane word]
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
     const SeqDev& sq = b.seqs[s];
     int pl;
     if (mode == 0) {
         const int lev = sq.L - it;
-        if (lev < 1 || lev == sq.L) return;       // top level: no parents
+        if (lev < 1 || lev == sq.L) return;           // top level: no parents
         pl = lev + 1;
     } else {
-        if (sq.T == 0) return;                    // dense attention: no union
+        if (sq.T == 0) return;                        // dense attention: no union
         pl = 1;
     }
     const int nu = w.ucount[grp];
-    const int lw = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int y = lw * 32 + lane;
-    const bool ok = y < b.n_gl;
-    const uint32_t* kb = w.kept[pl] + lane_of(b, s, g, ok ? y : 0) * w.W[pl];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lw0 = blockIdx.y * 8;
+    const int y = lw0 * 32 + tid;                     // this thread's lane (load phase)
+    const bool yok = y < b.n_gl;
+    const uint32_t* kb = w.kept[pl] + lane_of(b, s, g, yok ? y : 0) * w.W[pl];
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
-    uint32_t* out = w.memb + (int64_t)grp * w.ms * w.mwords + lw;
-    for (int c = blockIdx.x * 8 + warp; c * 32 < nu; c += gridDim.x * 8) {
-        const int u0 = c * 32, n = min(32, nu - u0);
-        const int pmy = lane < n ? __ldg(ul + u0 + lane) : -1;
-        const int p0 = __shfl_sync(0xffffffffu, pmy, 0);
-        const int pn = __shfl_sync(0xffffffffu, pmy, n - 1);
-        uint32_t mine = 0;
-        if (n == 32 && (p0 & 31) == 0 && pn == p0 + 31) {
-            // 32 consecutive parents: one bitmap word per lane, transposed by ballots
-            const uint32_t word = ok ? __ldg(kb + (p0 >> 5)) : 0u;
+    uint32_t* out = w.memb + (int64_t)grp * w.ms * w.mwords + lw0;
+    for (int tx = blockIdx.x; tx * 256 < nu; tx += gridDim.x) {
+        const int u0 = tx * 256, cnt = min(256, nu - u0);
+        const int p0 = __ldg(ul + u0), pn = __ldg(ul + u0 + cnt - 1);
+        const bool dense = cnt == 256 && pn == p0 + 255;   // 256 consecutive nodes; uniform in the block
+        if (dense) {
+            // the lane's 256 bits for nodes p0 .. p0 + 255: 9 words realigned by funnel shifts
+            const int w0 = p0 >> 5, sh = p0 & 31;
+            const int64_t W = w.W[pl];
+            uint32_t wv[9];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const uint32_t r = __ballot_sync(0xffffffffu, (word >> t) & 1u);
-                if (lane == t) mine = r;
+            for (int k = 0; k < 9; ++k) wv[k] = (yok && w0 + k < W) ? __ldg(kb + w0 + k) : 0u;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) T[tid][k] = __funnelshift_r(wv[k], wv[k + 1], sh);
+            __syncthreads();
+            // warp i: node word i of the tile, for each of the 8 lane words
+#pragma unroll 1
+            for (int lw = 0; lw < 8; ++lw) {
+                const uint32_t v = T[lw * 32 + lane][warp];
+                uint32_t mine = 0;
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const uint32_t r = __ballot_sync(0xffffffffu, (v >> t) & 1u);
+                    if (lane == t) mine = r;
+                }
+                O[warp * 32 + lane][lw] = mine;
             }
+            __syncthreads();
+            uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(u0 + tid) * w.mwords);
+            dst[0] = make_uint4(O[tid][0], O[tid][1], O[tid][2], O[tid][3]);
+            dst[1] = make_uint4(O[tid][4], O[tid][5], O[tid][6], O[tid][7]);
+            __syncthreads();                          // T and O are reused by the next tile
         } else {
-            for (int t = 0; t < n; ++t) {
-                const int pt = __shfl_sync(0xffffffffu, pmy, t);
-                const uint32_t bit = ok ? (__ldg(kb + (pt >> 5)) >> (pt & 31)) & 1u : 0u;
-                const uint32_t r = __ballot_sync(0xffffffffu, bit);
-                if (lane == t) mine = r;
+            // warp i: entries u0 + 32 i .., lane words lw0 .. lw0 + 7
+            const int e0 = u0 + warp * 32;
+            const int n = min(32, nu - e0);
+            if (n > 0) {
+                const int pmy = lane < n ? __ldg(ul + e0 + lane) : 0;
+#pragma unroll 1
+                for (int lw = 0; lw < 8; ++lw) {
+                    const int yl = (lw0 + lw) * 32 + lane;
+                    if ((lw0 + lw) * 32 >= b.n_gl) break;             // uniform in the warp
+                    const bool ok = yl < b.n_gl;
+                    const uint32_t* kl = w.kept[pl] + lane_of(b, s, g, ok ? yl : 0) * w.W[pl];
+                    // all 32 entries' bits of this lane first (independent loads), then ballots
+                    uint32_t bits = 0;
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) {
+                        const int pt = __shfl_sync(0xffffffffu, pmy, t);
+                        if (t < n && ok) bits |= ((__ldg(kl + (pt >> 5)) >> (pt & 31)) & 1u) << t;
+                    }
+                    uint32_t mine = 0;
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) {
+                        const uint32_t r = __ballot_sync(0xffffffffu, (bits >> t) & 1u);
+                        if (lane == t) mine = r;
+                    }
+                    if (lane < n) out[(int64_t)(e0 + lane) * w.mwords + lw] = mine;
+                }
             }
         }
-        if (lane < n) out[(int64_t)(u0 + lane) * w.mwords] = mine;
     }
 }
 
@@ -448,6 +493,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
         float* ex = w.e + x * w.es;
         float fmax = -INFINITY;
         int fcnt = 0;
+#pragma unroll 1
         for (int i = 0; i < nt; ++i) {
             const int st = i % kStages, q = i * LT + lt, slot = q & 1;
             if (!mbar_wait(smem_u32(&bar_acc_full[slot]), (uint32_t)((q >> 1) & 1))) {
@@ -501,18 +547,11 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                 }
             }
             if (ok) {
+                // candidate order: tile i holds candidates k0 .. k0 + 7 (rows padded past nc)
+                float4* dst = reinterpret_cast<float4*>(ex + (blockIdx.x + i * gridDim.x) * kNodes);
 #pragma unroll
-                for (int q4 = 0; q4 < kNodes / 4; ++q4) {
-                    const int j0 = jv[4 * q4], j3 = jv[4 * q4 + 3];
-                    if (j0 >= 0 && (j0 & 3) == 0 && j3 == j0 + 3) {
-                        *reinterpret_cast<float4*>(ex + j0) =
-                            make_float4(best[4 * q4], best[4 * q4 + 1], best[4 * q4 + 2], best[4 * q4 + 3]);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            if (jv[4 * q4 + c] >= 0) ex[jv[4 * q4 + c]] = best[4 * q4 + c];
-                    }
-                }
+                for (int q4 = 0; q4 < kNodes / 4; ++q4)
+                    dst[q4] = make_float4(best[4 * q4], best[4 * q4 + 1], best[4 * q4 + 2], best[4 * q4 + 3]);
             }
         }
         if (ok && fcnt > 0) {
@@ -548,20 +587,22 @@ size_t score_tc_smem_lt(int d, int lt) {
 size_t score_tc_smem(int d) { return score_tc_smem_lt(d, 2); }
 
 cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaStream_t st) {
-    const int lw = (b.n_gl + 31) / 32;
-    int nbm = (int)((w.ms + 255) / 256);
-    nbm = nbm < 1 ? 1 : (nbm > 148 ? 148 : nbm);
-    k_member<<<dim3(nbm, lw, b.n_groups), 256, 0, st>>>(b, w, it, mode);
+    ProfScope ps_("k_member", st);
+    const int lwg = (b.n_gl + 255) / 256;             // groups of 8 lane words
+    int nbx = (int)((w.ms + 255) / 256);
+    const int cap = (148 * 8) / max(1, lwg * b.n_groups);
+    nbx = nbx < 1 ? 1 : (nbx > cap ? (cap < 1 ? 1 : cap) : nbx);
+    k_member<<<dim3(nbx, lwg, b.n_groups), 256, 0, st>>>(b, w, it, mode);
     return cudaGetLastError();
 }
 
 cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
-    ProfScope ps_("k_score_tc", st);
     if (it > 0) {
         // membership words of the group's union parents (the level above the scored one)
         const cudaError_t e = launch_member(b, w, it, 0, st);
         if (e != cudaSuccess) return e;
     }
+    ProfScope ps_("k_score_tc", st);
     const int lane_tiles = (b.n_gl + kTileM - 1) / kTileM;
     if (lane_tiles >= 2) {
         const int pairs = (lane_tiles + 1) / 2;
