@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: union index, -1 all, -2 none
     uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_slot0 + 2 * kPos);   // [2][kPos] slot of each position
     uint32_t* s_valid0 = reinterpret_cast<uint32_t*>(s_pslot0 + 2 * kPos); // [2][kPos/32] positions with a token
-    uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][kPos][4] lane masks per slot
+    uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][4][kPos] lane masks: [lane word][slot]
     float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [2][kRows] tile max per half
     float* s_xsum = s_xmax + 2 * kRows;                                     // [2][kRows] row sums per half
     __shared__ __align__(8) uint64_t mbar;
@@ -250,9 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 // lane masks land asynchronously with the tile's K/V gather (same commit
                 // group, waited at the top of the tile that uses them); zero-filled if none
                 const uint32_t* src = memb + (int64_t)(code >= 0 ? code : 0) * w.mwords;
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(s_mw0 + (st * kPos + slot) * 4)),
-                             "l"(src), "r"(code >= 0 ? 16u : 0u)
-                             : "memory");
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                                     su32(s_mw0 + (st * 4 + q) * kPos + slot)),
+                                 "l"(src + q), "r"(code >= 0 ? 4u : 0u)
+                                 : "memory");
             }
             const unsigned vb = __ballot_sync(0xffffffffu, tok >= 0);
             if (lane == 0) s_valid0[st * (kPos / 32) + warp] = vb;
@@ -300,23 +303,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         }
         __syncwarp();
 
-        // This row's membership on its half of the tile, slot by slot from the staged lane
-        // masks: a slot covers a run of consecutive positions.
+        // This row's membership on its half of the tile from the staged lane masks.  When C
+        // divides 16 (tiles start on multiples of 128 positions) the half holds 64/C whole
+        // slots, a multiple of 4: gather their bits (vector loads of the lane word's slot row)
+        // and spread each over its C positions; otherwise walk the slots.
         uint64_t mem = 0;
         {
-            const uint8_t* ps = s_pslot0 + st * kPos;
             const int hs = half * kHalf;
-            const int k0 = ps[hs], k1 = ps[hs + kHalf - 1];
             const int lw = row >> 5, bit = row & 31;
-            // slot k spans positions [k C - o0, (k+1) C - o0) of the tile, o0 = p0 mod C
-            const int o0 = (int)(p0 % C);
-            for (int k = k0; k <= k1; ++k) {
-                const int32_t code = s_slot0[st * kPos + k];
-                const bool in = code == -1 || (code >= 0 && ((s_mw0[(st * kPos + k) * 4 + lw] >> bit) & 1u));
-                if (in) {
-                    const int a = max(k * (int)C - o0, hs) - hs, e = min((k + 1) * (int)C - o0, hs + kHalf) - hs;
-                    const uint64_t hi_mask = e >= 64 ? ~0ull : ((1ull << e) - 1ull);
-                    mem |= hi_mask & ~((1ull << a) - 1ull);
+            const uint32_t* mrow = s_mw0 + (st * 4 + lw) * kPos;
+            const int32_t* codes = s_slot0 + st * kPos;
+            if (C <= 16 && 64 % C == 0) {              // slot rows read as 16-byte vectors
+                const int ns_ = 64 / (int)C, k0 = hs / (int)C;
+                uint64_t sb = 0;                       // bit k: slot k0 + k holds the row
+                for (int k = 0; k < ns_; k += 4) {
+                    const uint4 mv = *reinterpret_cast<const uint4*>(mrow + k0 + k);
+                    const int4 cv = *reinterpret_cast<const int4*>(codes + k0 + k);
+                    const uint32_t m4[4] = {mv.x, mv.y, mv.z, mv.w};
+                    const int c4[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const bool in = c4[q] == -1 || (c4[q] >= 0 && ((m4[q] >> bit) & 1u));
+                        sb |= (uint64_t)(in ? 1u : 0u) << (k + q);
+                    }
+                }
+                const uint64_t ones = (1ull << C) - 1ull;
+                for (int k = 0; k < ns_; ++k)
+                    if ((sb >> k) & 1ull) mem |= ones << (k * (int)C);
+            } else {
+                const uint8_t* ps = s_pslot0 + st * kPos;
+                const int k0 = ps[hs], k1 = ps[hs + kHalf - 1];
+                // slot k spans positions [k C - o0, (k+1) C - o0) of the tile, o0 = p0 mod C
+                const int o0 = (int)(p0 % C);
+                for (int k = k0; k <= k1; ++k) {
+                    const int32_t code = codes[k];
+                    const bool in = code == -1 || (code >= 0 && ((mrow[k] >> bit) & 1u));
+                    if (in) {
+                        const int a = max(k * (int)C - o0, hs) - hs, e = min((k + 1) * (int)C - o0, hs + kHalf) - hs;
+                        const uint64_t hi_mask = e >= 64 ? ~0ull : ((1ull << e) - 1ull);
+                        mem |= hi_mask & ~((1ull << a) - 1ull);
+                    }
                 }
             }
             const uint32_t* vw = s_valid0 + st * (kPos / 32) + half * 2;
@@ -337,9 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         for (int c = 0; c < kHalf / 16; ++c) {
             float v[16];
             tld16(tS + lane_t + half * kHalf + c * 16, v);
+            const uint32_t m16 = (uint32_t)(mem >> (c * 16));
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                if ((mem >> (c * 16 + i)) & 1ull) tmax = fmaxf(tmax, v[i]);
+                if ((m16 >> i) & 1u) tmax = fmaxf(tmax, v[i]);
         }
         s_xmax[half * kRows + row] = tmax;
         __syncthreads();                       // partner maxima visible; next tile's tokens visible
@@ -374,13 +401,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         for (int c = 0; c < kHalf / 16; ++c) {
             float v[16];
             tld16(tS + lane_t + half * kHalf + c * 16, v);
+            const uint32_t m16 = (uint32_t)(mem >> (c * 16));
             uint32_t hi[8], lo[8];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
                 const float e0 = ex2_approx(fmaf(sl, v[i], -ml));
                 const float e1 = ex2_approx(fmaf(sl, v[i + 1], -ml));
-                const float p0v = ((mem >> (c * 16 + i)) & 1ull) ? e0 : 0.0f;
-                const float p1v = ((mem >> (c * 16 + i + 1)) & 1ull) ? e1 : 0.0f;
+                const float p0v = ((m16 >> i) & 1u) ? e0 : 0.0f;
+                const float p1v = ((m16 >> (i + 1)) & 1u) ? e1 : 0.0f;
                 lsum += p0v;
                 lsum += p1v;
                 // bf16 hi = p rounded to 8 significant bits (integer add on the bits), lo =
