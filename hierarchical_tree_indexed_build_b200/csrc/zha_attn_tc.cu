@@ -278,30 +278,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
+    // S = Q K^T of the tile whose keys sit in sK (issued by thread 0)
+    auto issue_s = [&]() {
+        const uint32_t q0 = su32(sQ), k0 = su32(sK);
+#pragma unroll
+        for (int kb = 0; kb < KBD; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t off = kb * kBlock + kk * 32;
+                mma_bf16(tS, desc_sw128(q0 + off, 16, 1024), desc_sw128(k0 + off, 16, 1024), idesc_bf16(kPos, 0),
+                         (kb | kk) ? 1u : 0u);
+            }
+    };
+
+    // Pipeline: tile i's S was issued (with tile i-1's P V) at the end of the previous
+    // iteration; its K/V were gathered during tile i-1's softmax.  One commit per tile.
     resolve(0, 0);
     __syncthreads();
     issue_kv(0);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+        issue_s();
+        commit(su32(&mbar));
+    }
+    __syncwarp();
     int st = 0;
     for (int64_t p0 = 0; p0 < npos; p0 += kPos, st ^= 1) {
         const bool more = p0 + kPos < npos;
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0) {
-            const uint32_t q0 = su32(sQ), k0 = su32(sK);
-#pragma unroll
-            for (int kb = 0; kb < KBD; ++kb)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t off = kb * kBlock + kk * 32;
-                    mma_bf16(tS, desc_sw128(q0 + off, 16, 1024), desc_sw128(k0 + off, 16, 1024),
-                             idesc_bf16(kPos, 0), (kb | kk) ? 1u : 0u);
-                }
-            commit(su32(&mbar));
-        }
-        __syncwarp();
 
         // This row's membership on its half of the tile from the staged lane masks.  When C
         // divides 16 (tiles start on multiples of 128 positions) the half holds 64/C whole
@@ -428,6 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             *reinterpret_cast<uint4*>(sPl + kmaj(row, c16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             *reinterpret_cast<uint4*>(sPl + kmaj(row, c16 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
         }
+        // the next tile's K/V (gathered during this softmax) and lane masks must have landed
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
@@ -446,17 +453,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                              idesc_bf16(D, 1), (first_pv && pass == 0 && ks == 0) ? 0u : 1u);
                 }
             }
-            // no commit: the next tile's S commit tracks these MMAs too (a commit covers every
-            // earlier tcgen05 operation of the issuing thread), so P V overlaps the next
-            // tile's gather wait, slot table and membership
+            // S of the next tile reads only sQ / sK and writes the S columns, whose values
+            // this tile no longer needs; one commit covers both
+            if (more && !abort_sh) issue_s();
+            commit(su32(&mbar));
         }
         __syncwarp();
         first_pv = false;
         if (abort_sh) break;
     }
-    // the last P V: one more commit, then O is final
-    if (tid == 0) commit(su32(&mbar));
-    __syncwarp();
+    // the commit of the last tile (its P V): wait once more, then O is final
     if (!wait_phase(su32(&mbar), phase) && lane == 0) {
         atomicOr(w.status, kStatusTimeout);
         abort_sh = 1;
