@@ -57,6 +57,30 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+# Kernel -> source file whose contents its DRAM-traffic record was taken against.
+KERNEL_SOURCES = {
+    "k_score_tc": "zha_score_tc.cu", "k_attn_tc": "zha_attn_tc.cu", "k_select": "zha_route.cu",
+    "k_score": "zha_route.cu", "k_attn": "zha_attn.cu", "k_build_stream": "zha_build.cu",
+}
+
+
+def measured_traffic(name, workload):
+    """DRAM bytes (read + write) per launch of `name` from profiles/traffic.txt, written from
+    an ncu capture of this workload (JSON text); None when absent or when the kernel's source has changed
+    since (the record stores the source's SHA-256)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
+            rec = json.load(f)[workload][name]
+        src = os.path.join(ROOT, "hierarchical_tree_indexed_build_b200", "csrc", KERNEL_SOURCES[name])
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return float(rec["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def tensor_peak(dtype):
     """Dense tensor peak for the kernel's MMA dtype: the measured bf16 burst figure (fp16
     runs at the bf16 rate, tf32 at half of it)."""
@@ -219,6 +243,7 @@ def run_ours(args, rank, world, dev):
         ach = nbytes / (avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
                 "traffic": None, "kernel": name, "peak_source": peak_src}
+    roof["traffic"] = measured_traffic(name, wl.name)
     roof["algorithmic_bytes_per_launch"] = nbytes
     roof["algorithmic_flops_per_launch"] = nflops
     roof["avg_launch_ms"] = avg_ms
