@@ -31,7 +31,8 @@ namespace {
 
 constexpr int kRows = 128;      // lanes per tile (MMA M)
 constexpr int kPos = 128;       // token positions per tile (MMA N of QK^T, K of PV)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;   // 16 warps: 4 per TMEM lane quarter, each a quarter of the positions
+constexpr int kParts = kThreads / 128;
 constexpr float kLazy = 8.0f;   // raise the running max only when exceeded by this much
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
 constexpr int kBlock = kRows * 128;   // bytes of one 128-byte-wide block of 128 rows
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     constexpr int KBD = D / 64;                 // 128-byte blocks along d (bf16)
     constexpr int PR = D + 4;
     constexpr int TCOLS = 256;                  // S: columns [0,128), O: [128, 128+D)
-    constexpr int kHalf = kPos / 2;             // positions per warp of a row pair
+    constexpr int kPart = kPos / kParts;        // positions per warp of a row (32)
     constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -145,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_slot0 + 2 * kPos);   // [2][kPos] slot of each position
     uint32_t* s_valid0 = reinterpret_cast<uint32_t*>(s_pslot0 + 2 * kPos); // [2][kPos/32] positions with a token
     uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][4][kPos] lane masks: [lane word][slot]
-    float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [2][kRows] tile max per half
-    float* s_xsum = s_xmax + 2 * kRows;                                     // [2][kRows] row sums per half
+    float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [kParts][kRows] tile max per part
+    float* s_xsum = s_xmax + kParts * kRows;                                // [kParts][kRows] row sums per part
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_sh;
     __shared__ int abort_flag;
@@ -193,15 +194,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const uint32_t tmem = tmem_sh;
     const uint32_t tS = tmem, tO = tmem + 128;
 
-    // Row (lane) state.  Warps w and w+4 read the same TMEM lanes 32(w%4).. and share the
-    // row; `half` selects positions [64 half, 64 half + 64) and O columns [D/2 half, ...).
-    const int half = warp >> 2;
+    // Row (lane) state.  Warps w, w+4, w+8, w+12 read the same TMEM lanes 32(w%4).. and share
+    // the row; `part` selects positions [32 part, 32 part + 32) and O columns [D/4 part, ...).
+    const int part = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const int y = y0 + row;
     const bool y_ok = y < b.n_gl;
     const int64_t x = lane_of(b, s, g, y_ok ? y : 0);
     const uint32_t lane_t = (uint32_t)((warp & 3) * 32) << 16;
-    float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in both warps of a row
+    float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in the 4 warps of a row
 
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     const __nv_bfloat16* Kg = sq.K + (int64_t)g * sq.ld * D;
@@ -308,19 +309,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     for (int64_t p0 = 0; p0 < npos; p0 += kPos, st ^= 1) {
         const bool more = p0 + kPos < npos;
 
-        // This row's membership on its half of the tile from the staged lane masks.  When C
-        // divides 16 (tiles start on multiples of 128 positions) the half holds 64/C whole
+        // This row's membership on its part of the tile from the staged lane masks.  When C
+        // divides 8 (tiles start on multiples of 128 positions) the part holds 32/C whole
         // slots, a multiple of 4: gather their bits (vector loads of the lane word's slot row)
         // and spread each over its C positions; otherwise walk the slots.
-        uint64_t mem = 0;
+        uint32_t mem = 0;
         {
-            const int hs = half * kHalf;
+            const int hs = part * kPart;
             const int lw = row >> 5, bit = row & 31;
             const uint32_t* mrow = s_mw0 + (st * 4 + lw) * kPos;
             const int32_t* codes = s_slot0 + st * kPos;
-            if (C <= 16 && 64 % C == 0) {              // slot rows read as 16-byte vectors
-                const int ns_ = 64 / (int)C, k0 = hs / (int)C;
-                uint64_t sb = 0;                       // bit k: slot k0 + k holds the row
+            if (C <= 8 && 32 % C == 0) {               // slot rows read as 16-byte vectors
+                const int ns_ = 32 / (int)C, k0 = hs / (int)C;
+                uint32_t sb = 0;                       // bit k: slot k0 + k holds the row
                 for (int k = 0; k < ns_; k += 4) {
                     const uint4 mv = *reinterpret_cast<const uint4*>(mrow + k0 + k);
                     const int4 cv = *reinterpret_cast<const int4*>(codes + k0 + k);
@@ -329,29 +330,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const bool in = c4[q] == -1 || (c4[q] >= 0 && ((m4[q] >> bit) & 1u));
-                        sb |= (uint64_t)(in ? 1u : 0u) << (k + q);
+                        sb |= (in ? 1u : 0u) << (k + q);
                     }
                 }
-                const uint64_t ones = (1ull << C) - 1ull;
+                const uint32_t ones = (1u << C) - 1u;
                 for (int k = 0; k < ns_; ++k)
-                    if ((sb >> k) & 1ull) mem |= ones << (k * (int)C);
+                    if ((sb >> k) & 1u) mem |= ones << (k * (int)C);
             } else {
                 const uint8_t* ps = s_pslot0 + st * kPos;
-                const int k0 = ps[hs], k1 = ps[hs + kHalf - 1];
+                const int k0 = ps[hs], k1 = ps[hs + kPart - 1];
                 // slot k spans positions [k C - o0, (k+1) C - o0) of the tile, o0 = p0 mod C
                 const int o0 = (int)(p0 % C);
                 for (int k = k0; k <= k1; ++k) {
                     const int32_t code = codes[k];
                     const bool in = code == -1 || (code >= 0 && ((mrow[k] >> bit) & 1u));
                     if (in) {
-                        const int a = max(k * (int)C - o0, hs) - hs, e = min((k + 1) * (int)C - o0, hs + kHalf) - hs;
-                        const uint64_t hi_mask = e >= 64 ? ~0ull : ((1ull << e) - 1ull);
-                        mem |= hi_mask & ~((1ull << a) - 1ull);
+                        const int a = max(k * (int)C - o0, hs) - hs, e = min((k + 1) * (int)C - o0, hs + kPart) - hs;
+                        const uint32_t hi_mask = e >= 32 ? ~0u : ((1u << e) - 1u);
+                        mem |= hi_mask & ~((1u << a) - 1u);
                     }
                 }
             }
-            const uint32_t* vw = s_valid0 + st * (kPos / 32) + half * 2;
-            mem &= (uint64_t)vw[0] | ((uint64_t)vw[1] << 32);
+            mem &= s_valid0[st * (kPos / 32) + part];
             if (!y_ok) mem = 0;
         }
         if (more) resolve(p0 + kPos, st ^ 1);
@@ -362,26 +362,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         phase ^= 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-        // tile max over this half's member positions, combined with the partner warp
+        // tile max over this part's member positions, combined with the row's other parts
         float tmax = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < kHalf / 16; ++c) {
+        for (int c = 0; c < kPart / 16; ++c) {
             float v[16];
-            tld16(tS + lane_t + half * kHalf + c * 16, v);
-            const uint32_t m16 = (uint32_t)(mem >> (c * 16));
+            tld16(tS + lane_t + part * kPart + c * 16, v);
+            const uint32_t m16 = mem >> (c * 16);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 if ((m16 >> i) & 1u) tmax = fmaxf(tmax, v[i]);
         }
-        s_xmax[half * kRows + row] = tmax;
+        s_xmax[part * kRows + row] = tmax;
         __syncthreads();                       // partner maxima visible; next tile's tokens visible
         if (more) issue_kv(st ^ 1);            // overlaps this tile's softmax and P V
-        tmax = fmaxf(s_xmax[row], s_xmax[kRows + row]);
+        tmax = fmaxf(fmaxf(s_xmax[row], s_xmax[kRows + row]), fmaxf(s_xmax[2 * kRows + row], s_xmax[3 * kRows + row]));
         tmax = tmax > -INFINITY ? scale * tmax : -INFINITY;
 
-        // Raise the row's reference max if the tile exceeds it by more than kLazy; both warps
+        // Raise the row's reference max if the tile exceeds it by more than kLazy; the 4 warps
         // of the row take the same decision.  O is rescaled warp-collectively (factor 1 on
-        // rows that keep theirs), each warp its half of the columns.
+        // rows that keep theirs), each warp its quarter of the columns.
         const bool need = tmax > -INFINITY && m_ref > -INFINITY && tmax > m_ref + kLazy;
         const float f = need ? exp2f((m_ref - tmax) * kLog2e) : 1.0f;
         if (tmax > -INFINITY && m_ref == -INFINITY) m_ref = tmax;
@@ -391,9 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         }
         if (__any_sync(0xffffffffu, need) && !first_pv) {
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / (16 * kParts); ++c) {
                 float o[16];
-                const uint32_t col = tO + lane_t + half * (D / 2) + c * 16;
+                const uint32_t col = tO + lane_t + part * (D / kParts) + c * 16;
                 tld16(col, o);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) o[i] *= f;
@@ -403,10 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         // P = exp(s S - m) on member positions, split into bf16 hi + lo
         const float sl = scale * kLog2e, ml = m_ref * kLog2e;
 #pragma unroll 1
-        for (int c = 0; c < kHalf / 16; ++c) {
+        for (int c = 0; c < kPart / 16; ++c) {
             float v[16];
-            tld16(tS + lane_t + half * kHalf + c * 16, v);
-            const uint32_t m16 = (uint32_t)(mem >> (c * 16));
+            tld16(tS + lane_t + part * kPart + c * 16, v);
+            const uint32_t m16 = mem >> (c * 16);
             uint32_t hi[8], lo[8];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
@@ -426,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 hi[i / 2] = __byte_perm(h0, h1, 0x7632);
                 lo[i / 2] = __byte_perm(l0, l1, 0x7632);
             }
-            // positions 64 half + 16 c .. +15 are 16-byte chunks 8 half + 2c, +1 of this row
-            const int c16 = half * 8 + 2 * c;
+            // positions 32 part + 16 c .. +15 are 16-byte chunks 4 part + 2c, +1 of this row
+            const int c16 = part * 4 + 2 * c;
             *reinterpret_cast<uint4*>(sPh + kmaj(row, c16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4*>(sPh + kmaj(row, c16 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
             *reinterpret_cast<uint4*>(sPl + kmaj(row, c16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -470,26 +470,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     phase ^= 1;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // partial (o, m, l) of every lane row of the tile: each warp writes its half of o
-    s_xsum[half * kRows + row] = lsum;
+    // partial (o, m, l) of every lane row of the tile: each warp writes its quarter of o
+    s_xsum[part * kRows + row] = lsum;
     __syncthreads();
     {
         float* pp = w.part + (x * w.s_cap + split) * PR;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / (16 * kParts); ++c) {
             float o[16];
-            tld16(tO + lane_t + half * (D / 2) + c * 16, o);
+            tld16(tO + lane_t + part * (D / kParts) + c * 16, o);
             if (y_ok && !abort_sh) {
-                float4* po = reinterpret_cast<float4*>(pp + half * (D / 2) + c * 16);
+                float4* po = reinterpret_cast<float4*>(pp + part * (D / kParts) + c * 16);
                 po[0] = make_float4(o[0], o[1], o[2], o[3]);
                 po[1] = make_float4(o[4], o[5], o[6], o[7]);
                 po[2] = make_float4(o[8], o[9], o[10], o[11]);
                 po[3] = make_float4(o[12], o[13], o[14], o[15]);
             }
         }
-        if (half == 0 && y_ok && !abort_sh) {
+        if (part == 0 && y_ok && !abort_sh) {
             pp[D] = m_ref;
-            pp[D + 1] = s_xsum[row] + s_xsum[kRows + row];
+            pp[D + 1] = (s_xsum[row] + s_xsum[kRows + row]) + (s_xsum[2 * kRows + row] + s_xsum[3 * kRows + row]);
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
     return (size_t)(4 * kbd + 4) * kBlock + 2 * kPos * 4 + 2 * kPos * 4 + 2 * kPos + 2 * (kPos / 32) * 4 +
-           2 * kPos * 4 * 4 + 4 * kRows * 4 + 1024;
+           2 * kPos * 4 * 4 + 2 * kParts * kRows * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
