@@ -150,10 +150,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // lanes (8 lane words): where the tile's entries are 256 consecutive nodes (a dense stretch
 // of the union), each lane reads the 9 bitmap words covering them and realigns them by
 // funnel shifts, warps transpose 32 x 32 bit blocks with ballots through shared memory, and
-// each entry's 8 words are written as one 32-byte segment; other tiles go entry by entry.
+// each entry's 8 words are written as one 32-byte segment.  A tile whose entries lie within
+// 1,024 nodes stages each lane's words of that window and transposes entry by entry from
+// shared memory; sparser tiles read each entry's word from global memory.
 // Grid (tiles, lane-word groups of 8, groups), 256 threads.
 __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mode) {
-    __shared__ uint32_t T[256][9];                    // [lane][node word], padded
+    __shared__ uint32_t T[256][33];                   // [lane][bitmap word of the tile's node window], padded
     __shared__ __align__(16) uint32_t O[256][8];      // [entry][lane word]
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
@@ -205,6 +207,35 @@ __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mod
             uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(u0 + tid) * w.mwords);
             dst[0] = make_uint4(O[tid][0], O[tid][1], O[tid][2], O[tid][3]);
             dst[1] = make_uint4(O[tid][4], O[tid][5], O[tid][6], O[tid][7]);
+            __syncthreads();                          // T and O are reused by the next tile
+        } else if (pn - p0 < 1024) {
+            // the tile's entries lie in a window of <= 1,024 nodes: each lane stages the <= 33
+            // bitmap words of the window once, then warps transpose entry by entry from there
+            const int w0 = p0 >> 5, nw = (pn >> 5) - w0 + 1;
+            const int64_t W = w.W[pl];
+            for (int k = 0; k < nw; ++k) T[tid][k] = (yok && w0 + k < W) ? __ldg(kb + w0 + k) : 0u;
+            __syncthreads();
+            const int e0 = u0 + warp * 32;
+            const int n = max(0, min(32, nu - e0));
+            const int pmy = lane < n ? __ldg(ul + e0 + lane) : p0;
+#pragma unroll 1
+            for (int lw = 0; lw < 8; ++lw) {
+                uint32_t mine = 0;
+#pragma unroll 4
+                for (int t = 0; t < 32; ++t) {
+                    const int pt = __shfl_sync(0xffffffffu, pmy, t);
+                    const uint32_t v = T[lw * 32 + lane][(pt >> 5) - w0];
+                    const uint32_t r = __ballot_sync(0xffffffffu, (v >> (pt & 31)) & 1u);
+                    if (lane == t) mine = r;
+                }
+                O[warp * 32 + lane][lw] = mine;
+            }
+            __syncthreads();
+            if (tid < cnt) {
+                uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(u0 + tid) * w.mwords);
+                dst[0] = make_uint4(O[tid][0], O[tid][1], O[tid][2], O[tid][3]);
+                dst[1] = make_uint4(O[tid][4], O[tid][5], O[tid][6], O[tid][7]);
+            }
             __syncthreads();                          // T and O are reused by the next tile
         } else {
             // warp i: entries u0 + 32 i .., lane words lw0 .. lw0 + 7
