@@ -163,12 +163,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
     const int64_t SEGS = segs_per_split(b.n_gl, (int)C);
-    const int64_t split = blockIdx.x;
+    // grid (lane tiles, splits, groups): the lane tiles of one split run together, so each
+    // K/V row they gather is read from DRAM once and from L2 by the others
+    const int64_t split = blockIdx.y;
     const int64_t sg0 = split * SEGS;
     if (sg0 >= nseg) return;
     const int64_t npos = (min(nseg, sg0 + SEGS) - sg0) * C;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int y0 = blockIdx.y * kRows;
+    const int y0 = blockIdx.x * kRows;
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_sh)), "r"(TCOLS));
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     // for that union chunk, s_pslot the slot of each position; s_valid marks positions
     // holding a token.  Positions and tokens fit 32 bits (caches hold < 2^31 rows).
     const int cs = (C & (C - 1)) == 0 ? __ffs((int)C) - 1 : -1;   // shift for power-of-two C
-    const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.y * 4;
+    const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.x * 4;
     auto resolve = [&](int64_t p0, int st) {
         if (tid < kPos) {
             const int pp = (int)p0 + tid;
@@ -512,7 +514,7 @@ cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, fl
     if (e != cudaSuccess) return e;
     ProfScope ps_("k_attn_tc", st);
     const int lane_tiles = (b.n_gl + kRows - 1) / kRows;
-    dim3 grid((unsigned)max_splits, lane_tiles, b.n_groups);
+    dim3 grid(lane_tiles, (unsigned)max_splits, b.n_groups);   // splits <= 65,535 (checked by the caller)
     const size_t smem = attn_tc_smem(b.d);
     if (b.d == 128) {
         cudaFuncSetAttribute(k_attn_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
