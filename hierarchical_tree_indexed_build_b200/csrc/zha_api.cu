@@ -238,9 +238,10 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
     int first_merge = 2;
     int64_t lo1 = n_old / C;
     if (n_old == 0) {
-        // Whole subtrees of up to 256 tokens are streamed by one worker each.
+        // Whole subtrees of up to 64 tokens are streamed by one worker each (more workers in
+        // flight than with larger spans; the levels above come from merges).
         int k_emit = 1;
-        while (k_emit < L && ipow(C, k_emit + 1) <= 256) ++k_emit;
+        while (k_emit < L && ipow(C, k_emit + 1) <= 64) ++k_emit;
         const int64_t n_emit = n_new / ipow(C, k_emit);
         ba.k_emit = k_emit;
         ba.u0 = 0;
