@@ -148,7 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][4][kPos] lane masks: [lane word][slot]
     float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [kParts][kRows] tile max per part
     float* s_xsum = s_xmax + kParts * kRows;                                // [kParts][kRows] row sums per part
-    __shared__ __align__(8) uint64_t mbar;
+    // mbS: the S = Q K^T of a tile is done; mbO: the P V of a tile is done (O, sP and that
+    // tile's V buffer free again).  One arrival each per tile, each waited once per tile.
+    __shared__ __align__(8) uint64_t mbS, mbO;
     __shared__ uint32_t tmem_sh;
     __shared__ int abort_flag;
     volatile int& abort_sh = abort_flag;
@@ -177,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbar)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbS)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbO)));
         asm volatile("fence.mbarrier_init.release.cluster;");
         abort_sh = 0;
     }
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     const __nv_bfloat16* Kg = sq.K + (int64_t)g * sq.ld * D;
     const __nv_bfloat16* Vg = sq.V + (int64_t)g * sq.ld * D;
-    uint32_t phase = 0;
+    uint32_t phS = 0, phO = 0;
     bool first_pv = true;
 
     // Tokens of tile p0 into buffer st (threads 0..127, one position each): sink segment
@@ -294,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             }
     };
 
-    // Pipeline: tile i's S was issued (with tile i-1's P V) at the end of the previous
-    // iteration; its K/V were gathered during tile i-1's softmax.  One commit per tile.
+    // Pipeline: tile i's S was issued at the end of the previous iteration, ahead of tile
+    // i-1's P V, so the softmax of tile i waits only for S; the P V runs under tile i's
+    // membership and row maxima and is waited for just before O, sP or its V buffer is
+    // reused.  Tile i's K/V were gathered during tile i-1's softmax.
     resolve(0, 0);
     __syncthreads();
     issue_kv(0);
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     __syncthreads();
     if (tid == 0) {
         issue_s();
-        commit(su32(&mbar));
+        commit(su32(&mbS));
     }
     __syncwarp();
     int st = 0;
@@ -357,11 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             if (!y_ok) mem = 0;
         }
         if (more) resolve(p0 + kPos, st ^ 1);
-        if (!wait_phase(su32(&mbar), phase) && lane == 0) {
+        if (!wait_phase(su32(&mbS), phS) && lane == 0) {
             atomicOr(w.status, kStatusTimeout);
             abort_sh = 1;
         }
-        phase ^= 1;
+        phS ^= 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
         // tile max over this part's member positions, combined with the row's other parts
@@ -376,6 +381,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 if ((m16 >> i) & 1u) tmax = fmaxf(tmax, v[i]);
         }
         s_xmax[part * kRows + row] = tmax;
+        // the previous tile's P V must be done before O is rescaled, sP rewritten and its V
+        // buffer refilled by the gather below
+        if (!first_pv) {
+            if (!wait_phase(su32(&mbO), phO) && lane == 0) {
+                atomicOr(w.status, kStatusTimeout);
+                abort_sh = 1;
+            }
+            phO ^= 1;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        }
         __syncthreads();                       // partner maxima visible; next tile's tokens visible
         if (more) issue_kv(st ^ 1);            // overlaps this tile's softmax and P V
         tmax = fmaxf(fmaxf(s_xmax[row], s_xmax[kRows + row]), fmaxf(s_xmax[2 * kRows + row], s_xmax[3 * kRows + row]));
@@ -442,6 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (tid == 0) {
+            // S of the next tile first (it reads only sQ / sK and writes the S columns, which
+            // this tile has finished reading), then this tile's P V
+            if (more && !abort_sh) {
+                issue_s();
+                commit(su32(&mbS));
+            }
             const uint32_t v0 = su32(sV0 + st * KBD * kBlock);
 #pragma unroll
             for (int pass = 0; pass < 2; ++pass) {
@@ -455,21 +476,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                              idesc_bf16(D, 1), (first_pv && pass == 0 && ks == 0) ? 0u : 1u);
                 }
             }
-            // S of the next tile reads only sQ / sK and writes the S columns, whose values
-            // this tile no longer needs; one commit covers both
-            if (more && !abort_sh) issue_s();
-            commit(su32(&mbar));
+            commit(su32(&mbO));
         }
         __syncwarp();
         first_pv = false;
         if (abort_sh) break;
     }
     // the commit of the last tile (its P V): wait once more, then O is final
-    if (!wait_phase(su32(&mbar), phase) && lane == 0) {
+    if (!wait_phase(su32(&mbO), phO) && lane == 0) {
         atomicOr(w.status, kStatusTimeout);
         abort_sh = 1;
     }
-    phase ^= 1;
+    phO ^= 1;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     // partial (o, m, l) of every lane row of the tile: each warp writes its quarter of o

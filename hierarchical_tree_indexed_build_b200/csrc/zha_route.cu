@@ -18,6 +18,8 @@
 //              max e - e, exact (e, j) ordering inside the boundary bin), kept bitmap out.
 #include <math.h>
 
+#include <type_traits>
+
 #include "zha_common.cuh"
 #include "zha_launch.h"
 #include "zha_profile.h"
@@ -294,7 +296,7 @@ constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
 constexpr int kUn = 2;               // 128-candidate blocks per warp in flight (gather path)
-constexpr int kPD = 6;               // per-thread prefetch ring depth (cp.async)
+constexpr int kPD = 4;               // per-thread prefetch ring depth (cp.async), a power of two
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -316,18 +318,46 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 // The cut's arithmetic is shared by every pass and kept off the quarter-rate conversion
 // unit: one ex2 per candidate, the rest on the FMA and integer pipes.
+// Adds the 64-bit mass (hi, lo) to a bin kept as two 32-bit words: lo into the low word
+// (with return, to see its wrap), hi plus the wrap into the high word.  Both atomics are
+// predicated (nothing for a zero mass; the second only when it adds something), so the
+// update has no branches.
+__device__ __forceinline__ void hist_add(uint32_t alo, uint32_t ahi, uint32_t lo, uint32_t hi) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .u32 old, sum, c;\n\t"
+        "setp.ne.u32 p, %2, 0;\n\t"
+        "mov.u32 old, 0;\n\t"
+        "@p atom.shared.add.u32 old, [%0], %3;\n\t"
+        "add.u32 sum, old, %3;\n\t"
+        "setp.lt.u32 q, sum, old;\n\t"
+        "selp.u32 c, 1, 0, q;\n\t"
+        "add.u32 c, c, %4;\n\t"
+        "setp.ne.and.u32 q, c, 0, p;\n\t"
+        "@q red.shared.add.u32 [%1], c;\n\t}\n"
+        ::"r"(alo), "r"(ahi), "r"(lo | hi), "r"(lo), "r"(hi)
+        : "memory");
+}
+
 struct SelMath {
     float nl2M;     // -M log2(e)
     float m64;      // M kBinScale
-    // fixed-point mass floor(exp(e - M) 2^39), read from the bits of the float exp(e - M)
-    __device__ __forceinline__ unsigned long long mass(float e) const {
-        const float f = ex2_approx(fmaf(e, 1.4426950408889634f, nl2M));   // in [0, 1]
+    // fixed-point mass floor(exp(e - M) 2^39) as 32-bit words (lo, hi), read from the bits of
+    // the float f = exp(e - M) in [0, 1]: the 24-bit significand shifted by exponent - 111
+    // (2^39 / 2^23 = 2^16 at f = 1), without branches: the clamped funnel shifts give 0 for
+    // shifts of 32 or more, which covers f = 0 (exponent field 0, shift -111)
+    __device__ __forceinline__ void mass2(float e, uint32_t& lo, uint32_t& hi) const {
+        const float f = ex2_approx(fmaf(e, 1.4426950408889634f, nl2M));
         const uint32_t u = __float_as_uint(f);
-        const int ex = (int)(u >> 23);                                        // f >= 0
+        const int sh = (int)(u >> 23) - 111;                                  // f >= 0: no sign bit
         const uint32_t mant = (u & 0x7fffffu) | 0x800000u;
-        const int sh = ex - 111;                                              // 2^39 / 2^23 = 2^16 at ex = 127
-        if (ex == 0) return 0ull;
-        return sh >= 0 ? ((unsigned long long)mant << sh) : (unsigned long long)(mant >> min(-sh, 31));
+        const uint32_t up = (uint32_t)max(sh, 0), dn = (uint32_t)max(-sh, 0);
+        hi = __funnelshift_lc(mant, 0u, up);                                  // (0:mant) << up, high word
+        lo = __funnelshift_rc(__funnelshift_lc(0u, mant, up), 0u, dn);        // low word, then >> dn
+    }
+    __device__ __forceinline__ unsigned long long mass(float e) const {
+        uint32_t lo, hi;
+        mass2(e, lo, hi);
+        return ((unsigned long long)hi << 32) | lo;
     }
     // bin = round((M - e) kBinScale), clamped to kNB - 1 (magic-number rounding, no conversion)
     __device__ __forceinline__ int bin(float e) const {
@@ -350,8 +380,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     uint32_t* hlo = reinterpret_cast<uint32_t*>(sel_smem);   // [kNB]
     uint32_t* hhi = hlo + kNB;                                // [kNB]
     unsigned long long* keys = sel_smem + kNB;                // [kCap]
-    float4* pref = reinterpret_cast<float4*>(keys + kCap);   // [threads][kPD] prefetched scores
-    int32_t* prefj = reinterpret_cast<int32_t*>(pref + (size_t)kSelThreads * kPD);   // [threads][kPD] union entries
+    float4* pref = reinterpret_cast<float4*>(keys + kCap);   // [kPD][threads] prefetched scores
+    int32_t* prefj = reinterpret_cast<int32_t*>(pref + (size_t)kSelThreads * kPD);   // [kPD][threads] union entries
     auto hist = [&](int i) -> unsigned long long { return ((unsigned long long)hhi[i] << 32) | hlo[i]; };
     __shared__ unsigned long long red_u[33];
     __shared__ int red_i[33];
@@ -418,21 +448,27 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     // every warp visits its blocks with kUn loads in flight; body(bk, scores[4], j0)
     // Contiguous layouts: every thread prefetches its own float4 of scores (and, when node
     // ids are needed, its union-list entry) kPD - 1 iterations ahead with cp.async into a
-    // private shared-memory ring; it reads back only what it copied, so no barrier is needed.
-    auto stream = [&](bool need_j, auto&& body) {
-        float4* my = pref + (size_t)threadIdx.x * kPD;
-        int32_t* myj = prefj + (size_t)threadIdx.x * kPD;
+    // private slot of a shared-memory ring laid out [slot][thread] (a warp's 32 float4 of one
+    // slot are 512 contiguous bytes); it reads back only what it copied, so no barrier is
+    // needed.  need_j is a compile-time flag (std::true_type / std::false_type).
+    auto stream = [&](auto nj, auto&& body) {
+        constexpr bool need_j = decltype(nj)::value;
         const int niter = warp < nblk ? (nblk - warp + nwarps - 1) / nwarps : 0;   // uniform in a warp
         const bool want_u = need_j && !top;
+        const int kStep = nwarps * 128;                 // candidates between a thread's iterations
+        const int kb0 = warp * 128 + 4 * lane;
+        const uint32_t ring = smem_u32(pref + threadIdx.x);
+        const uint32_t ringj = smem_u32(prefj + threadIdx.x);
         auto issue = [&](int t) {
-            const int k0 = (warp + t * nwarps) * 128 + 4 * lane;
+            const int k0 = kb0 + t * kStep;
             const bool in = t < niter && k0 < nc;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(my + t % kPD)),
+            const uint32_t sl = (uint32_t)(t & (kPD - 1));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ring + sl * (kSelThreads * 16)),
                          "l"(e + (in ? k0 : 0)), "r"(in ? 16u : 0u)
                          : "memory");
             if (want_u) {
                 const int uk = in ? (cs >= 0 ? (k0 >> cs) : k0 / C) : 0;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(myj + t % kPD)),
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(ringj + sl * (kSelThreads * 4)),
                              "l"(ul + uk), "r"(in ? 4u : 0u)
                              : "memory");
             }
@@ -443,38 +479,40 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         for (int t = 0; t < niter; ++t) {
             issue(t + kPD - 1);
             asm volatile("cp.async.wait_group %0;" ::"n"(kPD - 1) : "memory");
-            const int bk = warp + t * nwarps;
-            const int k0 = bk * 128 + 4 * lane;
-            const float4 xv = my[t % kPD];
-            float4 ev;
-            ev.x = k0 < nc ? xv.x : -INFINITY;
-            ev.y = k0 + 1 < nc ? xv.y : -INFINITY;
-            ev.z = k0 + 2 < nc ? xv.z : -INFINITY;
-            ev.w = k0 + 3 < nc ? xv.w : -INFINITY;
+            const int k0 = kb0 + t * kStep;
+            const int sl = t & (kPD - 1);
+            float4 ev = pref[sl * kSelThreads + threadIdx.x];
+            if (k0 + 3 >= nc) {                         // the row's last, partial float4
+                ev.x = k0 < nc ? ev.x : -INFINITY;
+                ev.y = k0 + 1 < nc ? ev.y : -INFINITY;
+                ev.z = k0 + 2 < nc ? ev.z : -INFINITY;
+                ev.w = -INFINITY;
+            }
             int j0 = -1;
-            if (need_j && k0 < nc) {
-                if (top) {
-                    j0 = k0;
-                } else {
-                    const int pj = myj[t % kPD];
-                    const int uk = cs >= 0 ? (k0 >> cs) : k0 / C;
-                    j0 = cs >= 0 ? (pj << cs) + (k0 & (C - 1)) : pj * C + (k0 - uk * C);
+            if constexpr (need_j) {
+                if (k0 < nc) {
+                    if (top) {
+                        j0 = k0;
+                    } else {
+                        const int pj = prefj[sl * kSelThreads + threadIdx.x];
+                        j0 = cs >= 0 ? (pj << cs) + (k0 & (C - 1)) : pj * C + (k0 - (k0 / C) * C);
+                    }
                 }
             }
-            body(bk, ev, j0);
+            body(warp + t * nwarps, ev, j0);
         }
         asm volatile("cp.async.wait_group 0;" ::: "memory");
     };
-    auto for_cands = [&](bool need_j, auto&& body) {
+    auto for_cands = [&](auto nj, auto&& body) {
         if (contig) {
-            stream(need_j, body);
+            stream(nj, body);
             return;
         }
         for (int b0 = warp; b0 < nblk; b0 += kUn * nwarps) {
             float4 ev[kUn];
             int j0[kUn];
 #pragma unroll
-            for (int u = 0; u < kUn; ++u) load(b0 + u * nwarps, ev[u], j0[u], need_j);
+            for (int u = 0; u < kUn; ++u) load(b0 + u * nwarps, ev[u], j0[u], decltype(nj)::value);
 #pragma unroll
             for (int u = 0; u < kUn; ++u) {
                 const int bk = b0 + u * nwarps;
@@ -517,20 +555,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         }
         if (threadIdx.x == 0) s_nkeys = 0;
         __syncthreads();
-        for_cands(false, [&](int bk, const float4 ev4, int j0) {
+        for_cands(std::false_type{}, [&](int bk, const float4 ev4, int j0) {
             const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
             // -inf (off the frontier) gives mass 0 and the last bin: computed without branches,
-            // only the atomic is predicated
+            // the atomics are predicated
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const unsigned long long ms = sm.mass(v[c]);
-                const int bn = sm.bin(v[c]);
-                if (ms) {
-                    const uint32_t lo = (uint32_t)ms, hi = (uint32_t)(ms >> 32);
-                    const uint32_t old = atomicAdd(&hlo[bn], lo);
-                    const uint32_t carry = old + lo < old ? 1u : 0u;
-                    if (hi + carry) atomicAdd(&hhi[bn], hi + carry);
-                }
+                uint32_t lo, hi;
+                sm.mass2(v[c], lo, hi);
+                hist_add(smem_u32(hlo + sm.bin(v[c])), smem_u32(hhi + sm.bin(v[c])), lo, hi);
             }
         });
         __syncthreads();
@@ -578,7 +611,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
 
     // pass 2: kept bits of the bins above the boundary; boundary-bin candidates collected
     unsigned long long cnt = 0;
-    for_cands(true, [&](int bk, const float4 ev4, int j0) {
+    for_cands(std::true_type{}, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
         uint32_t nib = 0, col = 0;
 #pragma unroll
@@ -667,7 +700,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     } else {
         // rare: too many candidates in one bin - bisection on the exact key order, then a pass
         unsigned long long klo = ~0ull, khi = 0ull;
-        for_cands(true, [&](int bk, const float4 ev4, int j0) {
+        for_cands(std::true_type{}, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -683,7 +716,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         while (lo < hi && iters < 70) {
             const unsigned long long mid = lo + (hi - lo) / 2;
             unsigned long long acc = 0;
-            for_cands(true, [&](int bk, const float4 ev4, int j0) {
+            for_cands(std::true_type{}, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
@@ -697,7 +730,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
         }
         if (threadIdx.x == 0 && iters >= 70) atomicOr(w.status, kStatusSelectFallbackLimit);
         unsigned long long extra = 0;
-        for_cands(true, [&](int bk, const float4 ev4, int j0) {
+        for_cands(std::true_type{}, [&](int bk, const float4 ev4, int j0) {
         const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c)

@@ -22,6 +22,11 @@ def _report(name, rep, e1, e2):
 
 # ----------------------------------------------------------------------------- build
 
+# Chunk sizes that neither divide nor are a multiple of the build's 8-token key groups, with
+# 8 reference queries (one warp of tensor-core dot products per node).
+ODD6 = inputs.Geometry(C=6, L=3, R=8, d=64, Hq=4, Hkv=2)
+ODD12 = inputs.Geometry(C=12, L=2, R=8, d=64, Hq=4, Hkv=2)
+
 @needs_cuda
 @pytest.mark.parametrize("geom,n_tokens", [
     (inputs.TINY, 4096),                 # the tiny workload's tree
@@ -29,6 +34,8 @@ def _report(name, rep, e1, e2):
     (inputs.DEEP, 3 * 4096 + 1234),      # C4 L6, ragged
     (inputs.MID, 2 * 4096 + 700),        # C16 L3, ragged
     (inputs.WIDE, 256 * 40 + 100),       # C256 L1, ragged
+    (ODD6, 4096 + 333),                  # C6: key groups of 6 tokens
+    (ODD12, 4096 + 333),                 # C12: chunks of 8 + 4 tokens
 ])
 def test_build_summaries_match_oracle(geom, n_tokens):
     seq = inputs.make_sequence(geom, n_tokens, n_tokens, seed=11)
@@ -49,7 +56,7 @@ def test_build_deep64k_all_nodes():
 
 
 @needs_cuda
-@pytest.mark.parametrize("geom", [inputs.DEEP, inputs.MID, inputs.WIDE, inputs.TINY])
+@pytest.mark.parametrize("geom", [inputs.DEEP, inputs.MID, inputs.WIDE, inputs.TINY, ODD6, ODD12])
 def test_append_is_bit_identical_to_rebuild(geom):
     """Growing a tree by appends (single tokens, then a bulk range) gives exactly the
     summaries of a tree built over the final length in one pass."""
