@@ -543,7 +543,14 @@ extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, fl
     for (int it = 0; it < dec->Lmax; ++it) {
         if (it > 0) ZHA_CUDA(launch_union(b, dec->w, it, 0, st));
         ZHA_CUDA(launch_score(b, dec->w, it, scale, st));
-        ZHA_CUDA(launch_select(b, dec->w, it, st));
+        // candidates of a lane at level L_s - it: at most that level's complete nodes
+        int64_t max_cands = 0;
+        for (int sq = 0; sq < dec->n_seq; ++sq) {
+            const SeqDev& h = dec->seq_host[sq];
+            const int lev = h.L - it;
+            if (lev >= 1) max_cands = std::max<int64_t>(max_cands, h.n[lev]);
+        }
+        ZHA_CUDA(launch_select(b, dec->w, it, max_cands, st));
     }
     dec->routed = true;
     dec->last_n_q = n_q;

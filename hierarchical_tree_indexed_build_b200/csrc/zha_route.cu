@@ -292,6 +292,8 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
 // ----------------------------------------------------------------------------- select
 
 constexpr int kSelThreads = 512;
+constexpr int kSelThreadsSmall = 128;  // block size when every lane has <= kSelSmallCands candidates
+constexpr int64_t kSelSmallCands = 16384;
 constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
@@ -372,7 +374,8 @@ struct SelMath {
 // lane's frontier maximum M and size F.  Two passes over the candidates: a histogram of fixed-point masses
 // over bins of M - e, then the kept bits of the bins above the boundary bin and the
 // boundary bin's candidates, which are sorted by (e desc, j asc) to finish the prefix.
-__global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int it) {
+template <int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int it) {
     extern __shared__ unsigned long long sel_smem[];
     // bin masses as two 32-bit words (shared-memory 64-bit atomics are several times slower):
     // hlo accumulates the low words, hhi the high words and every wrap of hlo, so a bin's
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
     uint32_t* hhi = hlo + kNB;                                // [kNB]
     unsigned long long* keys = sel_smem + kNB;                // [kCap]
     float4* pref = reinterpret_cast<float4*>(keys + kCap);   // [kPD][threads] prefetched scores
-    int32_t* prefj = reinterpret_cast<int32_t*>(pref + (size_t)kSelThreads * kPD);   // [kPD][threads] union entries
+    int32_t* prefj = reinterpret_cast<int32_t*>(pref + (size_t)NT * kPD);   // [kPD][threads] union entries
     auto hist = [&](int i) -> unsigned long long { return ((unsigned long long)hhi[i] << 32) | hlo[i]; };
     __shared__ unsigned long long red_u[33];
     __shared__ int red_i[33];
@@ -463,12 +466,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             const int k0 = kb0 + t * kStep;
             const bool in = t < niter && k0 < nc;
             const uint32_t sl = (uint32_t)(t & (kPD - 1));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ring + sl * (kSelThreads * 16)),
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ring + sl * (NT * 16)),
                          "l"(e + (in ? k0 : 0)), "r"(in ? 16u : 0u)
                          : "memory");
             if (want_u) {
                 const int uk = in ? (cs >= 0 ? (k0 >> cs) : k0 / C) : 0;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(ringj + sl * (kSelThreads * 4)),
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(ringj + sl * (NT * 4)),
                              "l"(ul + uk), "r"(in ? 4u : 0u)
                              : "memory");
             }
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             asm volatile("cp.async.wait_group %0;" ::"n"(kPD - 1) : "memory");
             const int k0 = kb0 + t * kStep;
             const int sl = t & (kPD - 1);
-            float4 ev = pref[sl * kSelThreads + threadIdx.x];
+            float4 ev = pref[sl * NT + threadIdx.x];
             if (k0 + 3 >= nc) {                         // the row's last, partial float4
                 ev.x = k0 < nc ? ev.x : -INFINITY;
                 ev.y = k0 + 1 < nc ? ev.y : -INFINITY;
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
                     if (top) {
                         j0 = k0;
                     } else {
-                        const int pj = prefj[sl * kSelThreads + threadIdx.x];
+                        const int pj = prefj[sl * NT + threadIdx.x];
                         j0 = cs >= 0 ? (pj << cs) + (k0 & (C - 1)) : pj * C + (k0 - (k0 / C) * C);
                     }
                 }
@@ -567,42 +570,48 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(Batch b, Work w, int 
             }
         });
         __syncthreads();
-        unsigned long long zloc = 0;
-        for (int i = threadIdx.x; i < kNB; i += blockDim.x) zloc += hist(i);
-        const unsigned long long Z = block_sum<unsigned long long>(zloc, red_u);
+        // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*).  Thread t owns the BPT
+        // bins from BPT t; one block-wide exclusive scan of the per-thread sums gives Z and
+        // each thread's prefix, and the thread whose range holds the target finds b* there.
+        constexpr int BPT = kNB / NT;
+        static_assert(BPT % 4 == 0, "whole 16-byte groups of bins per thread");
+        if (threadIdx.x == 0) {   // only kept if no range holds the target (Z = 0)
+            s_bstar = kNB - kNB / 32;
+            s_cumb = 0;
+        }
+        unsigned long long hb[BPT];
+#pragma unroll
+        for (int v = 0; v < BPT / 4; ++v) {
+            const uint4 l4 = reinterpret_cast<const uint4*>(hlo)[threadIdx.x * (BPT / 4) + v];
+            const uint4 h4 = reinterpret_cast<const uint4*>(hhi)[threadIdx.x * (BPT / 4) + v];
+            hb[4 * v + 0] = ((unsigned long long)h4.x << 32) | l4.x;
+            hb[4 * v + 1] = ((unsigned long long)h4.y << 32) | l4.y;
+            hb[4 * v + 2] = ((unsigned long long)h4.z << 32) | l4.z;
+            hb[4 * v + 3] = ((unsigned long long)h4.w << 32) | l4.w;
+        }
+        unsigned long long loc = 0;
+#pragma unroll
+        for (int k = 0; k < BPT; ++k) loc += hb[k];
+        unsigned long long Z;
+        const unsigned long long excl = block_excl_scan<unsigned long long>(loc, red_u, Z);
         unsigned long long target = (unsigned long long)ceil((double)b.p * (double)Z);
         if (target < 1ull) target = 1ull;
         if (target > Z) target = Z;
-        // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*)
-        if (warp == 0) {
-            constexpr int per = kNB / 32;
-            unsigned long long ls = 0;
-#pragma unroll 4
-            for (int k = 0; k < per; ++k) ls += hist(lane * per + k);
-            unsigned long long incl = ls;
+        if (excl < target && target <= excl + loc) {
+            unsigned long long cum = excl, cumb = excl;
+            int bs = BPT * threadIdx.x + BPT - 1;
+            bool hit = false;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long t = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += t;
-            }
-            const unsigned long long excl = incl - ls;
-            const unsigned bal = __ballot_sync(kFull, excl < target && target <= incl);
-            const int src = bal ? __ffs(bal) - 1 : 31;
-            if (lane == src) {
-                unsigned long long cum = excl;
-                int bs = lane * per + per - 1;
-#pragma unroll 1
-                for (int k = 0; k < per; ++k) {
-                    const int bb = lane * per + k;
-                    if (cum + hist(bb) >= target) {
-                        bs = bb;
-                        break;
-                    }
-                    cum += hist(bb);
+            for (int k = 0; k < BPT; ++k) {
+                if (!hit && cum + hb[k] >= target) {
+                    hit = true;
+                    bs = BPT * threadIdx.x + k;
+                    cumb = cum;
                 }
-                s_bstar = bs;
-                s_cumb = cum;
+                cum += hb[k];
             }
+            s_bstar = bs;
+            s_cumb = cumb;
         }
         __syncthreads();
         bstar = s_bstar;
@@ -783,11 +792,18 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
     return cudaGetLastError();
 }
 
-cudaError_t launch_select(const Batch& b, const Work& w, int it, cudaStream_t st) {
-    const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8 + (size_t)kSelThreads * kPD * (16 + 4);
-    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t launch_select(const Batch& b, const Work& w, int it, int64_t max_cands, cudaStream_t st) {
     ProfScope ps_("k_select", st);
-    k_select<<<b.n_lanes, kSelThreads, smem, st>>>(b, w, it);
+    // Lanes with few candidates (upper levels) are latency-bound: small blocks, more per SM.
+    auto go = [&](auto kern, int nt) {
+        const size_t smem = (size_t)kNB * 8 + (size_t)kCap * 8 + (size_t)nt * kPD * (16 + 4);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<b.n_lanes, nt, smem, st>>>(b, w, it);
+    };
+    if (max_cands <= kSelSmallCands)
+        go(k_select<kSelThreadsSmall>, kSelThreadsSmall);
+    else
+        go(k_select<kSelThreads>, kSelThreads);
     return cudaGetLastError();
 }
 
