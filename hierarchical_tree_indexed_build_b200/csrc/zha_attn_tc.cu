@@ -134,8 +134,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     constexpr int kPart = kPos / kParts;        // positions per warp of a row (32)
     constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~uintptr_t(1023));
+    // 1024-byte aligned start, reached by pointer arithmetic on the shared array so that every
+    // pointer derived from it stays a shared-memory pointer (plain shared loads and stores)
+    unsigned char* base = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sQ = base;                               // KBD blocks
     unsigned char* sK = sQ + KBD * kBlock;                  // KBD blocks
     unsigned char* sV0 = sK + KBD * kBlock;                 // 2 x KBD blocks (MN-major, double buffer)

@@ -307,8 +307,9 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     constexpr uint32_t kCols = 512;
     constexpr uint32_t kNodeBytes = kPlanes * KB * 16 * 128;   // both planes of one node
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* base = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned start, reached by pointer arithmetic on the shared array so that every
+    // pointer derived from it stays a shared-memory pointer (plain shared loads and stores)
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sB0 = base;                                             // [kStages][2 planes][P_BYTES]
     float* sBv = reinterpret_cast<float*>(sB0 + kStages * STAGE);          // [kStages][kNodes][16] b values
     uint32_t* sMask = reinterpret_cast<uint32_t*>(sBv + kStages * kTileN); // [kStages][kNodes][kLW] membership
