@@ -117,8 +117,14 @@ __device__ __forceinline__ void fold_child(float& mx, float& z, float (&acc)[D /
     const float cp = expf(mx - mn);   // mx = -inf -> 0
     const float cc = expf(lc - mn);
     z = fmaf(z, cp, cc);
+    // packed fp32x2: the same multiply and fused multiply-add per element
+    const float2 cp2 = make_float2(cp, cp), cc2 = make_float2(cc, cc);
 #pragma unroll
-    for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], cp, mc[k] * cc);
+    for (int k = 0; k < D / 4; k += 2) {
+        const float2 a2 = __ffma2_rn(make_float2(acc[k], acc[k + 1]), cp2, __fmul2_rn(make_float2(mc[k], mc[k + 1]), cc2));
+        acc[k] = a2.x;
+        acc[k + 1] = a2.y;
+    }
     mx = mn;
 }
 
@@ -173,7 +179,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // every node of levels 1..k_emit beneath it.  Level-1 state lives in registers, levels
 // 2..k_emit in shared memory ([level][field][thread]).
 template <int D>
-__global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
+__global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
     extern __shared__ float smem_state[];
     const int wt = 4 * a.R;
     const int wpb = blockDim.x / wt;
@@ -233,30 +239,36 @@ __global__ void __launch_bounds__(128) k_build_stream(BuildArgs a) {
         const int ntk = (int)(rest < kTok ? rest : kTok);
         for (int tk = 0; tk < ntk; ++tk) {
             const int64_t tt = (int64_t)grp * kTok + tk;
-            float kv[D / 4];
+            // packed fp32x2 arithmetic: two independent IEEE single-precision operations per
+            // instruction (dims 2j, 2j+1 of this thread's D/4)
+            float2 kv[D / 8];
             {
                 const uint2* p = reinterpret_cast<const uint2*>(kb + tk * D);
 #pragma unroll
                 for (int i = 0; i < D / 16; ++i) {
                     const uint2 uu = p[4 * i + q];
-                    const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.x));
-                    const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.y));
-                    kv[4 * i + 0] = x0.x;
-                    kv[4 * i + 1] = x0.y;
-                    kv[4 * i + 2] = x1.x;
-                    kv[4 * i + 3] = x1.y;
+                    kv[2 * i + 0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.x));
+                    kv[2 * i + 1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu.y));
                 }
             }
-            float dot = 0.0f;
+            // q_r.k_t over this thread's dims as two interleaved partial sums
+            float2 d2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int k = 0; k < D / 4; ++k) dot = fmaf(qv[k], kv[k], dot);
-            const float sc = a.scale * quad_sum(dot);
+            for (int j = 0; j < D / 8; ++j) d2 = __ffma2_rn(make_float2(qv[2 * j], qv[2 * j + 1]), kv[j], d2);
+            const float sc = a.scale * quad_sum(d2.x + d2.y);
             const float mn = fmaxf(mx, sc);
             const float c = expf(mx - mn);
             const float wgt = expf(sc - mn);
             z = fmaf(z, c, wgt);
+            {
+                const float2 c2 = make_float2(c, c), w2 = make_float2(wgt, wgt);
 #pragma unroll
-            for (int k = 0; k < D / 4; ++k) acc[k] = fmaf(acc[k], c, wgt * kv[k]);
+                for (int j = 0; j < D / 8; ++j) {
+                    const float2 a2 = __ffma2_rn(make_float2(acc[2 * j], acc[2 * j + 1]), c2, __fmul2_rn(w2, kv[j]));
+                    acc[2 * j] = a2.x;
+                    acc[2 * j + 1] = a2.y;
+                }
+            }
             mx = mn;
             if (--left == 0) {
                 left = C;
