@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--p", type=float, default=0.95)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", default="deep1m", choices=["deep1m", "deep64k", "wide256k"],
+    ap.add_argument("--workload", default="deep1m", choices=["deep1m", "deep64k", "deep256k", "wide256k"],
                     help="deep1m is the benchmark; the smaller ones serve profiling runs")
     return ap.parse_args()
 
@@ -309,6 +309,12 @@ def load_workload(name):
     if name == "wide256k":
         wl = inputs.wide_256k()
         wl.n_append = 0
+        return wl
+    if name == "deep256k":
+        # the 1M workload's shapes over 262,144 tokens: K/V and tree (1.7 GB) exceed L2 while a
+        # full ncu capture stays small
+        wl = inputs.deep_1m(n_tokens=262144, n_append=0)
+        wl.name = "deep_256k_C4L6"
         return wl
     return inputs.deep_1m()
 

@@ -428,8 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             uint32_t hi[8], lo[8];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
-                const float e0 = ex2_approx(fmaf(sl, v[i], -ml));
-                const float e1 = ex2_approx(fmaf(sl, v[i + 1], -ml));
+                const float2 a2 = __ffma2_rn(make_float2(sl, sl), make_float2(v[i], v[i + 1]), make_float2(-ml, -ml));
+                const float e0 = ex2_approx(a2.x);
+                const float e1 = ex2_approx(a2.y);
                 const float p0v = ((m16 >> i) & 1u) ? e0 : 0.0f;
                 const float p1v = ((m16 >> (i + 1)) & 1u) ? e1 : 0.0f;
                 lsum += p0v;

@@ -553,14 +553,18 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                 tmem_ld32(tmem + tlane + (uint32_t)(slot * kTileN + pr * 2 * kR), v);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    // s D + b_r as packed fp32x2 fused multiply-adds (two records per
+                    // instruction, the same rounding as one FMA each), then the maximum
                     float bb = -INFINITY;
+                    const float2 s2 = make_float2(scale, scale);
 #pragma unroll
                     for (int r4 = 0; r4 < kR / 4; ++r4) {
                         const float4 bq = bv4[(pr * 2 + h) * (kR / 4) + r4];
-                        bb = fmaxf(bb, fmaf(scale, v[h * kR + 4 * r4 + 0], bq.x));
-                        bb = fmaxf(bb, fmaf(scale, v[h * kR + 4 * r4 + 1], bq.y));
-                        bb = fmaxf(bb, fmaf(scale, v[h * kR + 4 * r4 + 2], bq.z));
-                        bb = fmaxf(bb, fmaf(scale, v[h * kR + 4 * r4 + 3], bq.w));
+                        const float2 e0 = __ffma2_rn(s2, make_float2(v[h * kR + 4 * r4 + 0], v[h * kR + 4 * r4 + 1]),
+                                                     make_float2(bq.x, bq.y));
+                        const float2 e1 = __ffma2_rn(s2, make_float2(v[h * kR + 4 * r4 + 2], v[h * kR + 4 * r4 + 3]),
+                                                     make_float2(bq.z, bq.w));
+                        bb = fmaxf(bb, fmaxf(fmaxf(e0.x, e0.y), fmaxf(e1.x, e1.y)));
                     }
                     best[pr * 2 + h] = bb;
                 }
