@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--p", type=float, default=0.95)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparison")
     ap.add_argument("--workload", default="deep1m", choices=["deep1m", "deep64k", "deep256k", "wide256k"],
                     help="deep1m is the benchmark; the smaller ones serve profiling runs")
     return ap.parse_args()
@@ -263,6 +264,33 @@ def run_ours(args, rank, world, dev):
         "stages_ms": stages,
     }
 
+    # The dense side of the pages' speedup comparison, after the timed region: exact attention
+    # of the same queries over the whole grown cache (no routing) against the routed decode
+    # (route + sparse attention) on the same tree, for the whole batch and for one query token.
+    if not args.no_dense:
+        def timed(fn):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.steps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / args.steps
+
+        Q1 = Q[:, :1].contiguous()
+        out1 = torch.empty(Q1.shape, dtype=torch.float32, device=dev)
+        dense_ms = timed(lambda: dec.dense_attn([K], [V], Q, out))
+        zha_ms = timed(lambda: dec.decode([K], [V], Q, args.p, out))
+        dense1_ms = timed(lambda: dec.dense_attn([K], [V], Q1, out1))
+        zha1_ms = timed(lambda: dec.decode([K], [V], Q1, args.p, out1))
+        res["dense"] = {"n_tokens": N0 + n_app, "batch_queries": n_q,
+                        "dense_ms": dense_ms, "zha_decode_ms": zha_ms, "speedup": dense_ms / zha_ms,
+                        "one_query_dense_ms": dense1_ms, "one_query_zha_decode_ms": zha1_ms,
+                        "one_query_speedup": dense1_ms / zha1_ms}
+
     # end to end through the public API with host buffers
     if not args.no_e2e:
         Kh = seq.K.pin_memory()
@@ -398,6 +426,8 @@ def main():
                               int(wl.Q.shape[2]) * wl.seqs[0].geom.Hq * (wl.seqs[0].n_tokens + wl.n_append))}
         line["stages_ms"] = res["stages_ms"]
         line["stats"] = res["stats"]
+        if "dense" in res:
+            line["dense"] = res["dense"]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.p)
         print(json.dumps(line))

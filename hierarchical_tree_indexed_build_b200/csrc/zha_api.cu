@@ -586,6 +586,38 @@ extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, co
     return ZHA_OK;
 }
 
+extern "C" zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, const void* const* V,
+                                     const void* Q, int32_t n_q, float* out, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (n_q < 1 || n_q > dec->max_q) return fail(ZHA_ERR_CAPACITY, "n_q must be in [1, max_queries]");
+    if (!K || !V || !Q || !out) return fail(ZHA_ERR_ARG, "K, V, Q and out must be non-NULL");
+    if (!aligned16(Q) || !aligned16(out)) return fail(ZHA_ERR_ARG, "Q and out must be 16-byte aligned");
+    for (int s = 0; s < dec->n_seq; ++s)
+        if (!K[s] || !V[s] || !aligned16(K[s]) || !aligned16(V[s]))
+            return fail(ZHA_ERR_ARG, "K[s] and V[s] must be 16-byte aligned device pointers");
+    zha_status s = fill_seqs(dec, K, V);
+    if (s != ZHA_OK) return s;
+    // No complete top node: no sink, no routed chunks, every token in the tail that every
+    // lane attends.  The next zha_route / zha_sparse_attn uploads the trees' own counts again.
+    for (SeqDev& sd : dec->seq_host) sd.T = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ZHA_CUDA(cudaMemcpyAsync(dec->seq_dev, dec->seq_host.data(), sizeof(SeqDev) * dec->n_seq,
+                             cudaMemcpyHostToDevice, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.ctr + kCtrUnionTokens, 0, 2 * 8, st));
+    Batch b = make_batch(dec, Q, n_q, 1.0f);
+    b.dense = 1;
+    int64_t max_splits = 0;
+    for (const SeqDev& sd : dec->seq_host) {
+        const int64_t nseg = (sd.N + sd.C - 1) / sd.C;
+        const int64_t segs = segs_per_split(b.n_gl, sd.C);
+        max_splits = std::max<int64_t>(max_splits, (nseg + segs - 1) / segs);
+    }
+    if (max_splits > dec->w.s_cap) return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
+    ZHA_CUDA(launch_attn(b, dec->w, max_splits, score_scale(dec->d), st));
+    ZHA_CUDA(launch_combine(b, dec->w, out, st));
+    return ZHA_OK;
+}
+
 extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                                  const void* Q, int32_t n_q, float p, float* out, void* stream) {
     zha_status s = zha_route(dec, Q, n_q, p, stream);

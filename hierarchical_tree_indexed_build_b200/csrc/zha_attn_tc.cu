@@ -530,8 +530,10 @@ size_t attn_tc_smem(int d) {
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
     if (max_splits <= 0) return cudaSuccess;
-    cudaError_t e = launch_member(b, w, 0, 1, st);   // lane masks of the kept level-1 chunks
-    if (e != cudaSuccess) return e;
+    if (!b.dense) {
+        const cudaError_t e = launch_member(b, w, 0, 1, st);   // lane masks of the kept level-1 chunks
+        if (e != cudaSuccess) return e;
+    }
     ProfScope ps_("k_attn_tc", st);
     const int lane_tiles = (b.n_gl + kRows - 1) / kRows;
     dim3 grid(lane_tiles, (unsigned)max_splits, b.n_groups);   // splits <= 65,535 (checked by the caller)

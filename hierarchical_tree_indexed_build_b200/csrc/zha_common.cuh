@@ -78,6 +78,7 @@ struct Batch {
     int32_t score_path;              // 0 auto, 1 CUDA cores, 2 tensor cores (R = 16 only)
     int32_t attn_path;               // 0 auto, 1 CUDA cores, 2 tensor cores
     int32_t all_r16;                 // every tree of the batch has R = 16
+    int32_t dense = 0;               // every lane attends every token (no routed sets, no lane masks)
 };
 
 // Global lane index of group lane y of group (s, g): lane = (s*n_q + i)*Hq + h.

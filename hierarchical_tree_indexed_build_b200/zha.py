@@ -25,7 +25,7 @@ _STATUS = {0: "ZHA_OK", 1: "ZHA_ERR_ARG", 2: "ZHA_ERR_CAPACITY", 3: "ZHA_ERR_CUD
 # Every function declared in include/zha.h.
 EXPORTS = ["zha_last_error", "zha_tree_create", "zha_tree_destroy", "zha_tree_info", "zha_build_tree",
            "zha_append", "zha_tree_export", "zha_decoder_create", "zha_decoder_destroy", "zha_route",
-           "zha_sparse_attn", "zha_sparse_attn_static", "zha_decode", "zha_decoder_set_kernels", "zha_decoder_export_kept", "zha_decoder_words",
+           "zha_sparse_attn", "zha_sparse_attn_static", "zha_dense_attn", "zha_decode", "zha_decoder_set_kernels", "zha_decoder_export_kept", "zha_decoder_words",
            "zha_decoder_stats", "zha_profile_enable", "zha_profile_read", "zha_profile_reset"]
 
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.zha_sparse_attn.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, _vp, _vp]
         L.zha_sparse_attn_static.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _i32,
                                              _vp, _i64, _vp, _vp]
+        L.zha_dense_attn.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, _vp, _vp]
         L.zha_decode.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, ctypes.c_float,
                                  _vp, _vp]
         L.zha_decoder_set_kernels.argtypes = [_vp, _i32, _i32]
@@ -171,6 +172,10 @@ def zha_sparse_attn(dec: int, K, V, Q: int, n_q: int, out: int, stream: int):
 def zha_sparse_attn_static(K: int, V: int, ld: int, n_tokens: int, C: int, L: int, Hq: int, Hkv: int, d: int,
                            Q: int, n_q: int, kept1: int, words: int, out: int, stream: int):
     _check(lib().zha_sparse_attn_static(K, V, ld, n_tokens, C, L, Hq, Hkv, d, Q, n_q, kept1, words, out, stream))
+
+
+def zha_dense_attn(dec: int, K, V, Q: int, n_q: int, out: int, stream: int):
+    _check(lib().zha_dense_attn(dec, K, V, Q, n_q, out, stream))
 
 
 def zha_decode(dec: int, K, V, Q: int, n_q: int, p: float, out: int, stream: int):
@@ -302,6 +307,16 @@ class Decoder:
         _need(out, torch.float32, "out")
         zha_sparse_attn(self.handle, _ptr_array(Ks), _ptr_array(Vs), Q.data_ptr(), Q.shape[1], out.data_ptr(),
                         _stream(stream))
+
+    def dense_attn(self, Ks, Vs, Q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+        """Dense exact attention of every query lane over its whole sequence (no routing)."""
+        _need(Q, torch.bfloat16, "Q")
+        if out is None:
+            out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+        _need(out, torch.float32, "out")
+        zha_dense_attn(self.handle, _ptr_array(Ks), _ptr_array(Vs), Q.data_ptr(), Q.shape[1], out.data_ptr(),
+                       _stream(stream))
+        return out
 
     def decode(self, Ks, Vs, Q: torch.Tensor, p: float, out: Optional[torch.Tensor] = None, stream=None):
         _need(Q, torch.bfloat16, "Q")

@@ -170,6 +170,19 @@ zha_status zha_sparse_attn_static(const void* K, const void* V, int64_t ld, int6
                                   const void* Q, int32_t n_q, const uint32_t* kept1, int64_t words,
                                   float* out, void* stream);
 
+/* Dense exact attention: every query lane over all n_tokens tokens of its sequence,
+ *   o = sum_t softmax_t(s q.k_t) v_t,  t in [0, N),  s = 1/sqrt(d),
+ * with no routing.  The pages measure the routed decode against dense attention over the
+ * whole cache (the speedup of their figures); this is that comparison's dense side on the
+ * same kernels: the split-KV attention (tcgen05 or CUDA cores, as zha_decoder_set_kernels
+ * selects) with every token a tail token of every lane, then the split combine.  K, V, Q
+ * and out as for zha_sparse_attn; the decoder's trees give only each sequence's token
+ * count and chunk size (the split granularity) and must be built.  Needs no zha_route and
+ * leaves the last route's kept sets as they were (a later zha_sparse_attn still attends
+ * them).  ZHA_ERR_CAPACITY if n_q exceeds the decoder's max_queries. */
+zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, const void* const* V,
+                          const void* Q, int32_t n_q, float* out, void* stream);
+
 /* zha_route followed by zha_sparse_attn. */
 zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                       const void* Q, int32_t n_q, float p, float* out, void* stream);

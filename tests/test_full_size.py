@@ -3,7 +3,8 @@
 * The 1M-token deep tree (C4 L6, R16, GQA 16/2, d128) built over 1,048,576 tokens, grown by a
   4,096-token append, then decoded for all 128 queries in one batch at p = 0.95 with the
   default kernel choice: exactly the step the benchmark times.  Sampled summaries of every
-  level, and every lane of two queries, are replayed by the oracle.
+  level, and every lane of two queries, are replayed by the oracle; so is one query's dense
+  attention over the whole grown cache (the benchmark's dense comparison).
 * The batched workload: 32 sequences x 131,072 tokens, half C16 L3 and half C4 L6, one
   appended token and one query per sequence per step; two steps, four sequences compared.
 """
@@ -12,6 +13,7 @@ import pytest
 import torch
 
 from hierarchical_tree_indexed_build_b200 import inputs, zha
+from oracle import oracle as O
 import zha_testlib as TL
 
 pytestmark = pytest.mark.gpu
@@ -44,6 +46,17 @@ def test_full_size_deep1m_benchmark_step():
     assert res.stats.status == 0
     rep, e1, e2, _ = TL.check_decode(seq, n, Q[0], 0.95, res.out[0], res.kept[0], [0, 77])
     _report("deep1m full batch", rep, e1, e2)
+    # the dense baseline of the same batch over the whole grown cache, one query's lanes
+    # replayed by the oracle over all n tokens
+    dec = zha.Decoder([tree], Q.shape[1])
+    dense = dec.dense_attn([K], [V], Q.cuda().contiguous())
+    torch.cuda.synchronize()
+    q, lane_g, ids = TL.lanes_for(seq, Q[0], [5])
+    o = O.attend_batch(TL.f64(seq.K), TL.f64(seq.V), q, lane_g, [np.arange(n)] * len(ids))
+    e = TL.rel_err(dense.cpu().numpy().astype(np.float64).reshape(-1, g.d)[ids], o)
+    print("[deep1m dense] max rel err %.2e" % e.max())
+    assert e.max() <= TL.OUT_TOL
+    dec.close()
     tree.close()
 
 

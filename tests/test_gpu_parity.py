@@ -324,3 +324,62 @@ def test_tensor_core_and_cuda_core_attention_agree(n_q, p):
     assert e <= 1e-4
     rep, e1, e2, _ = TL.check_decode(seq, n, Q[0], p, b.out[0], b.kept[0], list(range(min(n_q, 3))))
     _report("attn tensor n_q=%d p=%g" % (n_q, p), rep, e1, e2)
+
+
+# ----------------------------------------------------------------------------- dense baseline
+
+@needs_cuda
+@pytest.mark.parametrize("geom,n_tokens,n_q,attn", [
+    (inputs.TINY, 4096 + 77, 16, zha.ZHA_KERNELS_AUTO),      # 16 lanes: CUDA-core split-KV
+    (inputs.DEEP, 3 * 4096 + 1234, 8, zha.ZHA_KERNELS_AUTO),  # 64 lanes per group: tcgen05
+    (inputs.DEEP, 3 * 4096 + 1234, 8, zha.ZHA_KERNELS_SIMT),
+    (inputs.MID, 2 * 4096 + 700, 3, zha.ZHA_KERNELS_TENSOR),  # 24 lanes: a ragged lane tile on tcgen05
+])
+def test_dense_attention_matches_oracle(geom, n_tokens, n_q, attn):
+    """zha_dense_attn is exact softmax attention of every lane over all N tokens: the
+    oracle's attention over the whole token range (pinned to float64 SDPA)."""
+    seq = inputs.make_sequence(geom, n_tokens, n_tokens, seed=21)
+    tree, K, V, qr = TL.make_tree(seq)
+    rng = np.random.default_rng(3)
+    Q = torch.from_numpy(rng.standard_normal((1, n_q, geom.Hq, geom.d), dtype=np.float32)).to(torch.bfloat16)
+    dec = zha.Decoder([tree], n_q)
+    dec.set_kernels(zha.ZHA_KERNELS_AUTO, attn)
+    out = dec.dense_attn([K], [V], Q.cuda().contiguous())
+    torch.cuda.synchronize()
+    q, lane_g, ids = TL.lanes_for(seq, Q[0], range(n_q))
+    o = O.attend_batch(TL.f64(seq.K), TL.f64(seq.V), q, lane_g, [np.arange(n_tokens)] * len(ids))
+    e = TL.rel_err(out.cpu().numpy().astype(np.float64).reshape(-1, geom.d)[ids], o)
+    print("[dense %s N=%d n_q=%d attn=%d] max rel err %.2e" % (geom, n_tokens, n_q, attn, e.max()))
+    assert e.max() <= TL.OUT_TOL
+    dec.close()
+    tree.close()
+
+
+@needs_cuda
+def test_dense_attention_equals_routed_decode_at_p1():
+    """At p = 1 every frontier node is kept at every level, so the routed set is every token
+    and the routed decode computes dense attention (in another summation order); a dense
+    call between a route and its sparse attention leaves the route's kept sets in place."""
+    geom, n_tokens, n_q = inputs.DEEP, 3 * 4096 + 1234, 8
+    seq = inputs.make_sequence(geom, n_tokens, n_tokens, seed=22)
+    tree, K, V, qr = TL.make_tree(seq)
+    rng = np.random.default_rng(4)
+    Q = torch.from_numpy(rng.standard_normal((1, n_q, geom.Hq, geom.d), dtype=np.float32)).to(torch.bfloat16).cuda()
+    dec = zha.Decoder([tree], n_q)
+    routed = dec.decode([K], [V], Q, 1.0)
+    dense = dec.dense_attn([K], [V], Q)
+    torch.cuda.synchronize()
+    e = TL.rel_err(dense.cpu().numpy().astype(np.float64).reshape(-1, geom.d),
+                   routed.cpu().numpy().astype(np.float64).reshape(-1, geom.d))
+    print("[dense vs routed p=1] max rel diff %.2e" % e.max())
+    assert e.max() <= 1e-4
+    dec.route(Q, 0.9)
+    dense2 = dec.dense_attn([K], [V], Q)
+    sparse = torch.empty_like(dense2)
+    dec.sparse_attn([K], [V], Q, sparse)
+    again = dec.decode([K], [V], Q, 0.9)
+    torch.cuda.synchronize()
+    assert torch.equal(dense, dense2)
+    assert torch.equal(sparse, again)
+    dec.close()
+    tree.close()
