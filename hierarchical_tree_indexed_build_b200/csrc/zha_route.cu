@@ -289,6 +289,117 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
     }
 }
 
+// Scorer for groups of at most kFewLanes lanes with R = 16 (one or two query tokens): one
+// warp per candidate node reads the node's whole record at once - thread t holds half of
+// plane row r = t / 2 (dims (t % 2) D/2 ..), D/16 16-byte loads per fp16 plane, all issued
+// together, so a node costs one DRAM round trip - decodes m = hi + lo once and scores every
+// lane of the group from it (the lanes' query rows in shared memory).  The same estimate as
+// k_score: e = max_r (s q.m_r + b_r), -inf off the lane's frontier, in candidate order.
+constexpr int kFewLanes = 16;
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, float scale) {
+    constexpr int kHalf = D / 2;      // dims per thread
+    constexpr int kV = kHalf / 8;     // 16-byte pieces per plane per thread
+    constexpr int kRow = kHalf + 4;   // shared row stride of a query half (the two halves of a
+                                      // row fall in different banks)
+    __shared__ __align__(16) float sqy[kFewLanes][2][kRow];
+    const int grp = blockIdx.z;
+    const int s = grp / b.Hkv, g = grp % b.Hkv;
+    const SeqDev& sq = b.seqs[s];
+    const int lev = sq.L - it;
+    if (lev < 1) return;
+    const bool top = (lev == sq.L);
+    const int C = sq.C;
+    const int64_t nc = top ? sq.T : (int64_t)w.ucount[grp] * C;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
+        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+    }
+    if (nc == 0) return;
+    const int nl = b.n_gl;            // <= kFewLanes (checked by the launcher)
+    for (int i = threadIdx.x; i < nl * D; i += blockDim.x) {
+        const int y = i / D, k = i - y * D;
+        sqy[y][k / kHalf][k % kHalf] = __bfloat162float(b.Q[lane_of(b, s, g, y) * D + k]);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 1, hf = lane & 1;
+    const int R = sq.R;               // 16
+    const int64_t ns = sq.ns;
+    const float* base = sq.rec[lev] + (int64_t)g * sq.cap[lev] * ns;
+    const int32_t* ul = w.ulist + (int64_t)grp * w.us;
+    // lane y = this thread's lane (threads 0 .. nl-1): its frontier test and statistics
+    const int64_t xm = lane_of(b, s, g, lane < nl ? lane : 0);
+    const uint32_t* Pb = top ? nullptr : w.kept[lev + 1] + xm * w.W[lev + 1];
+    float* ex = w.e + xm * w.es;
+    float fmax = -INFINITY;
+    int fcnt = 0;
+    const int64_t wstep = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t k = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; k < nc; k += wstep) {
+        const int64_t j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
+        const float* rec = base + j * ns;
+        const __half* rh = reinterpret_cast<const __half*>(rec);
+        const uint4* hp = reinterpret_cast<const uint4*>(rh + (int64_t)r * D + hf * kHalf);
+        const uint4* lp = reinterpret_cast<const uint4*>(rh + (int64_t)R * D + (int64_t)r * D + hf * kHalf);
+        uint4 hv[kV], lv[kV];
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            hv[v] = __ldg(hp + v);
+            lv[v] = __ldg(lp + v);
+        }
+        const float br = __ldg(rec + (int64_t)R * D + r);
+        float m[kHalf];
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const uint32_t hw[4] = {hv[v].x, hv[v].y, hv[v].z, hv[v].w};
+            const uint32_t lw[4] = {lv[v].x, lv[v].y, lv[v].z, lv[v].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float2 f = m_decode2(hw[c], lw[c]);
+                m[8 * v + 2 * c] = f.x;
+                m[8 * v + 2 * c + 1] = f.y;
+            }
+        }
+        float mine = -INFINITY;
+#pragma unroll 1
+        for (int y = 0; y < nl; ++y) {
+            const float4* q4 = reinterpret_cast<const float4*>(sqy[y][hf]);
+            float d0 = 0.0f, d1 = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kHalf / 4; ++i) {
+                const float4 qv = q4[i];
+                d0 = fmaf(qv.x, m[4 * i], d0);
+                d1 = fmaf(qv.y, m[4 * i + 1], d1);
+                d0 = fmaf(qv.z, m[4 * i + 2], d0);
+                d1 = fmaf(qv.w, m[4 * i + 3], d1);
+            }
+            float dot = d0 + d1;
+            dot += __shfl_xor_sync(kFull, dot, 1);            // the row's two halves
+            float e = fmaf(scale, dot, br);
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) e = fmaxf(e, __shfl_xor_sync(kFull, e, o));   // max over r
+            if (lane == y) mine = e;
+        }
+        if (lane < nl) {
+            bool mb = true;
+            if (!top) {
+                const int64_t pj = j / C;
+                mb = (__ldg(Pb + (pj >> 5)) >> (pj & 31)) & 1u;
+            }
+            ex[k] = mb ? mine : -INFINITY;   // candidate order
+            if (mb) {
+                fmax = fmaxf(fmax, mine);
+                ++fcnt;
+            }
+        }
+    }
+    if (lane < nl && fcnt > 0) {
+        atomicMax(w.lane_max + (int64_t)lev * w.lanes_cap + xm, ord_bits(fmax));
+        atomicAdd(w.lane_cnt + (int64_t)lev * w.lanes_cap + xm, fcnt);
+    }
+}
+
 // ----------------------------------------------------------------------------- select
 
 constexpr int kSelThreads = 512;
@@ -781,6 +892,16 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
     const bool tc = b.all_r16 && w.tmaps &&
                     (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
     if (tc) return launch_score_tc(b, w, it, scale, st);
+    if (b.all_r16 && b.n_gl <= kFewLanes) {
+        // one wave: 2 blocks of 8 warps per SM, shared by the groups
+        const int bx = std::max(1, 2 * 148 / std::max(1, b.n_groups));
+        ProfScope ps_("k_score", st);
+        if (b.d == 128)
+            k_score_few<128><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        else
+            k_score_few<64><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        return cudaGetLastError();
+    }
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
     dim3 grid(score_blocks_x(lane_blocks, b.n_groups), lane_blocks, b.n_groups);
