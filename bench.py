@@ -165,6 +165,21 @@ def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
     return 0.0, 0.0
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's); x itself on one
+    rank.  Every rank must call it at the same point."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank per step."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, rank, world, dev):
     from hierarchical_tree_indexed_build_b200 import zha
     torch.cuda.set_device(dev)
@@ -214,12 +229,9 @@ def run_ours(args, rank, world, dev):
     ms = e0.elapsed_time(e1)
     prof = zha.zha_profile_read()
     st = dec.stats()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
-    value = world * n_q / (ms_step / 1e3)
+    value = whole_job_rate(world, n_q, ms_step)
 
     # dominant kernel and its roofline
     n_lanes = n_q * g.Hq
@@ -321,12 +333,9 @@ def run_ours(args, rank, world, dev):
         e1.record(stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(ems, world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (Kh, Vh, qh, Qh))
-        res["e2e"] = {"value": world * n_q / (ems / args.steps / 1e3), "unit": "queries/s",
+        res["e2e"] = {"value": whole_job_rate(world, n_q, ems / args.steps), "unit": "queries/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outh.numel() * 4}
     res["wl"] = wl
     return res
