@@ -67,6 +67,7 @@ def test_null_handles_are_rejected(libzha):
     assert libzha.zha_decoder_create(None, 0, 1, ctypes.byref(h)) == zha.ZHA_ERR_ARG
     assert libzha.zha_route(None, None, 1, 0.9, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_sparse_attn(None, None, None, None, 1, None, None) == zha.ZHA_ERR_ARG
+    assert libzha.zha_dense_attn(None, None, None, None, 1, None, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_decoder_export_kept(None, 1, None, None, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_decoder_words(None, 1) == 0
     assert libzha.zha_decoder_stats(None, None, None) == zha.ZHA_ERR_ARG
