@@ -8,7 +8,12 @@ One step = the whole hot path over one batch of the 1M-token deep-tree workload:
 value = decoded queries per second of device time (max over ranks, summed over ranks).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun every rank runs an independent replica (no data-path collective).
+                  [--p P] [--workload deep1m|deep256k|deep64k|wide256k] [--n-q N]
+                  [--no-e2e] [--no-cpu-baseline] [--no-dense]
+Under torchrun every rank runs an independent replica (no data-path collective).  After the
+timed region the line also carries the end-to-end rate with host buffers (e2e), the dense
+comparison (dense: zha_dense_attn against the routed decode, the batch and one query token)
+and, on rank 0 at N = 1, the oracle timed on the host cores (cpu_baseline).
 """
 from __future__ import annotations
 
