@@ -71,17 +71,27 @@ KERNEL_SOURCES = {
 }
 
 
+def source_code_sha256(text: str) -> str:
+    """SHA-256 of a C/CUDA source with its comments and blank lines removed, so a traffic
+    record stays valid across comment edits but not across code changes."""
+    import hashlib
+    import re
+    t = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    t = re.sub(r"//[^\n]*", "", t)
+    lines = [l.rstrip() for l in t.splitlines() if l.strip()]
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def measured_traffic(name, workload):
     """DRAM bytes (read + write) per launch of `name` from profiles/traffic.txt, written from
-    an ncu capture of this workload (JSON text); None when absent or when the kernel's source has changed
-    since (the record stores the source's SHA-256)."""
-    import hashlib
+    an ncu capture of this workload (JSON text); None when absent or when the kernel's source
+    code has changed since (the record stores source_code_sha256 of the capture-time source)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
             rec = json.load(f)[workload][name]
         src = os.path.join(ROOT, "hierarchical_tree_indexed_build_b200", "csrc", KERNEL_SOURCES[name])
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+        with open(src, encoding="utf-8") as f:
+            if source_code_sha256(f.read()) != rec["source_code_sha256"]:
                 return None
         return float(rec["bytes_per_launch"])
     except (OSError, KeyError, ValueError):

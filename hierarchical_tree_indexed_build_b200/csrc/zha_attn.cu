@@ -1,8 +1,8 @@
 // zha_attn.cu - exact attention over the routed token set (split-KV flash-decode).
 //
 // What is computed (pages: fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的 —
-// 只对少量保留下来的原始 KV 条目做精确注意力; wqu.guru, section "How does top-p routing pick
-// tokens?" — the first token is always kept as an attention sink): for lane x,
+// exact attention only over the raw rows that routing kept; wqu.guru, section "How does top-p
+// routing pick tokens?" — token 0 attended as a sink every time): for lane x,
 //     A_x = {0} U {tokens of the level-1 chunks kept by x} U [T C^L, N)
 //     o_x = sum_{t in A_x} exp(s q.k_t - M) v_t / sum_{t in A_x} exp(s q.k_t - M).
 //

@@ -1,8 +1,8 @@
 // zha_attn_tc.cu - exact attention over the routed token set on the tcgen05 tensor cores.
 //
 // Same result as k_attn (fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的 —
-// 只对少量保留下来的原始 KV 条目做精确注意力; wqu.guru, section "How does top-p routing pick
-// tokens?" — token 0 is always attended): for every lane x of a (sequence, KV head) group,
+// exact attention only over the raw rows that routing kept; wqu.guru, section "How does top-p
+// routing pick tokens?" — token 0 is always attended): for every lane x of a (sequence, KV head) group,
 //     o_x = sum_{t in A_x} exp(s q.k_t - M) v_t / sum_{t in A_x} exp(s q.k_t - M),
 // A_x = {0} U tokens of the level-1 chunks x kept U tail.  Used when a group holds many
 // lanes, so that a tile of 128 lanes x 128 token positions is a dense contraction:

@@ -1,8 +1,8 @@
 // zha_route.cu - top-down top-p routing kernels.
 //
 // What is computed (pages: fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的 —
-// 先给顶层节点打分，保留覆盖估计注意力质量比例 p 的最小节点集合，再逐层展开; wqu.guru, section
-// "How does top-p routing pick tokens?"): for every lane (query token, query head h, KV head
+// score the top level, keep the fewest nodes whose estimated mass reaches the fraction p, then
+// descend one level at a time; wqu.guru, section "How does top-p routing pick tokens?"): for every lane (query token, query head h, KV head
 // g = h*Hkv/Hq) and level l from L down to 1, each frontier node j gets the plane estimate
 //     e_j = max_r ( s q.m_r(j) + b_r(j) ),
 // the frontier's softmax masses P_j = exp(e_j - max e) / sum exp(e - max e) are ordered by

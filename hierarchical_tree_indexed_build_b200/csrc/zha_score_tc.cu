@@ -1,7 +1,7 @@
 // zha_score_tc.cu - plane-estimate scoring on the 5th-generation tensor cores (tcgen05).
 //
 // Same quantity as k_score (fluxbbs.com "Zyphra ZHA 稀疏注意力…", section 树形索引是怎么搭的:
-// 取这些平面的最大值; wqu.guru, section "Building the tree"): for every lane of a
+// the estimate is the largest of the planes; wqu.guru, section "Building the tree"): for every lane of a
 // (sequence, KV head) group and every candidate node j on the lane's frontier,
 //     e_j = max_r ( s q.m_r(j) + b_r(j) ),
 // and -inf for candidates off the lane's frontier (children of nodes other lanes kept).

@@ -9,16 +9,17 @@
  *    tokens; for each of R reference queries q_r a chunk is summarised by the tangent
  *    plane of its log attention mass at q_r: lse_r = log sum_t exp(s q_r.k_t) and slope
  *    m_r = softmax-weighted mean of the keys (s = 1/sqrt(d)); b_r = lse_r - s q_r.m_r.
- *    Summaries are compressed again level by level: a level-l node covers C^l tokens;
+ *    Summaries are merged upward one level at a time: a level-l node covers C^l tokens;
  *    this library merges the C children's (lse_r, m_r) with the online-softmax combine,
  *    which equals the summary of the C^l raw tokens.
- *  - Routing: fluxbbs section "树形索引是怎么搭的" (解码时的路由是自顶向下的); wqu.guru
- *    section "How does top-p routing pick tokens?".  Per query head, the complete
+ *  - Routing: fluxbbs section "树形索引是怎么搭的"; wqu.guru section "How does top-p
+ *    routing pick tokens?".  Per query head, the complete
  *    top-level nodes are scored by max_r (s q.m_r + b_r); at each level the smallest
  *    (score desc, index asc) prefix of the candidates whose softmax mass over the
  *    candidates reaches p is kept, and only the kept nodes' children are scored next.
- *  - Sparse attention: fluxbbs (只对少量保留下来的原始 KV 条目做精确注意力), wqu.guru
- *    ("The first token is always kept as an attention sink").  Exact softmax attention
+ *  - Sparse attention: fluxbbs section "树形索引是怎么搭的" (exact attention over the raw
+ *    rows routing keeps), wqu.guru section "How does top-p routing pick tokens?" (token 0
+ *    attended as a sink every time).  Exact softmax attention
  *    over token 0, the tokens of the kept level-1 chunks and the tail of tokens after the
  *    last complete top node.
  *

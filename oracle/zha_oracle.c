@@ -47,8 +47,8 @@ int zo_num_threads(void) { return omp_get_max_threads(); }
 
 /*
  * Summary of the node made of tokens [t0, t1) of one KV head, for each reference
- * query q_r ([fluxbbs] 树形索引是怎么搭的: each reference query gives a tangent-plane
- * estimate of the chunk's attention mass; [wqu] Building the tree):
+ * query q_r (fluxbbs.com, section 树形索引是怎么搭的, and wqu.guru, section Building the
+ * tree: every reference query yields a tangent plane of the chunk's log attention mass):
  *   a_t   = s (q_r . k_t)
  *   lse_r = log sum_t exp(a_t)                       (computed max-shifted)
  *   m_r   = sum_t exp(a_t - lse_r) k_t               (softmax-weighted mean of keys)
@@ -112,7 +112,8 @@ void zo_summaries(const double* K, int d, const double* qref, int R, int64_t spa
 /*
  * Plane estimate of a node's log attention mass for query q: the maximum over the
  * R tangent planes, est = max_r [ s (q . m_r) + b_r ]
- * ([fluxbbs] 取这些平面的最大值; [wqu] "The max over these planes approximates ...").
+ * (fluxbbs.com, section 树形索引是怎么搭的, and wqu.guru, section Building the tree: the
+ * estimate is the largest of the R planes).
  */
 double zo_plane_estimate(const double* m, const double* b, int R, int d, const double* q)
 {
@@ -159,8 +160,9 @@ static int cand_cmp(const void* pa, const void* pb)
 }
 
 /*
- * Top-p cut over n candidates ([fluxbbs] 保留覆盖估计注意力质量比例 p 的最小节点集合;
- * [wqu] "keeps the smallest set holding a fraction p of estimated attention mass").
+ * Top-p cut over n candidates (fluxbbs.com, section 树形索引是怎么搭的, and wqu.guru,
+ * section How does top-p routing pick tokens?: the kept nodes are the fewest whose
+ * estimated mass together reaches the fraction p).
  * P_i = exp(e_i - max e) / sum_j exp(e_j - max e) over the candidates; order by
  * (e desc, idx asc); k* = min{k >= 1 : sum_{t<k} P_(t) >= p}; p >= 1 keeps all.
  * keep[i] is set for kept candidates (positions as given).  Returns k*.
@@ -208,9 +210,9 @@ int64_t zo_topp(const double* e, const int64_t* idx, int64_t n, double p, uint8_
 
 /*
  * Top-down routing of n_lanes (query, head) lanes through the tree of one sequence
- * ([fluxbbs] 解码时的路由是自顶向下的: score the top-level nodes, keep the smallest set
- * holding fraction p, expand level by level down to the raw KV entries; [wqu] "It then
- * expands only those children, repeating until it reaches raw KV entries").
+ * (fluxbbs.com, section 树形索引是怎么搭的, and wqu.guru, section How does top-p routing
+ * pick tokens?: routing starts at the top level, cuts each level at mass p and descends
+ * only into the kept nodes' children, down to level 1).
  *
  * K: [Hkv][ld][d] keys (rows t < N used); qref: [Hkv][R][d]; q: [n_lanes][d];
  * lane_g[x]: KV head of lane x.  Level l (1..L) has n_l = N / C^l nodes; the frontier
@@ -308,8 +310,9 @@ void zo_route(const double* K, int64_t ld, int64_t N, int Hkv, int d,
 }
 
 /*
- * Attended token set of one lane ([fluxbbs] 只对少量保留下来的原始 KV 条目做精确注意力;
- * [wqu] "The first token is always kept as an attention sink"):
+ * Attended token set of one lane (fluxbbs.com, section 树形索引是怎么搭的: exact attention
+ * runs only over the raw rows the routing kept; wqu.guru, section How does top-p routing
+ * pick tokens?: token 0 is attended as a sink in every case):
  *   A = {0} U {jC .. jC+C-1 : j kept at level 1} U [T C^L, N),  T = N / C^L;
  * with T = 0 (no complete top node) A = [0, N).  kept1: [N / C].
  * Writes the sorted token list (capacity N) and returns |A|.
@@ -337,8 +340,9 @@ int64_t zo_attended_set(const uint8_t* kept1, int64_t N, int C, int L, int64_t* 
 }
 
 /*
- * Exact softmax attention over a token set ([fluxbbs] 精确注意力; [wqu] What is ZHA:
- * "The tree only decides which cached keys each query reads"):
+ * Exact softmax attention over a token set (fluxbbs.com, section 树形索引是怎么搭的;
+ * wqu.guru, section What is Zyphra Hierarchical Attention (ZHA)?: the tree only chooses
+ * the keys, the attention over them is ordinary softmax attention):
  *   o = sum_{t in A} exp(s q.k_t - M) v_t / sum_{t in A} exp(s q.k_t - M),  M = max.
  * K, V: [*][d] rows of one head.
  */

@@ -78,3 +78,11 @@ def test_reference_arm_prints_one_line_with_the_contract_keys():
     assert line["e2e"] == {"value": line["value"], "unit": "queries/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == "deep_64k_C4L6"
+
+
+def test_traffic_record_hash_ignores_comments_not_code():
+    a = "int f(int x) {\n    return x + 1;   // one more\n}\n"
+    b = "/* header\n   comment */\nint f(int x) {\n\n    return x + 1;\n}\n"
+    c = "int f(int x) {\n    return x + 2;\n}\n"
+    assert bench.source_code_sha256(a) == bench.source_code_sha256(b)
+    assert bench.source_code_sha256(a) != bench.source_code_sha256(c)
