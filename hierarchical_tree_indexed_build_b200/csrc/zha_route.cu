@@ -892,14 +892,12 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
     const bool tc = b.all_r16 && w.tmaps &&
                     (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
     if (tc) return launch_score_tc(b, w, it, scale, st);
-    if (b.all_r16 && b.n_gl <= kFewLanes) {
-        // one wave: 2 blocks of 8 warps per SM, shared by the groups
+    if (b.all_r16 && b.n_gl <= kFewLanes && b.d == 128) {
+        // one wave: 2 blocks of 8 warps per SM, shared by the groups (d = 128, the geometry
+        // the few-lane kernel is validated on; d = 64 takes k_score)
         const int bx = std::max(1, 2 * 148 / std::max(1, b.n_groups));
         ProfScope ps_("k_score", st);
-        if (b.d == 128)
-            k_score_few<128><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
-        else
-            k_score_few<64><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        k_score_few<128><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
         return cudaGetLastError();
     }
     const int WB = min(8, (b.n_gl + 7) / 8);
