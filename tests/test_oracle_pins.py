@@ -171,6 +171,32 @@ def test_topp_worked_example():
     assert sorted(idx[perm][keep].tolist()) == [10, 11, 12]
 
 
+def test_topp_worked_example_margins():
+    """The decision margins the parity tests use to excuse a near-tie, worked by hand on the
+    masses 1/2, 1/4, 1/8, 1/8 (sorted order 10, 11, 12, 13; cumulative 1/2, 3/4, 7/8, 1):
+      p = 0.7: k* = 2, cum_2 - p = 0.05, p - cum_1 = 0.2, P_(2) - P_(3) = 1/4 - 1/8,
+               e_(2) - e_(3) = ln 2 - ln 1;
+      p = 0.8: k* = 3, cum_3 - p = 0.075, p - cum_2 = 0.05, and the last kept and the first
+               dropped node tie (both 1/8), so the last two margins are 0;
+      p = 0.9: k* = 4 = n, cum_4 - p = 0.1, p - cum_3 = 0.025, no dropped node (+inf);
+      p = 1:   every node kept without a cut: every margin +inf."""
+    e = np.log([4.0, 2.0, 1.0, 1.0])
+    idx = np.array([10, 11, 12, 13])
+    inf = math.inf
+    for p, want in [(0.7, (0.05, 0.2, 0.125, math.log(2.0))), (0.8, (0.075, 0.05, 0.0, 0.0)),
+                    (0.9, (0.1, 0.025, inf, inf)), (1.0, (inf, inf, inf, inf))]:
+        _, _, info = O.topp(e, idx, p)
+        for got, w in zip(info, want):
+            if w == inf:
+                assert got == inf, (p, info)
+            else:
+                assert got == pytest.approx(w, abs=1e-15), (p, info)
+    # the candidates in another order: the margins describe the sorted order, not the input's
+    perm = np.array([2, 0, 3, 1])
+    _, _, info2 = O.topp(e[perm], idx[perm], 0.7)
+    np.testing.assert_allclose(info2, [0.05, 0.2, 0.125, math.log(2.0)], atol=1e-15)
+
+
 def _bf_topp(e, p):
     """Brute force: the smallest k such that some k-subset holds mass >= p; returns k and a
     k-subset of maximal mass.  Up to 14 candidates every subset is enumerated; above that
@@ -195,6 +221,17 @@ def _bf_topp(e, p):
     return n, tuple(range(n)), 1.0
 
 
+def _bf_topp_size(e, k):
+    """Brute force: the largest mass any k-subset of the candidates holds (every subset)."""
+    P = softmax(e)
+    best, arg = -1.0, None
+    for c in itertools.combinations(range(len(e)), k):
+        v = sum(P[list(c)])
+        if v > best:
+            best, arg = v, c
+    return k, arg, best
+
+
 @pytest.mark.parametrize("seed", range(12))
 def test_topp_brute_force(seed):
     rng = np.random.default_rng(seed)
@@ -212,6 +249,19 @@ def test_topp_brute_force(seed):
         perm = rng.permutation(n)
         keep2, _, _ = O.topp(e[perm], idx[perm], p)
         assert set(idx[perm][keep2].tolist()) == set(idx[keep].tolist())
+        # decision margins against brute force: the best k*-subset's mass and the best
+        # (k*-1)-subset's mass (every subset enumerated), and the masses and scores on the
+        # two sides of the cut from scipy's softmax sorted by numpy
+        _, _, prev = _bf_topp_size(e, k - 1) if k > 1 else (0, (), 0.0)
+        assert info[0] == pytest.approx(best - p, abs=1e-12)
+        assert info[1] == pytest.approx(p - prev, abs=1e-12)
+        if k < n:
+            Ps = np.sort(P)[::-1]
+            es = np.sort(e)[::-1]
+            assert info[2] == pytest.approx(Ps[k - 1] - Ps[k], abs=1e-12)
+            assert info[3] == pytest.approx(es[k - 1] - es[k], abs=1e-12)
+        else:
+            assert info[2] == math.inf and info[3] == math.inf
 
 
 def test_topp_ties_prefer_lower_index():
@@ -224,8 +274,9 @@ def test_topp_ties_prefer_lower_index():
 
 # ----------------------------------------------------------------------------- routing
 
-def _bf_route(K, qref, C, L, N, q, g, p):
-    """Independent router: scipy summaries per frontier node, brute-force top-p per level."""
+def _bf_route(K, qref, C, L, N, q, g, p, scores=None):
+    """Independent router: scipy summaries per frontier node, brute-force top-p per level.
+    With a dict ``scores``, scores[l] gets {node: plane estimate} of every frontier node."""
     d = K.shape[2]
     s = 1 / math.sqrt(d)
     front = list(range(N // C ** L))
@@ -241,6 +292,8 @@ def _bf_route(K, qref, C, L, N, q, g, p):
             bb = lse - s * np.sum(qref[g] * m, axis=1)
             e.append(np.max(s * m @ q + bb))
         e = np.array(e)
+        if scores is not None:
+            scores[l] = dict(zip(front, e.tolist()))
         k, choice, best = _bf_topp(e, p)
         sel = sorted(front[i] for i in choice)
         kept[l] = sel
@@ -259,11 +312,29 @@ def test_route_matches_brute_force(C, L, N, p, seed):
     n_lanes = 4
     q = 2.0 * rng.standard_normal((n_lanes, d))
     lane_g = np.array([0, 1, 0, 1], dtype=np.int32)
-    r = O.route(K, qref, C, L, N, q, lane_g, p)
+    r = O.route(K, qref, C, L, N, q, lane_g, p, return_scores=True)
     for x in range(n_lanes):
-        bf = _bf_route(K, qref, C, L, N, q[x], lane_g[x], p)
+        sc = {}
+        bf = _bf_route(K, qref, C, L, N, q[x], lane_g[x], p, scores=sc)
         for l in range(1, L + 1):
             assert np.flatnonzero(r.kept[l - 1][x]).tolist() == bf[l], (x, l)
+            # every frontier node's estimate at its own index; the others left untouched (NaN)
+            row = r.scores[l - 1][x]
+            front = sorted(sc[l])
+            np.testing.assert_allclose(row[front], [sc[l][j] for j in front], rtol=0, atol=1e-12)
+            off = np.setdiff1d(np.arange(row.size), front)
+            assert np.isnan(row[off]).all(), (x, l)
+            assert r.nfront[l - 1][x] == len(front)
+            # the margins of this lane's cut from the brute-force estimates: cumulative masses
+            # of the sorted softmax (scipy) on both sides of k*
+            e = np.array([sc[l][j] for j in front])
+            P = np.sort(softmax(e))[::-1]
+            k = int(r.kstar[l - 1][x])
+            cum = np.concatenate([[0.0], np.cumsum(P)])
+            info = r.info[l - 1][x]
+            if p < 1:
+                assert info[0] == pytest.approx(cum[k] - p, abs=1e-12)
+                assert info[1] == pytest.approx(p - cum[k - 1], abs=1e-12)
 
 
 def test_route_replay_with_own_sets_is_identity():
