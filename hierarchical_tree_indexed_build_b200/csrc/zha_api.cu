@@ -2,6 +2,7 @@
 // the launch sequences of tree build, append, routing and sparse attention.
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
@@ -97,6 +98,7 @@ struct zha_decoder {
     std::vector<const zha_tree*> trees;
     int32_t n_seq, max_q, Hq, Hkv, d, G, Lmax;
     int64_t lanes_cap, groups_cap;
+    int64_t part_slots;   // attention partial records: lanes x splits of one call
     Work w;
     SeqDev* seq_dev;
     std::vector<SeqDev> seq_host;
@@ -107,6 +109,12 @@ struct zha_decoder {
     int32_t score_path;
     int32_t attn_path;
     int32_t all_r16;
+    // Device status word as the host sees it: every routing / attention call ends by copying
+    // the word into pinned host memory and recording `status_ev` after the copy.
+    int32_t* status_host;
+    cudaEvent_t status_ev;
+    bool status_pending;     // a copy was enqueued and not yet looked at
+    int32_t sync;            // calls wait for their own work and report its status
 };
 
 extern "C" const char* zha_last_error(void) { return g_err.c_str(); }
@@ -365,7 +373,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
 
     Work& w = dec->w;
     memset(&w, 0, sizeof(w));
-    int64_t cap1 = 1, s_cap = 1;
+    int64_t cap1 = 1, part_slots = 1;
     for (int l = 1; l <= dec->Lmax; ++l) {
         int64_t W = 1;
         for (auto* t : dec->trees)
@@ -376,8 +384,17 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         cap1 = std::max<int64_t>(cap1, t->cap[1]);
         const int64_t top = ipow(t->g.C, t->g.L);
         const int64_t nseg_max = 1 + t->cap[1] + (std::min<int64_t>(top, t->g.capacity) + t->g.C - 1) / t->g.C;
-        const int64_t segs = segs_per_split(1, t->g.C);
-        s_cap = std::max<int64_t>(s_cap, (nseg_max + segs - 1) / segs);
+        // attention partials: the most lanes x splits any call can need.  The split size
+        // depends on the lanes per group (decoder_split_tokens), so take the largest query
+        // count of each split-size bucket (<= 16, <= 64, more lanes per group).
+        for (int bk = 0; bk < 3; ++bk) {
+            const int64_t gl_lim = bk == 0 ? 16 : (bk == 1 ? 64 : (int64_t)max_queries * dec->G);
+            const int64_t nq = std::min<int64_t>(max_queries, gl_lim / dec->G);
+            if (nq < 1) continue;
+            const int64_t segs = std::max<int64_t>(1, decoder_split_tokens((int)(nq * dec->G)) / t->g.C);
+            const int64_t lanes = (int64_t)n_seq * nq * dec->Hq;
+            part_slots = std::max<int64_t>(part_slots, lanes * ((nseg_max + segs - 1) / segs));
+        }
     }
     // union lists whose lane masks are transposed: parents of a scored level (level >= 2)
     // and the kept level-1 chunks attention gathers
@@ -386,7 +403,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.lanes_cap = dec->lanes_cap;
     w.es = (cap1 + 127) / 128 * 128;   // score rows padded to whole 128-candidate blocks
     w.us = (cap1 + 7) / 8 * 8 + 8;   // union lists: room for 16-byte-rounded bulk reads past the end
-    w.s_cap = s_cap;
+    w.s_cap = 0;   // the partials' split stride, set per call
+    dec->part_slots = part_slots;
 
     size_t off = 0;
     size_t kept_off[kMaxL + 2] = {0};
@@ -406,7 +424,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     const size_t uword_off = off;
     off += up256((size_t)dec->groups_cap * w.uw * 4);
     const size_t part_off = off;
-    off += up256((size_t)dec->lanes_cap * w.s_cap * (dec->d + 4) * 4);
+    off += up256((size_t)part_slots * (dec->d + 4) * 4);
     const size_t memb_off = off;
     off += up256((size_t)dec->groups_cap * w.ms * w.mwords * 4);
     const size_t lmax_off = off;
@@ -462,6 +480,19 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     }
     cudaMemset(w.ctr, 0, (size_t)kCtrCount * 8);
     cudaMemset(w.status, 0, 4);
+    dec->status_host = nullptr;
+    dec->status_ev = nullptr;
+    dec->status_pending = false;
+    dec->sync = 0;
+    if ((e = cudaHostAlloc(reinterpret_cast<void**>(&dec->status_host), 4, cudaHostAllocDefault)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&dec->status_ev, cudaEventDisableTiming)) != cudaSuccess) {
+        const std::string msg = std::string("decoder status mirror: ") + cudaGetErrorString(e);
+        if (dec->status_host) cudaFreeHost(dec->status_host);
+        cudaFree(dec->block);
+        delete dec;
+        return fail(ZHA_ERR_CUDA, msg);
+    }
+    *dec->status_host = 0;
     *out = dec;
     return ZHA_OK;
 }
@@ -470,7 +501,55 @@ extern "C" zha_status zha_decoder_destroy(zha_decoder* dec) {
     if (!dec) return ZHA_OK;
     cudaDeviceSynchronize();
     cudaFree(dec->block);
+    if (dec->status_ev) cudaEventDestroy(dec->status_ev);
+    if (dec->status_host) cudaFreeHost(dec->status_host);
     delete dec;
+    return ZHA_OK;
+}
+
+// Text of the device status bits for an error message.
+static std::string status_text(int32_t st) {
+    std::string t;
+    char buf[32];
+    snprintf(buf, sizeof(buf), "device status 0x%x:", (unsigned)st);
+    t = buf;
+    if (st & kStatusSelectFallbackLimit) t += " top-p select ran out of bisection steps;";
+    if (st & kStatusCapacity) t += " a union list reached its capacity;";
+    if (st & kStatusTimeout) t += " a tensor-core pipeline wait gave up;";
+    if (st & kStatusRange) t += " an input or summary outside the fp16 range reached the tensor-core scorer;";
+    return t;
+}
+
+// Start of a routing / attention call: a completed earlier call whose status word was not
+// 0 is reported now (once), and nothing of this call is enqueued.
+static zha_status check_previous(zha_decoder* dec) {
+    if (!dec->status_pending) return ZHA_OK;
+    const cudaError_t before = cudaPeekAtLastError();
+    const cudaError_t q = cudaEventQuery(dec->status_ev);
+    if (q == cudaErrorNotReady) {
+        // "not ready" is not a failure: if the query left it as the thread's last error,
+        // clear it (and nothing that was there before)
+        if (before == cudaSuccess && cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();
+        return ZHA_OK;              // still running: a later call (or zha_decoder_stats) reports it
+    }
+    dec->status_pending = false;
+    if (q != cudaSuccess) return fail(ZHA_ERR_CUDA, std::string("cudaEventQuery: ") + cudaGetErrorString(q));
+    const int32_t st = *dec->status_host;
+    if (st) return fail(ZHA_ERR_DEVICE, "an earlier call on this decoder finished with " + status_text(st));
+    return ZHA_OK;
+}
+
+// End of a routing / attention call: the status word is copied to the host mirror behind
+// the call's kernels.  In synchronous mode the call waits for it and reports it.
+static zha_status finish_call(zha_decoder* dec, cudaStream_t st) {
+    ZHA_CUDA(cudaMemcpyAsync(dec->status_host, dec->w.status, 4, cudaMemcpyDeviceToHost, st));
+    ZHA_CUDA(cudaEventRecord(dec->status_ev, st));
+    dec->status_pending = true;
+    if (!dec->sync) return ZHA_OK;
+    ZHA_CUDA(cudaEventSynchronize(dec->status_ev));
+    dec->status_pending = false;
+    const int32_t s = *dec->status_host;
+    if (s) return fail(ZHA_ERR_DEVICE, status_text(s));
     return ZHA_OK;
 }
 
@@ -518,11 +597,11 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     b.score_path = dec->score_path;
     b.attn_path = dec->attn_path;
     b.all_r16 = dec->all_r16;
+    b.split_tok = decoder_split_tokens(b.n_gl);
     return b;
 }
 
-extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
-    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+static zha_status route_impl(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
     if (!Q || !aligned16(Q)) return fail(ZHA_ERR_ARG, "Q must be a 16-byte aligned device pointer");
     if (n_q < 1 || n_q > dec->max_q) return fail(ZHA_ERR_CAPACITY, "n_q must be in [1, max_queries]");
     if (!(p > 0.0f) || isnan(p)) return fail(ZHA_ERR_ARG, "p must be > 0");
@@ -557,9 +636,17 @@ extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, fl
     return ZHA_OK;
 }
 
-extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
-                                      const void* Q, int32_t n_q, float* out, void* stream) {
+extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    zha_status s = check_previous(dec);
+    if (s != ZHA_OK) return s;
+    s = route_impl(dec, Q, n_q, p, stream);
+    if (s != ZHA_OK) return s;
+    return finish_call(dec, static_cast<cudaStream_t>(stream));
+}
+
+static zha_status sparse_attn_impl(zha_decoder* dec, const void* const* K, const void* const* V,
+                                   const void* Q, int32_t n_q, float* out, void* stream) {
     if (!dec->routed || n_q != dec->last_n_q) return fail(ZHA_ERR_STATE, "zha_sparse_attn needs a zha_route with the same n_q first");
     if (!K || !V || !Q || !out) return fail(ZHA_ERR_ARG, "K, V, Q and out must be non-NULL");
     if (!aligned16(Q) || !aligned16(out)) return fail(ZHA_ERR_ARG, "Q and out must be 16-byte aligned");
@@ -576,19 +663,36 @@ extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, co
     int64_t max_splits = 0;
     for (const SeqDev& sd : dec->seq_host) {
         const int64_t nseg = 1 + sd.n[1] + (std::min<int64_t>(sd.top, sd.N) + sd.C - 1) / sd.C;
-        const int64_t segs = segs_per_split(b.n_gl, sd.C);
+        const int64_t segs = batch_segs(b, sd.C);
         max_splits = std::max<int64_t>(max_splits, (nseg + segs - 1) / segs);
     }
-    if (max_splits > dec->w.s_cap) return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
-    ZHA_CUDA(launch_union(b, dec->w, 0, 1, st));
-    ZHA_CUDA(launch_attn(b, dec->w, max_splits, score_scale(dec->d), st));
-    ZHA_CUDA(launch_combine(b, dec->w, out, st));
+    if ((int64_t)b.n_lanes * max_splits > dec->part_slots)
+        return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
+    Work wc = dec->w;
+    wc.s_cap = max_splits;   // partial record of (lane x, split) at x * max_splits + split
+    ZHA_CUDA(launch_union(b, wc, 0, 1, st));
+    ZHA_CUDA(launch_attn(b, wc, max_splits, score_scale(dec->d), st));
+    ZHA_CUDA(launch_combine(b, wc, out, st));
     return ZHA_OK;
+}
+
+extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
+                                      const void* Q, int32_t n_q, float* out, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    zha_status s = check_previous(dec);
+    if (s != ZHA_OK) return s;
+    s = sparse_attn_impl(dec, K, V, Q, n_q, out, stream);
+    if (s != ZHA_OK) return s;
+    return finish_call(dec, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, const void* const* V,
                                      const void* Q, int32_t n_q, float* out, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    {
+        const zha_status s0 = check_previous(dec);
+        if (s0 != ZHA_OK) return s0;
+    }
     if (n_q < 1 || n_q > dec->max_q) return fail(ZHA_ERR_CAPACITY, "n_q must be in [1, max_queries]");
     if (!K || !V || !Q || !out) return fail(ZHA_ERR_ARG, "K, V, Q and out must be non-NULL");
     if (!aligned16(Q) || !aligned16(out)) return fail(ZHA_ERR_ARG, "Q and out must be 16-byte aligned");
@@ -604,25 +708,40 @@ extern "C" zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, con
     ZHA_CUDA(cudaMemcpyAsync(dec->seq_dev, dec->seq_host.data(), sizeof(SeqDev) * dec->n_seq,
                              cudaMemcpyHostToDevice, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.ctr + kCtrUnionTokens, 0, 2 * 8, st));
+    ZHA_CUDA(cudaMemsetAsync(dec->w.status, 0, 4, st));
     Batch b = make_batch(dec, Q, n_q, 1.0f);
     b.dense = 1;
     int64_t max_splits = 0;
     for (const SeqDev& sd : dec->seq_host) {
         const int64_t nseg = (sd.N + sd.C - 1) / sd.C;
-        const int64_t segs = segs_per_split(b.n_gl, sd.C);
+        const int64_t segs = batch_segs(b, sd.C);
         max_splits = std::max<int64_t>(max_splits, (nseg + segs - 1) / segs);
     }
-    if (max_splits > dec->w.s_cap) return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
-    ZHA_CUDA(launch_attn(b, dec->w, max_splits, score_scale(dec->d), st));
-    ZHA_CUDA(launch_combine(b, dec->w, out, st));
-    return ZHA_OK;
+    if ((int64_t)b.n_lanes * max_splits > dec->part_slots)
+        return fail(ZHA_ERR_CAPACITY, "attention splits exceed workspace");
+    Work wc = dec->w;
+    wc.s_cap = max_splits;
+    ZHA_CUDA(launch_attn(b, wc, max_splits, score_scale(dec->d), st));
+    ZHA_CUDA(launch_combine(b, wc, out, st));
+    return finish_call(dec, st);
 }
 
 extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                                  const void* Q, int32_t n_q, float p, float* out, void* stream) {
-    zha_status s = zha_route(dec, Q, n_q, p, stream);
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    zha_status s = check_previous(dec);
     if (s != ZHA_OK) return s;
-    return zha_sparse_attn(dec, K, V, Q, n_q, out, stream);
+    s = route_impl(dec, Q, n_q, p, stream);
+    if (s != ZHA_OK) return s;
+    s = sparse_attn_impl(dec, K, V, Q, n_q, out, stream);
+    if (s != ZHA_OK) return s;
+    return finish_call(dec, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" zha_status zha_decoder_set_sync(zha_decoder* dec, int32_t on) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    dec->sync = on ? 1 : 0;
+    return ZHA_OK;
 }
 
 extern "C" zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, int32_t attn) {
@@ -675,6 +794,8 @@ extern "C" zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats
     ZHA_CUDA(cudaMemcpyAsync(ctr, dec->w.ctr, sizeof(ctr), cudaMemcpyDeviceToHost, st));
     ZHA_CUDA(cudaMemcpyAsync(&status, dec->w.status, 4, cudaMemcpyDeviceToHost, st));
     ZHA_CUDA(cudaStreamSynchronize(st));
+    if (dec->status_pending && cudaEventQuery(dec->status_ev) == cudaSuccess)
+        const_cast<zha_decoder*>(dec)->status_pending = false;   // reported here instead
     memset(out, 0, sizeof(*out));
     for (int l = 1; l <= kMaxL; ++l) {
         out->union_nodes[l - 1] = (int64_t)ctr[kCtrUnionNodes + l];

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256) k_attn(Batch b, Work w, float scale) {
     const int has_sink = T >= 1 ? 1 : 0;
     const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
-    const int64_t SEGS = segs_per_split(b.n_gl, (int)C);
+    const int64_t SEGS = batch_segs(b, (int)C);
     const int64_t split = blockIdx.x;
     const int64_t sg0 = split * SEGS;
     if (sg0 >= nseg) return;
@@ -201,7 +201,7 @@ __global__ void k_combine(Batch b, Work w, float* out) {
     const int has_sink = T >= 1 ? 1 : 0;
     const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
-    const int64_t SEGS = segs_per_split(b.n_gl, (int)C);
+    const int64_t SEGS = batch_segs(b, (int)C);
     const int64_t nsplit = (nseg + SEGS - 1) / SEGS;
     const float* pp = w.part + x * w.s_cap * PR;
     float M = -INFINITY;

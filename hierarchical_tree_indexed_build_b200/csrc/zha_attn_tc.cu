@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int has_sink = T >= 1 ? 1 : 0;
     const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
-    const int64_t SEGS = segs_per_split(b.n_gl, (int)C);
+    const int64_t SEGS = batch_segs(b, (int)C);
     // grid (lane tiles, splits, groups): the lane tiles of one split run together, so each
     // K/V row they gather is read from DRAM once and from L2 by the others
     const int64_t split = blockIdx.y;
@@ -270,9 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     };
     // Asynchronous gather of the K (K-major) and V (MN-major) rows of buffer st's tokens;
     // empty positions are zero-filled.
+    // Row group g (warps g, g+4, g+8, g+12: one TMEM lane quarter) gathers positions
+    // [32g, 32g + 32), the ones warp g resolved, so one 128-thread named barrier per group
+    // orders the resolve before the gather.
+    const int rg = warp & 3, rt = (warp >> 2) * 32 + lane;
     auto issue_kv = [&](int st) {
-        for (int i = tid; i < kPos * (D / 8); i += kThreads) {
-            const int t = i / (D / 8), c16 = i % (D / 8);
+        for (int i = rt; i < 32 * (D / 8); i += 128) {
+            const int t = 32 * rg + i / (D / 8), c16 = i % (D / 8);
             const int32_t tok = s_tok0[st * kPos + t];
             const uint32_t n = tok >= 0 ? 16u : 0u;
             const int64_t rw = tok >= 0 ? tok : 0;
@@ -392,7 +396,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             phO ^= 1;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         }
-        __syncthreads();                       // partner maxima visible; next tile's tokens visible
+        // partner maxima of the row and the next tile's tokens (resolved by warp rg of this
+        // group) visible to the group: every thread passes here once per tile
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + rg) : "memory");
         if (more) issue_kv(st ^ 1);            // overlaps this tile's softmax and P V
         tmax = fmaxf(fmaxf(s_xmax[row], s_xmax[kRows + row]), fmaxf(s_xmax[2 * kRows + row], s_xmax[3 * kRows + row]));
         tmax = tmax > -INFINITY ? scale * tmax : -INFINITY;

@@ -366,7 +366,7 @@ cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t H
                             float* m, cudaStream_t st) {
     const int64_t total = (int64_t)Hkv * n * R * d / 4;
     if (total <= 0) return cudaSuccess;
-    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148 * 16);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, sm_count() * 16);
     k_export_m<<<(unsigned)blocks, 256, 0, st>>>(rec, cap, ns, Hkv, R, d, n, m);
     return cudaGetLastError();
 }

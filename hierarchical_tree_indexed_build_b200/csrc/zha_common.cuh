@@ -79,6 +79,7 @@ struct Batch {
     int32_t attn_path;               // 0 auto, 1 CUDA cores, 2 tensor cores
     int32_t all_r16;                 // every tree of the batch has R = 16
     int32_t dense = 0;               // every lane attends every token (no routed sets, no lane masks)
+    int32_t split_tok = 0;           // attention split size in tokens (0: split_tokens(n_gl))
 };
 
 // Global lane index of group lane y of group (s, g): lane = (s*n_q + i)*Hq + h.
@@ -133,10 +134,31 @@ constexpr int32_t kStatusCapacity = 2;
 constexpr int32_t kStatusTimeout = 4;        // a bounded wait on the tensor-core pipeline gave up
 constexpr int32_t kStatusRange = 8;          // an entry of Q or of a summary exceeds the fp16 range
 
+// Streaming multiprocessors of the current device (grids are sized in multiples of it);
+// looked up once per device ordinal.
+inline int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 // Split size (tokens) of the attention work for a call with n_gl lanes per group.
 inline __host__ __device__ int split_tokens(int n_gl) { return n_gl <= 64 ? 1024 : 4096; }
 inline __host__ __device__ int64_t segs_per_split(int n_gl, int C) {
     const int64_t s = split_tokens(n_gl) / C;
+    return s > 0 ? s : 1;
+}
+// Split size of a decoder call: groups of a few lanes take short splits (more warps in flight
+// over a small kept set); the partials workspace is sized by lanes x splits.
+inline __host__ __device__ int decoder_split_tokens(int n_gl) { return n_gl <= 16 ? 256 : split_tokens(n_gl); }
+inline __host__ __device__ int64_t batch_segs(const Batch& b, int C) {
+    const int64_t s = (b.split_tok > 0 ? b.split_tok : split_tokens(b.n_gl)) / C;
     return s > 0 ? s : 1;
 }
 

@@ -28,6 +28,11 @@ namespace {
 
 std::mutex g_static_mu;
 void* g_static_ptr[64] = {nullptr};   // device address of g_static_scratch, per device ordinal
+// Host side of each call, per device ordinal: the one-sequence table the kernels read (its
+// upload reads this memory, which stays valid after the call returns) and the status word
+// read back at the end of the call.
+SeqDev g_static_seq[64];
+int32_t g_static_status[64];
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -97,7 +102,7 @@ extern "C" zha_status zha_sparse_attn_static(const void* K, const void* V, int64
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    SeqDev sd;
+    SeqDev& sd = g_static_seq[dev];
     memset(&sd, 0, sizeof(sd));
     sd.C = C;
     sd.L = L;
@@ -154,5 +159,17 @@ extern "C" zha_status zha_sparse_attn_static(const void* K, const void* V, int64
     if (launch_union(b, w, 0, 1, st) != cudaSuccess || launch_attn(b, w, splits, scale, st) != cudaSuccess ||
         launch_combine(b, w, out, st) != cudaSuccess)
         return sfail(ZHA_ERR_CUDA, "kernel launch failed");
+    // The call waits for its kernels and reads the device status word back (no kernel of this
+    // path is expected to set it: the union keeps only chunks under complete top nodes).
+    int32_t& hs = g_static_status[dev];
+    hs = 0;
+    if (cudaMemcpyAsync(&hs, base + status_off, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return sfail(ZHA_ERR_CUDA, "reading the device status word failed");
+    if (hs) {
+        char msg[96];
+        snprintf(msg, sizeof(msg), "device status 0x%x (a union list reached its capacity)", (unsigned)hs);
+        return sfail(ZHA_ERR_DEVICE, msg);
+    }
     return ZHA_OK;
 }

@@ -134,6 +134,14 @@ __device__ __forceinline__ int union_level(const SeqDev& sq, int it, int mode) {
     return sq.T == 0 ? 0 : 1;
 }
 
+// Nodes of level ulev that may enter a union: every complete node when routing; for
+// attention only the level-1 chunks under complete top nodes (T C^L / C of them).  Chunks
+// at or after the first tail token are attended as tail anyway, and bits past the complete
+// chunks name no rows: bits set there in a caller's bitmap are ignored.
+__device__ __forceinline__ int64_t union_limit(const SeqDev& sq, int ulev, int mode) {
+    return mode == 1 ? sq.T * (sq.top / sq.C) : sq.n[ulev];
+}
+
 // OR of the kept bitmaps of a chunk of a group's lanes into the group's union bitmap.
 // Grid: (word blocks, lane chunks of `lanes_per_block`, groups).
 __global__ void __launch_bounds__(256) k_union_or(Batch b, Work w, int it, int mode, int lanes_per_block) {
@@ -142,7 +150,8 @@ __global__ void __launch_bounds__(256) k_union_or(Batch b, Work w, int it, int m
     const SeqDev& sq = b.seqs[s];
     const int ulev = union_level(sq, it, mode);
     if (ulev == 0) return;
-    const int64_t nwords = (sq.n[ulev] + 31) / 32;
+    const int64_t lim = union_limit(sq, ulev, mode);
+    const int64_t nwords = (lim + 31) / 32;
     const int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (wi >= nwords) return;
     const int y0 = blockIdx.y * lanes_per_block;
@@ -152,6 +161,8 @@ __global__ void __launch_bounds__(256) k_union_or(Batch b, Work w, int it, int m
     uint32_t word = 0;
 #pragma unroll 8
     for (int y = y0; y < y1; ++y) word |= __ldg(kb + lane_of(b, s, g, y) * W + wi);
+    const int64_t rest = lim - wi * 32;          // valid bits of this word (>= 1)
+    if (rest < 32) word &= (1u << rest) - 1u;
     if (word) atomicOr(w.uword + (int64_t)grp * w.uw + wi, word);
 }
 
@@ -169,7 +180,7 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
         }
         return;
     }
-    const int64_t nwords = (sq.n[ulev] + 31) / 32;
+    const int64_t nwords = (union_limit(sq, ulev, mode) + 31) / 32;
     const uint32_t* uwp = w.uword + (int64_t)grp * w.uw;
     int32_t* out = w.ulist + (int64_t)grp * w.us;
     int base = 0;
@@ -182,9 +193,14 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
         while (word) {
             const int bit = __ffs(word) - 1;
             word &= word - 1;
-            out[k++] = (int32_t)(wi * 32 + bit);
+            if (k < w.us) out[k] = (int32_t)(wi * 32 + bit);   // the list never outgrows its row
+            ++k;
         }
         base += total;
+    }
+    if (base > w.us) {                                         // cannot happen with the limit above
+        if (threadIdx.x == 0) atomicOr(w.status, kStatusCapacity);
+        base = (int)w.us;
     }
     if (threadIdx.x == 0) {
         w.ucount[grp] = base;
@@ -870,7 +886,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
 }
 
 int score_blocks_x(int lane_blocks, int groups) {
-    const int target = 148 * 8;
+    const int target = sm_count() * 8;
     int nb = target / max(1, lane_blocks * groups);
     return nb < 1 ? 1 : (nb > 65535 ? 65535 : nb);
 }
@@ -895,7 +911,7 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
     if (b.all_r16 && b.n_gl <= kFewLanes && b.d == 128) {
         // one wave: 2 blocks of 8 warps per SM, shared by the groups (d = 128, the geometry
         // the few-lane kernel is validated on; d = 64 takes k_score)
-        const int bx = std::max(1, 2 * 148 / std::max(1, b.n_groups));
+        const int bx = std::max(1, 2 * sm_count() / std::max(1, b.n_groups));
         ProfScope ps_("k_score", st);
         k_score_few<128><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
         return cudaGetLastError();

@@ -25,7 +25,8 @@ _STATUS = {0: "ZHA_OK", 1: "ZHA_ERR_ARG", 2: "ZHA_ERR_CAPACITY", 3: "ZHA_ERR_CUD
 # Every function declared in include/zha.h.
 EXPORTS = ["zha_last_error", "zha_tree_create", "zha_tree_destroy", "zha_tree_info", "zha_build_tree",
            "zha_append", "zha_tree_export", "zha_decoder_create", "zha_decoder_destroy", "zha_route",
-           "zha_sparse_attn", "zha_sparse_attn_static", "zha_dense_attn", "zha_decode", "zha_decoder_set_kernels", "zha_decoder_export_kept", "zha_decoder_words",
+           "zha_sparse_attn", "zha_sparse_attn_static", "zha_dense_attn", "zha_decode", "zha_decoder_set_kernels",
+           "zha_decoder_set_sync", "zha_decoder_export_kept", "zha_decoder_words",
            "zha_decoder_stats", "zha_profile_enable", "zha_profile_read", "zha_profile_reset"]
 
 
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.zha_decode.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp, _i32, ctypes.c_float,
                                  _vp, _vp]
         L.zha_decoder_set_kernels.argtypes = [_vp, _i32, _i32]
+        L.zha_decoder_set_sync.argtypes = [_vp, _i32]
         L.zha_decoder_export_kept.argtypes = [_vp, _i32, _vp, _vp, _vp]
         L.zha_decoder_words.argtypes = [_vp, _i32]
         L.zha_decoder_words.restype = _i64
@@ -187,6 +189,10 @@ ZHA_KERNELS_AUTO, ZHA_KERNELS_SIMT, ZHA_KERNELS_TENSOR = 0, 1, 2
 
 def zha_decoder_set_kernels(dec: int, score: int, attn: int):
     _check(lib().zha_decoder_set_kernels(dec, score, attn))
+
+
+def zha_decoder_set_sync(dec: int, on: bool):
+    _check(lib().zha_decoder_set_sync(dec, 1 if on else 0))
 
 
 def zha_decoder_export_kept(dec: int, level: int, bits: int, counts: Optional[int], stream: int):
@@ -330,6 +336,11 @@ class Decoder:
 
     def set_kernels(self, score: int = ZHA_KERNELS_AUTO, attn: int = ZHA_KERNELS_AUTO):
         zha_decoder_set_kernels(self.handle, score, attn)
+
+    def set_sync(self, on: bool = True):
+        """Synchronous calls: each waits for its work and raises ZhaError(ZHA_ERR_DEVICE)
+        when a kernel set the device status word."""
+        zha_decoder_set_sync(self.handle, on)
 
     def words(self, level: int) -> int:
         return zha_decoder_words(self.handle, level)

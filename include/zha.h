@@ -34,6 +34,9 @@
  *  - Functions return a zha_status; on failure nothing was enqueued, and
  *    zha_last_error() returns a message for the calling thread.  No exception crosses
  *    the ABI.  Objects are not thread-safe; use one thread per object at a time.
+ *  - Conditions only a kernel can see (the device status word, bits listed at
+ *    zha_decoder_stats) are reported by the routing and attention calls themselves: see
+ *    zha_decoder_set_sync.  No kernel traps.
  */
 #ifndef ZHA_H
 #define ZHA_H
@@ -115,6 +118,21 @@ zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n_seq, int32
                               zha_decoder** out);
 zha_status zha_decoder_destroy(zha_decoder* dec);
 
+/* Reporting of the device status word by zha_route, zha_sparse_attn, zha_dense_attn and
+ * zha_decode (the word: bits listed at zha_decoder_stats; zha_route and zha_dense_attn
+ * clear it, zha_sparse_attn adds to what the last zha_route set).  Each of these calls
+ * ends by copying the word to pinned host memory behind its kernels.
+ *   on = 0 (default, asynchronous): the call returns as soon as its work is enqueued.  The
+ *          next of these calls on the decoder, if it starts after the earlier call's work
+ *          has completed on the GPU, returns ZHA_ERR_DEVICE when that word was not 0 (the
+ *          bits in zha_last_error) and enqueues nothing; an earlier call still running is
+ *          reported by a later call or by zha_decoder_stats, which synchronises.  Each
+ *          report is made once.
+ *   on = 1 (synchronous): each call waits for its own work and returns ZHA_ERR_DEVICE
+ *          when the word is not 0 at its end (outputs are then not valid).
+ * Host-side failures are returned at once in both modes. */
+zha_status zha_decoder_set_sync(zha_decoder* dec, int32_t on);
+
 /* Routing for n_q query tokens per sequence.
  *   Q  bf16 [n_seq][n_q][Hq][d] (device).
  *   p  top-p mass, 0 < p <= 1 (p >= 1 keeps every node).
@@ -154,7 +172,10 @@ zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, int32_t attn
  *   C, L   the tree geometry (chunk size; the tail starts at (n_tokens / C^L) C^L)
  *   Q      bf16 [n_q][Hq][d] (device)
  *   kept1  uint32 [n_q*Hq][words] (device): level-1 kept bitmaps, lane x = i*Hq + h,
- *          e.g. from zha_decoder_export_kept(dec, 1, ...); words >= ceil(n_tokens/C/32)
+ *          e.g. from zha_decoder_export_kept(dec, 1, ...); words >= ceil(n_tokens/C/32).
+ *          Only bits of chunks under complete top nodes count (chunk j < T C^L / C with
+ *          T = n_tokens / C^L); bits at or after the tail's first chunk, and bits past
+ *          n_tokens / C, are ignored (the tail is attended whole in any case)
  *   out    f32 [n_q][Hq][d] (device)
  * Working memory comes from one 16 MiB array in the library's device image, reserved on
  * every device that loads the library until the process exits; a call needing more
@@ -165,7 +186,9 @@ zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, int32_t attn
  * contents in it; each call clears what must start at zero, so back-to-back calls on one
  * stream are independent, but calls that can overlap on the GPU (different streams or
  * threads, same device) race on the array.  No cudaMalloc/cudaFree or allocating
- * library routine is called. */
+ * library routine is called.  Each call waits for its own work on `stream` to finish and
+ * reads the array's status word back: ZHA_ERR_DEVICE if a kernel set it (none is expected
+ * to on this path). */
 zha_status zha_sparse_attn_static(const void* K, const void* V, int64_t ld, int64_t n_tokens,
                                   int32_t C, int32_t L, int32_t Hq, int32_t Hkv, int32_t d,
                                   const void* Q, int32_t n_q, const uint32_t* kept1, int64_t words,
@@ -201,8 +224,8 @@ int64_t zha_decoder_words(const zha_decoder* dec, int32_t level);
  * nodes scored per level as the union over each (sequence, KV head) group of lanes and
  * as the per-lane sum, attended tokens (union per group and per-lane sum), and the
  * device status word (0 = ok; bit 1: the top-p select ran out of bisection steps,
- * bit 4: a tensor-core wait gave up after 2 s, bit 8: an input outside the fp16 range
- * reached the tensor-core scorer).
+ * bit 2: a union list reached its capacity, bit 4: a tensor-core wait gave up after 2 s,
+ * bit 8: an input outside the fp16 range reached the tensor-core scorer).
  * Returns ZHA_ERR_DEVICE when the status word is not 0. */
 typedef struct zha_decode_stats {
     int64_t union_nodes[ZHA_MAX_LEVELS];      /* index l-1 */

@@ -22,9 +22,7 @@ needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a C
 
 
 def _report(name, rep, e1, e2):
-    print("[%s] levels=%d exact=%d mass_ties=%d score_ties=%d  out/own max=%.2e  out/e2e max=%s"
-          % (name, rep.levels, rep.exact, rep.mass_ties, rep.score_ties, e1.max(),
-             "%.2e" % e2.max() if e2.size else "-"))
+    TL.record(name, rep, e1, e2)
 
 
 @needs_cuda

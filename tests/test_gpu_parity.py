@@ -15,9 +15,7 @@ needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a C
 
 
 def _report(name, rep, e1, e2):
-    print("[%s] levels=%d exact=%d mass_ties=%d score_ties=%d  out/own max=%.2e  out/e2e max=%s"
-          % (name, rep.levels, rep.exact, rep.mass_ties, rep.score_ties, e1.max(),
-             "%.2e" % e2.max() if e2.size else "-"))
+    TL.record(name, rep, e1, e2)
 
 
 # ----------------------------------------------------------------------------- build
@@ -383,3 +381,111 @@ def test_dense_attention_equals_routed_decode_at_p1():
     assert torch.equal(sparse, again)
     dec.close()
     tree.close()
+
+
+# ----------------------------------------------------------------------------- kernel configurations
+
+# Geometries that reach kernel variants the workloads above do not: d = 64 on both tensor-core
+# kernels, chunk sizes that are not a multiple of 4 on the tensor scorer (one-node copies of
+# each record instead of four-node runs), C = 16 on the tensor scorer, R = 32 (CUDA cores).
+D64 = inputs.Geometry(C=4, L=4, R=16, d=64, Hq=16, Hkv=2)
+C6R16 = inputs.Geometry(C=6, L=3, R=16, d=128, Hq=16, Hkv=2)
+C2R16 = inputs.Geometry(C=2, L=7, R=16, d=128, Hq=16, Hkv=2)
+R32 = inputs.Geometry(C=4, L=4, R=32, d=128, Hq=16, Hkv=2)
+
+
+@needs_cuda
+@pytest.mark.parametrize("name,geom,n_tokens,n_q,paths", [
+    # 64 lanes per (sequence, KV head) group: the automatic choice takes both tcgen05 kernels
+    ("d64 tensor", D64, 10 * 256 + 77, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("C6 R16 tensor", C6R16, 14 * 216 + 101, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("C2 R16 tensor", C2R16, 40 * 128 + 33, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("C16 MID tensor", inputs.MID, 3 * 4096 + 900, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("C16 MID tensor 24q", inputs.MID, 3 * 4096 + 900, 24, (zha.ZHA_KERNELS_TENSOR, zha.ZHA_KERNELS_TENSOR)),
+    # R = 32: scoring on CUDA cores (k_score), attention both ways
+    ("R32 simt", R32, 12 * 256 + 5, 2, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("R32 simt score, tensor attn", R32, 12 * 256 + 5, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+])
+def test_decode_kernel_configurations(name, geom, n_tokens, n_q, paths):
+    seq = inputs.make_sequence(geom, n_tokens, n_tokens, seed=41)
+    Q, _ = inputs.make_queries(seq, n_q, 8, n_tokens, np.random.default_rng(7))
+    tree, K, V, qr = TL.make_tree(seq)
+    w = TL.compare_summaries(tree, seq, n_tokens, sample=64)
+    assert max(w.values()) <= TL.SUM_TOL, w
+    dec = zha.Decoder([tree], n_q)
+    dec.set_kernels(*paths)
+    res = TL.gpu_decode([tree], [K], [V], Q[None], 0.9, dec=dec)
+    assert res.stats.status == 0
+    qs = sorted(set([0, n_q // 2, n_q - 1]))
+    rep, e1, e2, _ = TL.check_decode(seq, n_tokens, Q, 0.9, res.out[0], res.kept[0], qs)
+    _report(name, rep, e1, e2)
+    # the CUDA-core kernels on the same tree agree (kept sets up to logged ties, outputs)
+    ref_dec = zha.Decoder([tree], n_q)
+    ref_dec.set_kernels(zha.ZHA_KERNELS_SIMT, zha.ZHA_KERNELS_SIMT)
+    ref = TL.gpu_decode([tree], [K], [V], Q[None], 0.9, dec=ref_dec)
+    differ = sum(int((x != y).any(axis=1).sum()) for x, y in zip(res.kept[0], ref.kept[0]))
+    lanes = res.kept[0][0].shape[0]
+    assert differ <= max(2, lanes * geom.L // 50), differ
+    same = np.ones(lanes, dtype=bool)
+    for x, y in zip(res.kept[0], ref.kept[0]):
+        same &= ~(x != y).any(axis=1)
+    e = TL.rel_err(res.out[0].reshape(-1, geom.d)[same], ref.out[0].reshape(-1, geom.d)[same])
+    assert e.max() <= 1e-4, e.max()
+    dec.close()
+    ref_dec.close()
+    tree.close()
+
+
+# ----------------------------------------------------------------------------- device status at the boundary
+
+def _range_case():
+    """64 lanes per group (tensor-core scorer) with one query entry beyond the fp16 range."""
+    wl = inputs.deep_64k(n_q=8)
+    seq = wl.seqs[0]
+    tree, K, V, qr = TL.make_tree(seq)
+    Q = wl.Q[0].clone()
+    good = Q.cuda().contiguous()
+    Q[0, 3, 5, 7] = 1.0e5
+    return tree, K, V, Q.cuda().contiguous(), good
+
+
+@needs_cuda
+def test_decode_reports_device_status_in_sync_mode():
+    """A synchronous decoder returns ZHA_ERR_DEVICE from zha_decode itself when the tensor
+    scorer flags an input outside the fp16 range (status bit 8), and ZHA_OK again for valid
+    input."""
+    tree, K, V, bad, good = _range_case()
+    dec = zha.Decoder([tree], 8)
+    dec.set_kernels(zha.ZHA_KERNELS_TENSOR, zha.ZHA_KERNELS_AUTO)
+    dec.set_sync(True)
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.decode([K], [V], bad, 0.95)
+    assert ei.value.status == zha.ZHA_ERR_DEVICE
+    assert "0x8" in str(ei.value) and "fp16" in str(ei.value)
+    dec.decode([K], [V], good, 0.95)
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.route(bad, 0.95)
+    assert ei.value.status == zha.ZHA_ERR_DEVICE
+    dec.close()
+
+
+@needs_cuda
+def test_decode_reports_device_status_on_the_next_call_when_async():
+    """Asynchronous (default) decoder: the flagged call returns ZHA_OK; once its work has
+    completed, the next call on the decoder returns ZHA_ERR_DEVICE and enqueues nothing; the
+    call after that runs normally."""
+    tree, K, V, bad, good = _range_case()
+    dec = zha.Decoder([tree], 8)
+    dec.set_kernels(zha.ZHA_KERNELS_TENSOR, zha.ZHA_KERNELS_AUTO)
+    dec.decode([K], [V], bad, 0.95)
+    torch.cuda.synchronize()
+    out = torch.full((1, 8, 16, 128), 7.0, device="cuda")
+    with pytest.raises(zha.ZhaError) as ei:
+        dec.decode([K], [V], good, 0.95, out)
+    assert ei.value.status == zha.ZHA_ERR_DEVICE
+    torch.cuda.synchronize()
+    assert (out == 7.0).all()                    # nothing was enqueued
+    dec.decode([K], [V], good, 0.95, out)
+    torch.cuda.synchronize()
+    assert dec.stats().status == 0
+    dec.close()
