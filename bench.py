@@ -49,9 +49,15 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparison")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the wide 256K and batched 32 x 128K measurements")
     ap.add_argument("--n-q", type=int, default=0, help="decode only the workload's first n query tokens (profiling)")
     ap.add_argument("--workload", default="deep1m", choices=["deep1m", "deep64k", "deep256k", "wide256k"],
                     help="deep1m is the benchmark; the smaller ones serve profiling runs")
+    ap.add_argument("--stage-sweep", default="",
+                    help="comma-separated p values: instead of the benchmark line, print one JSON line "
+                         "per p with the decode's per-kernel device times and work counters (and one "
+                         "for the build), the measurements the stage model is fitted to")
     return ap.parse_args()
 
 
@@ -352,8 +358,168 @@ def run_ours(args, rank, world, dev):
         h2d = sum(x.numel() * x.element_size() for x in (Kh, Vh, qh, Qh))
         res["e2e"] = {"value": whole_job_rate(world, n_q, ems / args.steps), "unit": "queries/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outh.numel() * 4}
+    # the build phase of the benchmark step: tokens/s and the fraction of HBM bandwidth its
+    # algorithmic bytes (K read + every node record written) reach
+    b_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("k_build_stream", "k_merge")) / args.steps
+    if b_ms > 0:
+        hbm_peak, src = measured_peaks()
+        bb = build_bytes(g, N0 + n_app)
+        res["build"] = {"tokens": N0 + n_app, "ms": b_ms, "tokens_per_s": (N0 + n_app) / (b_ms / 1e3),
+                        "algorithmic_gb": bb / 1e9, "hbm_frac_of_%s" % src: bb / (b_ms / 1e3) / 1e9 / hbm_peak}
+    if not args.no_per_workload:
+        res["per_workload"] = per_workload(args, dev, stream)
     res["wl"] = wl
     return res
+
+
+def build_bytes(g, n_tokens):
+    """Bytes a build over n_tokens must move: K read (2d B per token per KV head) and every
+    complete node's record written ((R d + 2R) 4 B: m and b, and lse)."""
+    nodes = sum(n_tokens // g.C ** l for l in range(1, g.L + 1))
+    return g.Hkv * (n_tokens * 2 * g.d + nodes * (g.R * g.d + 2 * g.R) * 4)
+
+
+def per_workload(args, dev, stream):
+    """The other geometries of the metric, each timed with CUDA events on its own (after the
+    benchmark's timed region): the wide 256K tree (C256 L1) - build over the whole cache
+    and the decode of its 64 queries - and the batched workload (32 x 131,072 tokens, half
+    C16 L3, half C4 L6) - one appended token and one decoded query per sequence per step."""
+    from hierarchical_tree_indexed_build_b200 import zha
+    hbm_peak, src = measured_peaks()
+    frac_key = "hbm_frac_of_%s" % src
+    out = {}
+
+    def timed(fn, reps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # wide 256K
+    wl = inputs.wide_256k()
+    seq = wl.seqs[0]
+    g = seq.geom
+    K, V, qr = seq.K.to(dev), seq.V.to(dev), seq.qref.to(dev)
+    Q = wl.Q[0].to(dev).contiguous()
+    tree = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, seq.capacity)
+    n = seq.n_tokens
+    bms = timed(lambda: tree.build(K, n, qr), args.steps)
+    dec = zha.Decoder([tree], Q.shape[1])
+    o = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    dms = timed(lambda: dec.decode([K], [V], Q, args.p, o), args.steps)
+    st = dec.stats()
+    ub = sum(st.union_nodes) * st.node_bytes + st.union_tokens * 4 * g.d
+    bb = build_bytes(g, n)
+    out["wide_256k_C256L1"] = {
+        "n_tokens": n, "queries": int(Q.shape[1]), "p": args.p,
+        "decode_ms": dms, "queries_per_s": Q.shape[1] / (dms / 1e3),
+        "union_gb": ub / 1e9, "union_" + frac_key: ub / (dms / 1e3) / 1e9 / hbm_peak,
+        "keys_touched_frac": st.lane_tokens / (Q.shape[1] * g.Hq * n),
+        "build_ms": bms, "build_tokens_per_s": n / (bms / 1e3), "build_" + frac_key: bb / (bms / 1e3) / 1e9 / hbm_peak}
+    dec.close()
+    tree.close()
+    del K, V, qr, Q, o
+
+    # batched 32 x 128K, mixed geometries, 1-token append + 1 query per sequence per step
+    n_steps = max(3, args.warmup) + args.steps
+    wl = inputs.batched_32x128k(n_steps=n_steps)
+    trees, Ks, Vs = [], [], []
+    for sq in wl.seqs:
+        gg = sq.geom
+        Kd, Vd = sq.K.to(dev), sq.V.to(dev)
+        t = zha.Tree(gg.C, gg.L, gg.R, gg.d, gg.Hq, gg.Hkv, sq.capacity)
+        t.build(Kd, sq.n_tokens, sq.qref.to(dev))
+        trees.append(t)
+        Ks.append(Kd)
+        Vs.append(Vd)
+    dec = zha.Decoder(trees, 1)
+    Qs = wl.Q.to(dev)                               # [steps][32][1][16][128]
+    o = torch.empty(Qs.shape[1:], dtype=torch.float32, device=dev)
+    step = [0]
+
+    def bstep():
+        k = step[0]
+        for s, sq in enumerate(wl.seqs):
+            trees[s].append(Ks[s], sq.n_tokens + k, 1)
+        dec.decode(Ks, Vs, Qs[k], args.p, o)
+        step[0] += 1
+
+    sms = timed(bstep, args.steps)
+    st = dec.stats()
+    ub = sum(st.union_nodes) * st.node_bytes + st.union_tokens * 4 * 128
+    toks = sum(sq.n_tokens + step[0] for sq in wl.seqs)
+    out[wl.name] = {
+        "sequences": len(wl.seqs), "n_tokens_per_seq": wl.seqs[0].n_tokens, "queries_per_step": len(wl.seqs),
+        "p": args.p, "step": "1-token append per sequence + decode of one query per sequence",
+        "step_ms": sms, "queries_per_s": len(wl.seqs) / (sms / 1e3),
+        "union_gb_last_step": ub / 1e9, "union_" + frac_key: ub / (sms / 1e3) / 1e9 / hbm_peak,
+        "keys_touched_frac": st.lane_tokens / (16 * toks)}
+    dec.close()
+    for t in trees:
+        t.close()
+    return out
+
+
+def stage_sweep(args, dev):
+    """Per-kernel device times (library CUDA-event profile) and the decoder's work counters
+    of the workload's build and of its decode at each p, one JSON line each."""
+    from hierarchical_tree_indexed_build_b200 import zha
+    torch.cuda.set_device(dev)
+    wl = load_workload(args.workload)
+    seq = wl.seqs[0]
+    g = seq.geom
+    N0, n_app = seq.n_tokens, wl.n_append
+    K, V, qref = seq.K.to(dev), seq.V.to(dev), seq.qref.to(dev)
+    Q = wl.Q[0].contiguous()
+    if args.n_q > 0:
+        Q = Q[:, :args.n_q].contiguous()
+    Q = Q.to(dev)
+    tree = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, seq.capacity)
+    dec = zha.Decoder([tree], Q.shape[1])
+    out = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    geom = {"C": g.C, "L": g.L, "R": g.R, "d": g.d, "Hq": g.Hq, "Hkv": g.Hkv}
+
+    def profiled(fn, reps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        zha.zha_profile_reset()
+        zha.zha_profile_enable(True)
+        for _ in range(reps):
+            fn()
+        torch.cuda.synchronize()
+        zha.zha_profile_enable(False)
+        pr = zha.zha_profile_read()
+        return ({k: v[1] / reps for k, v in pr.items()}, {k: v[0] / reps for k, v in pr.items()})
+
+    def build():
+        tree.build(K, N0, qref)
+        if n_app:
+            tree.append(K, N0, n_app)
+
+    ms, la = profiled(build, args.steps)
+    print(json.dumps({"workload": wl.name, "stage": "build", "n_tokens": N0 + n_app, "geometry": geom,
+                      "kernel_ms": ms, "kernel_launches": la}))
+    for p in [float(x) for x in args.stage_sweep.split(",") if x]:
+        for nq in sorted({int(Q.shape[1]), 1}):
+            Qp = Q[:, :nq].contiguous()
+            op = out[:, :nq].contiguous()
+            ms, la = profiled(lambda: dec.decode([K], [V], Qp, p, op), args.steps)
+            st = dec.stats()
+            print(json.dumps({"workload": wl.name, "stage": "decode", "p": p, "n_q": nq, "n_tokens": N0 + n_app,
+                              "geometry": geom, "kernel_ms": ms, "kernel_launches": la,
+                              "stats": {"union_nodes": list(st.union_nodes)[:g.L],
+                                        "lane_nodes": list(st.lane_nodes)[:g.L],
+                                        "union_tokens": st.union_tokens, "lane_tokens": st.lane_tokens,
+                                        "node_bytes": st.node_bytes}}))
+    dec.close()
+    tree.close()
 
 
 def load_workload(name):
@@ -432,6 +598,10 @@ def main():
                      "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
         print(json.dumps(line))
         return
+    if args.stage_sweep:
+        if rank == 0:
+            stage_sweep(args, local)
+        return
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
                                              timeout=__import__("datetime").timedelta(seconds=120))
@@ -457,6 +627,10 @@ def main():
         line["stats"] = res["stats"]
         if "dense" in res:
             line["dense"] = res["dense"]
+        if "build" in res:
+            line["build"] = res["build"]
+        if "per_workload" in res:
+            line["per_workload"] = res["per_workload"]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.p)
         print(json.dumps(line))

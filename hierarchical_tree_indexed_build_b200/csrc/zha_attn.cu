@@ -186,11 +186,21 @@ __global__ void __launch_bounds__(256) k_attn(Batch b, Work w, float scale) {
 }
 
 // out[x] = sum_splits exp(m_s - M) o_s / sum_splits exp(m_s - M) l_s.
+// One block of kCombThreads per lane: the splits' maximum M by a block reduction, then warp
+// w sums splits w, w + 8, ... (each thread D/32 dims) and the warps' sums are added in warp
+// order, so the result does not depend on scheduling.
+constexpr int kCombThreads = 256;
+
 template <int D>
-__global__ void k_combine(Batch b, Work w, float* out) {
+__global__ void __launch_bounds__(kCombThreads) k_combine(Batch b, Work w, float* out) {
     constexpr int PR = D + 4;
+    constexpr int NW = kCombThreads / 32;
+    constexpr int DPT = D / 32;                  // dims per thread
+    __shared__ float s_red[NW];
+    __shared__ __align__(16) float s_num[NW][D];
+    __shared__ float s_den[NW];
     const int64_t x = blockIdx.x;
-    const int dd = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int s = (int)(x / ((int64_t)b.n_q * b.Hq));
     const int h = (int)(x % b.Hq);
     const int g = h / b.G;
@@ -205,19 +215,51 @@ __global__ void k_combine(Batch b, Work w, float* out) {
     const int64_t nsplit = (nseg + SEGS - 1) / SEGS;
     const float* pp = w.part + x * w.s_cap * PR;
     float M = -INFINITY;
-    for (int64_t sp = 0; sp < nsplit; ++sp)
+    for (int64_t sp = tid; sp < nsplit; sp += kCombThreads)
         if (pp[sp * PR + D + 1] > 0.0f) M = fmaxf(M, pp[sp * PR + D]);
-    float num = 0.0f, den = 0.0f;
-    for (int64_t sp = 0; sp < nsplit; ++sp) {
-        const float l = pp[sp * PR + D + 1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_red[warp] = M;
+    __syncthreads();
+    M = s_red[0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) M = fmaxf(M, s_red[i]);
+    float num[DPT];
+#pragma unroll
+    for (int k = 0; k < DPT; ++k) num[k] = 0.0f;
+    float den = 0.0f;
+    for (int64_t sp = warp; sp < nsplit; sp += NW) {
+        const float* rec = pp + sp * PR;
+        const float l = rec[D + 1];
         if (l > 0.0f) {
-            const float c = expf(pp[sp * PR + D] - M);
-            num = fmaf(c, pp[sp * PR + dd], num);
+            const float c = expf(rec[D] - M);
+            if constexpr (DPT == 4) {
+                const float4 o4 = reinterpret_cast<const float4*>(rec)[lane];
+                num[0] = fmaf(c, o4.x, num[0]);
+                num[1] = fmaf(c, o4.y, num[1]);
+                num[2] = fmaf(c, o4.z, num[2]);
+                num[3] = fmaf(c, o4.w, num[3]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < DPT; ++k) num[k] = fmaf(c, rec[lane * DPT + k], num[k]);
+            }
             den = fmaf(c, l, den);
         }
     }
-    out[x * D + dd] = num / den;
-    if (dd == 0) {
+#pragma unroll
+    for (int k = 0; k < DPT; ++k) s_num[warp][lane * DPT + k] = num[k];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+    if (tid < D) {
+        float nn = 0.0f, dd = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            nn += s_num[i][tid];
+            dd += s_den[i];
+        }
+        out[x * D + tid] = nn / dd;
+    }
+    if (tid == 0) {
         int64_t a = tail;
         if (has_sink) {
             const uint32_t first = w.kept[1][x * w.W[1]];
@@ -249,9 +291,9 @@ cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st) {
     ProfScope ps_("k_combine", st);
     if (b.d == 128)
-        k_combine<128><<<b.n_lanes, 128, 0, st>>>(b, w, out);
+        k_combine<128><<<b.n_lanes, kCombThreads, 0, st>>>(b, w, out);
     else
-        k_combine<64><<<b.n_lanes, 64, 0, st>>>(b, w, out);
+        k_combine<64><<<b.n_lanes, kCombThreads, 0, st>>>(b, w, out);
     return cudaGetLastError();
 }
 

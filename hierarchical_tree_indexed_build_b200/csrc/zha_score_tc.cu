@@ -25,10 +25,10 @@
 //               query tile (A) in tensor memory and the node tile (B) in shared memory;
 //   warps 2..   epilogue, 4 per lane tile: tensor memory -> max over planes + b -> scores.
 // With A in tensor memory an MMA reads only its B rows from shared memory.  Each lane tile
-// has one accumulator; while one lane tile's epilogue drains, the other's MMAs run (with
-// LT = 1 the accumulator is double-buffered instead).
-// Tensor memory: accumulators at columns 0 and 128, the queries of lane tile t at columns
-// 256 + t d/2 (two fp16 of a row per 32-bit column).
+// job (node tile, lane tile) takes the next of three accumulators in turn, so the MMAs of
+// up to two further jobs run while one job's epilogue drains.
+// Tensor memory: accumulators at columns 0, 128 and 256, the queries of lane tile t at
+// columns 384 + t d/2 (two fp16 of a row per 32-bit column).
 //
 // Frontier membership comes from k_member: for every union parent u of the level above
 // and every 32 lanes of the group, one word whose bit t says whether lane 32 w + t kept u
@@ -303,8 +303,10 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     constexpr int KB = D / 64;                        // 128-byte K blocks of fp16
     constexpr int P_BYTES = KB * kTileN * 128;        // one fp16 plane of one stage
     constexpr int STAGE = kPlanes * P_BYTES;
-    constexpr uint32_t kColA = 256;                   // queries; accumulators at 0 and 128
+    constexpr int kAcc = 3;                           // accumulator slots (columns 0, 128, 256)
+    constexpr uint32_t kColA = kAcc * kTileN;         // queries after the accumulators
     constexpr uint32_t kCols = 512;
+    static_assert(kColA + LT * (D / 2) <= kCols, "accumulators and queries must fit the 512 TMEM columns");
     constexpr uint32_t kNodeBytes = kPlanes * KB * 16 * 128;   // both planes of one node
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte aligned start, reached by pointer arithmetic on the shared array so that every
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     float* sBv = reinterpret_cast<float*>(sB0 + kStages * STAGE);          // [kStages][kNodes][16] b values
     uint32_t* sMask = reinterpret_cast<uint32_t*>(sBv + kStages * kTileN); // [kStages][kNodes][kLW] membership
     int32_t* sJ = reinterpret_cast<int32_t*>(sMask + kStages * kNodes * kLW);   // [kStages][kNodes] node ids
-    __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages], bar_acc_full[2], bar_acc_empty[2];
+    __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages], bar_acc_full[kAcc], bar_acc_empty[kAcc];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     volatile int& abort_sh = abort_flag;              // set by any role whose wait gave up
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
             mbar_init(smem_u32(&bar_full[i]), 1);
             mbar_init(smem_u32(&bar_empty[i]), kEpilogue);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kAcc; ++i) {
             mbar_init(smem_u32(&bar_acc_full[i]), 1);
             mbar_init(smem_u32(&bar_acc_empty[i]), kTileM);   // one lane tile drains a slot
         }
@@ -491,10 +493,10 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
         if (lane == 0) {
             const int jobs = nt * LT;
             for (int q = 0; q < jobs && !abort_sh; ++q) {
-                const int i = q / LT, t = q % LT, st = i % kStages, slot = q & 1;
+                const int i = q / LT, t = q % LT, st = i % kStages, slot = q % kAcc;
                 bool okw = true;
                 if (t == 0) okw = mbar_wait(smem_u32(&bar_full[st]), (uint32_t)((i / kStages) & 1));
-                if (okw && q >= 2) okw = mbar_wait(smem_u32(&bar_acc_empty[slot]), (uint32_t)(((q >> 1) - 1) & 1));
+                if (okw && q >= kAcc) okw = mbar_wait(smem_u32(&bar_acc_empty[slot]), (uint32_t)(((q / kAcc) - 1) & 1));
                 if (!okw) {
                     atomicOr(w.status, kStatusTimeout);
                     abort_sh = 1;
@@ -527,8 +529,8 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
         int fcnt = 0;
 #pragma unroll 1
         for (int i = 0; i < nt; ++i) {
-            const int st = i % kStages, q = i * LT + lt, slot = q & 1;
-            if (!mbar_wait(smem_u32(&bar_acc_full[slot]), (uint32_t)((q >> 1) & 1))) {
+            const int st = i % kStages, q = i * LT + lt, slot = q % kAcc;
+            if (!mbar_wait(smem_u32(&bar_acc_full[slot]), (uint32_t)((q / kAcc) & 1))) {
                 atomicOr(w.status, kStatusTimeout);
                 abort_sh = 1;
             }
@@ -604,7 +606,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
 
 template <int D, int LT>
 cudaError_t launch_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st, int pairs) {
-    int nb = 148 / max(1, pairs * b.n_groups);
+    int nb = sm_count() / max(1, pairs * b.n_groups);
     nb = nb < 1 ? 1 : nb;
     dim3 grid(nb, pairs, b.n_groups);
     const size_t smem = score_tc_smem_lt(D, LT);
@@ -626,7 +628,7 @@ cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaS
     ProfScope ps_("k_member", st);
     const int lwg = (b.n_gl + 255) / 256;             // groups of 8 lane words
     int nbx = (int)((w.ms + 255) / 256);
-    const int cap = (148 * 8) / max(1, lwg * b.n_groups);
+    const int cap = (sm_count() * 8) / max(1, lwg * b.n_groups);
     nbx = nbx < 1 ? 1 : (nbx > cap ? (cap < 1 ? 1 : cap) : nbx);
     k_member<<<dim3(nbx, lwg, b.n_groups), 256, 0, st>>>(b, w, it, mode);
     return cudaGetLastError();
