@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparison")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the bf16-record router measurement")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the wide 256K and batched 32 x 128K measurements")
     ap.add_argument("--n-q", type=int, default=0, help="decode only the workload's first n query tokens (profiling)")
@@ -73,7 +74,7 @@ def measured_peaks():
 # Kernel -> source file whose contents its DRAM-traffic record was taken against.
 KERNEL_SOURCES = {
     "k_score_tc": "zha_score_tc.cu", "k_attn_tc": "zha_attn_tc.cu", "k_select": "zha_route.cu",
-    "k_score": "zha_route.cu", "k_attn": "zha_attn.cu", "k_build_stream": "zha_build.cu",
+    "k_score": "zha_route.cu", "k_attn": "zha_attn.cu", "k_build_stream": "zha_build.cu", "k_build_tc": "zha_build_tc.cu",
 }
 
 
@@ -178,10 +179,10 @@ def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
         return st.union_tokens * 4 * d / launches, st.lane_tokens * 4 * d / launches
     if name == "k_select":
         return sum(st.lane_nodes) * 4 / launches, 0.0
-    if name in ("k_build_stream", "k_merge"):
+    if name in ("k_build_tc", "k_build_stream", "k_merge"):
         nodes = sum((N + n_append) // geom.C ** l for l in range(1, geom.L + 1))
         rec = (R * d + 2 * R) * 4
-        reads = geom.Hkv * (N + n_append) * 2 * d if name == "k_build_stream" else 0
+        reads = geom.Hkv * (N + n_append) * 2 * d if name in ("k_build_tc", "k_build_stream") else 0
         return (reads + geom.Hkv * nodes * rec) / launches, 0.0
     return 0.0, 0.0
 
@@ -327,6 +328,56 @@ def run_ours(args, rank, world, dev):
                         "one_query_dense_ms": dense1_ms, "one_query_zha_decode_ms": zha1_ms,
                         "one_query_speedup": dense1_ms / zha1_ms}
 
+    # The reduced-precision router: the same grown cache indexed by a tree whose records hold
+    # the slopes as one bf16 plane (half the bytes per scored node, one tensor-core pass), the
+    # same queries decoded; per-kernel times from the library profile.
+    if not args.no_bf16:
+        tree16 = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, seq.capacity, zha.ZHA_SUMMARY_BF16)
+        tree16.build(K, N0, qref)
+        if n_app:
+            tree16.append(K, N0, n_app)
+        dec16 = zha.Decoder([tree16], n_q)
+        out16 = torch.empty_like(out)
+        for _ in range(max(3, args.warmup)):
+            dec16.decode([K], [V], Q, args.p, out16)
+        torch.cuda.synchronize()
+        zha.zha_profile_reset()
+        zha.zha_profile_enable(True)
+        for _ in range(args.steps):
+            dec16.decode([K], [V], Q, args.p, out16)
+        torch.cuda.synchronize()
+        zha.zha_profile_enable(False)
+        pr16 = zha.zha_profile_read()
+        st16 = dec16.stats()
+        d16 = sum(v[1] for v in pr16.values()) / args.steps
+        ub16 = sum(st16.union_nodes) * st16.node_bytes + st16.union_tokens * 4 * g.d
+        hbm_peak, src = measured_peaks()
+        obj = {"format": "bf16 slopes (one plane)", "node_bytes": st16.node_bytes, "decode_ms": d16,
+               "queries_per_s": n_q / (d16 / 1e3), "union_gb": ub16 / 1e9,
+               "union_frac_of_%s_hbm" % src: ub16 / (d16 / 1e3) / 1e9 / hbm_peak,
+               "stages_ms": {k: round(v[1] / args.steps, 4) for k, v in sorted(pr16.items())},
+               "max_abs_out_diff_vs_two_plane_tree": float((out16 - out).abs().max().item())}
+        for kn in ("k_score_tc", "k_score", "k_score_few"):
+            if kn in pr16:
+                la, tms = pr16[kn]
+                per = la / args.steps
+                nb, nf = kernel_algorithmic(kn, st16, g, N0, n_app, n_q * g.Hq, per)
+                avg = tms / la
+                if kn == "k_score_tc":
+                    peak, psrc = tensor_peak("bf16")
+                    obj["roofline"] = {"kernel": kn, "bound": "tensor", "achieved": nf / (avg / 1e3) / 1e12,
+                                       "peak": peak, "unit": "TFLOP/s", "frac": nf / (avg / 1e3) / 1e12 / peak,
+                                       "hbm_frac": nb / (avg / 1e3) / 1e9 / hbm_peak, "avg_launch_ms": avg,
+                                       "peak_source": psrc}
+                else:
+                    obj["roofline"] = {"kernel": kn, "bound": "hbm", "achieved": nb / (avg / 1e3) / 1e9,
+                                       "peak": hbm_peak, "unit": "GB/s", "frac": nb / (avg / 1e3) / 1e9 / hbm_peak,
+                                       "avg_launch_ms": avg, "peak_source": src}
+                break
+        res["bf16_router"] = obj
+        dec16.close()
+        tree16.close()
+
     # end to end through the public API with host buffers
     if not args.no_e2e:
         Kh = seq.K.pin_memory()
@@ -360,7 +411,7 @@ def run_ours(args, rank, world, dev):
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outh.numel() * 4}
     # the build phase of the benchmark step: tokens/s and the fraction of HBM bandwidth its
     # algorithmic bytes (K read + every node record written) reach
-    b_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("k_build_stream", "k_merge")) / args.steps
+    b_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("k_build_tc", "k_build_stream", "k_merge")) / args.steps
     if b_ms > 0:
         hbm_peak, src = measured_peaks()
         bb = build_bytes(g, N0 + n_app)
@@ -631,6 +682,8 @@ def main():
             line["build"] = res["build"]
         if "per_workload" in res:
             line["per_workload"] = res["per_workload"]
+        if "bf16_router" in res:
+            line["bf16_router"] = res["bf16_router"]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.p)
         print(json.dumps(line))

@@ -48,7 +48,7 @@ float score_scale(int d) { return (float)(1.0 / sqrt((double)d)); }
 //   maps[0] planes, boxes of 64 dims x R planes x 1 node
 //   maps[1] planes, boxes of 64 dims x R planes x 4 nodes
 //   maps[2] b, boxes of R values x 4 nodes
-bool encode_level_maps(CUtensorMap* maps, const float* rec, int d, int R, int64_t nodes, int ns) {
+bool encode_level_maps(CUtensorMap* maps, const float* rec, int d, int R, int64_t nodes, int ns, int fmt) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
@@ -58,12 +58,15 @@ bool encode_level_maps(CUtensorMap* maps, const float* rec, int d, int R, int64_
             return false;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)R, 2, (cuuint64_t)nodes};
+    // planes viewed as (dim, slope r, plane, node): two fp16 planes, or one bf16 plane
+    const cuuint64_t planes = fmt == kFmtBf16 ? 1 : 2;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)R, planes, (cuuint64_t)nodes};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)R * d * 2, (cuuint64_t)ns * 4};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapDataType dt = fmt == kFmtBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     for (int k = 0; k < 2; ++k) {
         const cuuint32_t box[4] = {64, (cuuint32_t)R, 1, k == 0 ? 1u : 4u};
-        if (encode(&maps[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<float*>(rec), dims, strides, box, estr,
+        if (encode(&maps[k], dt, 4, const_cast<float*>(rec), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
@@ -72,7 +75,7 @@ bool encode_level_maps(CUtensorMap* maps, const float* rec, int d, int R, int64_
     const cuuint64_t bstrides[1] = {(cuuint64_t)ns * 4};
     const cuuint32_t bbox[2] = {(cuuint32_t)R, 4};
     const cuuint32_t bestr[2] = {1, 1};
-    return encode(&maps[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(rec) + (int64_t)R * d, bdims,
+    return encode(&maps[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(rec) + b_offset(R, d, fmt), bdims,
                   bstrides, bbox, bestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -138,6 +141,8 @@ static zha_status check_geometry(const zha_geometry* g) {
         return fail(ZHA_ERR_ARG, "capacity / C must be <= 2^24 level-1 nodes");
     double top = pow((double)g->C, (double)g->L);
     if (top > 4.0e15) return fail(ZHA_ERR_ARG, "C^L too large");
+    if (g->format != ZHA_SUMMARY_F16X2 && g->format != ZHA_SUMMARY_BF16)
+        return fail(ZHA_ERR_ARG, "format must be ZHA_SUMMARY_F16X2 or ZHA_SUMMARY_BF16");
     return ZHA_OK;
 }
 
@@ -148,7 +153,7 @@ extern "C" zha_status zha_tree_create(const zha_geometry* g, zha_tree** out) {
     zha_tree* t = new zha_tree();
     memset(t, 0, sizeof(*t));
     t->g = *g;
-    t->ns = record_stride(g->R, g->d);
+    t->ns = record_stride(g->R, g->d, g->format);
     size_t off = 0;
     size_t rec_off[kMaxL + 1] = {0}, lse_off[kMaxL + 1] = {0};
     for (int l = 1; l <= g->L; ++l) {
@@ -215,6 +220,7 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
     ba.R = g.R;
     ba.C = C;
     ba.ns = t->ns;
+    ba.fmt = g.format;
     ba.scale = score_scale(g.d);
     for (int l = 1; l <= L; ++l) {
         ba.rec[l] = t->rec[l];
@@ -231,6 +237,7 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
         ma.R = g.R;
         ma.C = C;
         ma.ns = t->ns;
+        ma.fmt = g.format;
         ma.p0 = lo;
         ma.np = hi - lo;
         ma.scale = score_scale(g.d);
@@ -243,6 +250,42 @@ static zha_status run_levels(zha_tree* t, const void* K, int64_t n_old, int64_t 
         ZHA_CUDA(launch_merge(ma, g.d, st));
         return ZHA_OK;
     };
+    if (build_tc_supported(C, g.R, g.d, g.format)) {
+        // levels 1..3 on the tensor cores, over whole 128-token tiles holding a new chunk (the
+        // tile's other nodes are rewritten with the same bits); the levels above by merges
+        const int k_emit = std::min(3, L);
+        const int64_t lo = n_old / C, hi = n_new / C;
+        if (hi > lo) {
+            BuildTcArgs ta;
+            memset(&ta, 0, sizeof(ta));
+            ta.K = static_cast<const __nv_bfloat16*>(K);
+            ta.ld = g.capacity;
+            ta.n_tokens = n_new;
+            ta.qref = t->qref;
+            ta.rflag = t->rflag;
+            ta.Hkv = g.n_kv_heads;
+            ta.ns = t->ns;
+            ta.k_emit = k_emit;
+            ta.t0 = lo / 32;
+            ta.t1 = (hi - 1) / 32 + 1;
+            ta.n1 = n_new / C;
+            ta.n2 = n_new / (C * C);
+            ta.n3 = n_new / (C * C * C);
+            ta.scale = score_scale(g.d);
+            for (int l = 1; l <= k_emit; ++l) {
+                ta.rec[l] = t->rec[l];
+                ta.lse[l] = t->lse[l];
+                ta.cap[l] = t->cap[l];
+            }
+            ZHA_CUDA(launch_build_tc(ta, g.d, st));
+        }
+        for (int l = k_emit + 1; l <= L; ++l) {
+            const int64_t span = ipow(C, l);
+            zha_status s2 = merge(l, n_old / span, n_new / span);
+            if (s2 != ZHA_OK) return s2;
+        }
+        return ZHA_OK;
+    }
     int first_merge = 2;
     int64_t lo1 = n_old / C;
     if (n_old == 0) {
@@ -323,11 +366,11 @@ extern "C" zha_status zha_tree_export(const zha_tree* t, int32_t level, float* m
     const int64_t nl = t->n_tokens / ipow(g.C, level);
     if (nl == 0) return ZHA_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (m) ZHA_CUDA(launch_export_m(t->rec[level], t->cap[level], t->ns, g.n_kv_heads, g.R, g.d, nl, m, st));
+    if (m) ZHA_CUDA(launch_export_m(t->rec[level], t->cap[level], t->ns, g.n_kv_heads, g.R, g.d, g.format, nl, m, st));
     for (int h = 0; h < g.n_kv_heads; ++h) {
         const float* src = t->rec[level] + (int64_t)h * t->cap[level] * t->ns;
         if (b)
-            ZHA_CUDA(cudaMemcpy2DAsync(b + (int64_t)h * nl * g.R, (size_t)g.R * 4, src + (int64_t)g.R * g.d,
+            ZHA_CUDA(cudaMemcpy2DAsync(b + (int64_t)h * nl * g.R, (size_t)g.R * 4, src + b_offset(g.R, g.d, g.format),
                                        (size_t)t->ns * 4, (size_t)g.R * 4, (size_t)nl,
                                        cudaMemcpyDeviceToDevice, st));
         if (lse)
@@ -348,8 +391,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
         if (!trees[s]) return fail(ZHA_ERR_ARG, "a tree is NULL");
         const zha_geometry& a = trees[s]->g;
         const zha_geometry& b0 = trees[0]->g;
-        if (a.d != b0.d || a.n_q_heads != b0.n_q_heads || a.n_kv_heads != b0.n_kv_heads)
-            return fail(ZHA_ERR_ARG, "trees of one decoder must share d, n_q_heads and n_kv_heads");
+        if (a.d != b0.d || a.n_q_heads != b0.n_q_heads || a.n_kv_heads != b0.n_kv_heads || a.format != b0.format)
+            return fail(ZHA_ERR_ARG, "trees of one decoder must share d, n_q_heads, n_kv_heads and format");
     }
     zha_decoder* dec = new zha_decoder();
     dec->trees.assign(trees, trees + n_seq);
@@ -470,7 +513,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
             const zha_tree* t = dec->trees[s];
             for (int l = 1; l <= t->g.L && ok; ++l)
                 ok = encode_level_maps(&maps[((size_t)s * (kMaxL + 1) + l) * kMapsPerLevel], t->rec[l], t->g.d, t->g.R,
-                                       (int64_t)t->g.n_kv_heads * t->cap[l], t->ns);
+                                       (int64_t)t->g.n_kv_heads * t->cap[l], t->ns, t->g.format);
         }
         if (ok) {
             CUtensorMap* dst = reinterpret_cast<CUtensorMap*>(base + tmap_off);
@@ -564,6 +607,7 @@ static zha_status fill_seqs(zha_decoder* dec, const void* const* K, const void* 
         sd.L = t->g.L;
         sd.R = t->g.R;
         sd.ns = t->ns;
+        sd.fmt = t->g.format;
         sd.N = t->n_tokens;
         sd.top = ipow(t->g.C, t->g.L);
         sd.T = sd.N / sd.top;
@@ -597,6 +641,7 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     b.score_path = dec->score_path;
     b.attn_path = dec->attn_path;
     b.all_r16 = dec->all_r16;
+    b.fmt = dec->trees[0]->g.format;
     b.split_tok = decoder_split_tokens(b.n_gl);
     return b;
 }
@@ -804,7 +849,7 @@ extern "C" zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats
     out->union_tokens = (int64_t)ctr[kCtrUnionTokens];
     out->lane_tokens = (int64_t)ctr[kCtrLaneTokens];
     const zha_geometry& g = dec->trees[0]->g;
-    out->node_bytes = (int64_t)(g.R * g.d + g.R) * 4;
+    out->node_bytes = scored_node_bytes(g.R, g.d, g.format);
     out->status = status;
     return status ? fail(ZHA_ERR_DEVICE, "device status word is set") : ZHA_OK;
 }

@@ -48,9 +48,22 @@ __device__ __forceinline__ float quad_sum(float v) {
     return v;
 }
 
-// m values of plane r held by thread quarter q (dims 16 i + 4 q + c) of a stored record.
+// m values of slope r held by thread quarter q (dims 16 i + 4 q + c) of a stored record.
 template <int D>
-__device__ __forceinline__ void load_row_m(const float* rec, int R, int r, int q, float (&v)[D / 4]) {
+__device__ __forceinline__ void load_row_m(const float* rec, int R, int r, int q, float (&v)[D / 4], int fmt) {
+    if (fmt == kFmtBf16) {
+        const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(rec) + (int64_t)r * D;
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(p + 16 * i + 4 * q));
+            const float2 x = m_decode_bf16(u.x), y = m_decode_bf16(u.y);
+            v[4 * i + 0] = x.x;
+            v[4 * i + 1] = x.y;
+            v[4 * i + 2] = y.x;
+            v[4 * i + 3] = y.y;
+        }
+        return;
+    }
     const __half* h = reinterpret_cast<const __half*>(rec);
 #pragma unroll
     for (int i = 0; i < D / 16; ++i) {
@@ -65,18 +78,19 @@ __device__ __forceinline__ void load_row_m(const float* rec, int R, int r, int q
 }
 
 // Turn a running state into the stored summary of one node and write it:
-// m_r = acc / z (stored as fp16 hi + lo planes), lse_r = mx + log z, b_r = lse_r - s q_r.m_r
-// with the stored m.  Returns lse_r; the stored m (decoded) is left in `m` so the parent
-// folds exactly what a merge from the record would read.
+// m_r = acc / z (stored in the tree's format: fp16 hi + lo planes, or one bf16 plane),
+// lse_r = mx + log z, b_r = lse_r - s q_r.m_r with the stored m.  Returns lse_r; the stored m
+// (decoded) is left in `m` so the parent folds exactly what a merge from the record would read.
 template <int D>
 __device__ __forceinline__ float finalize_store(float mx, float z, const float (&acc)[D / 4],
                                                 const float (&qv)[D / 4], float scale, float* rec,
                                                 float* lse, int r, int q, int R, bool store, int32_t* rflag,
-                                                float (&m)[D / 4]) {
+                                                float (&m)[D / 4], int fmt) {
     const float inv = 1.0f / z;
     float qm = 0.0f;
     bool bad = false;
     __half* hp = reinterpret_cast<__half*>(rec);
+    __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(rec);
 #pragma unroll
     for (int i = 0; i < D / 16; ++i) {
         float a[4];
@@ -85,24 +99,36 @@ __device__ __forceinline__ float finalize_store(float mx, float z, const float (
             a[c] = acc[4 * i + c] * inv;
             bad |= !(fabsf(a[c]) < 65504.0f);
         }
-        uint32_t h0, l0, h1, l1;
-        m_encode2(a[0], a[1], h0, l0, m[4 * i], m[4 * i + 1]);
-        m_encode2(a[2], a[3], h1, l1, m[4 * i + 2], m[4 * i + 3]);
+        if (fmt == kFmtBf16) {
+            const __nv_bfloat162 b0 = __floats2bfloat162_rn(a[0], a[1]), b1 = __floats2bfloat162_rn(a[2], a[3]);
+            const float2 f0 = __bfloat1622float2(b0), f1 = __bfloat1622float2(b1);
+            m[4 * i] = f0.x;
+            m[4 * i + 1] = f0.y;
+            m[4 * i + 2] = f1.x;
+            m[4 * i + 3] = f1.y;
+            if (store)
+                *reinterpret_cast<uint2*>(bp + (int64_t)r * D + 16 * i + 4 * q) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        } else {
+            uint32_t h0, l0, h1, l1;
+            m_encode2(a[0], a[1], h0, l0, m[4 * i], m[4 * i + 1]);
+            m_encode2(a[2], a[3], h1, l1, m[4 * i + 2], m[4 * i + 3]);
+            if (store) {
+                *reinterpret_cast<uint2*>(hp + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(h0, h1);
+                *reinterpret_cast<uint2*>(hp + (int64_t)R * D + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(l0, l1);
+            }
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) qm = fmaf(qv[4 * i + c], m[4 * i + c], qm);
-        if (store) {
-            *reinterpret_cast<uint2*>(hp + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(h0, h1);
-            *reinterpret_cast<uint2*>(hp + (int64_t)R * D + (int64_t)r * D + 16 * i + 4 * q) = make_uint2(l0, l1);
-        }
     }
     qm = quad_sum(qm);
     const float l = mx + logf(z);
     if (store) {
         if (q == 0) {
-            rec[(int64_t)R * D + r] = fmaf(-scale, qm, l);
+            rec[b_offset(R, D, fmt) + r] = fmaf(-scale, qm, l);
             lse[r] = l;
         }
-        if (bad) atomicOr(rflag, 1);
+        if (bad && fmt != kFmtBf16) atomicOr(rflag, 1);   // bf16 holds every finite f32 range
     }
     return l;
 }
@@ -278,7 +304,7 @@ __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
                 const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
                                                    a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
                                                    a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
-                                                   active, a.rflag, m1);
+                                                   active, a.rflag, m1, a.fmt);
                 if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
                 mx = -INFINITY;
                 z = 0.0f;
@@ -296,7 +322,7 @@ __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
                     const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
                                                        a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
                                                        a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
-                                                       active, a.rflag, ml);
+                                                       active, a.rflag, ml, a.fmt);
                     if (l < a.k_emit)
                         fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
                     reset_smem<D>(st, stride);
@@ -333,24 +359,24 @@ __global__ void __launch_bounds__(128) k_merge(MergeArgs a) {
 #pragma unroll
     for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
     for (int c = 0; c < a.C; ++c) {
-        load_row_m<D>(crec + (int64_t)c * a.ns, a.R, r, q, mc);
+        load_row_m<D>(crec + (int64_t)c * a.ns, a.R, r, q, mc, a.fmt);
         const float lc = __ldg(clse + (int64_t)c * a.R + r);
         fold_child<D>(mx, z, acc, lc, mc);
     }
     finalize_store<D>(mx, z, acc, qv, a.scale, a.rec + ((int64_t)g * a.cap + P) * a.ns,
-                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, a.rflag, mo);
+                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, a.rflag, mo, a.fmt);
 }
 
 // Decodes the m planes of nodes [0, n) of every KV head into f32 [Hkv][n][R][d].
-__global__ void k_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
-                           float* m) {
+__global__ void k_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int32_t fmt,
+                           int64_t n, float* m) {
     const int64_t per = (int64_t)R * d / 4;   // float4 per node
     const int64_t total = (int64_t)Hkv * n * per;
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
         const int64_t node = t / per, e4 = t % per;
         const int64_t h = node / n, j = node % n;
         const int r = (int)(e4 * 4 / d), k = (int)(e4 * 4 % d);
-        const float4 v = m_load4(rec + (h * cap + j) * ns, R, d, r, k);
+        const float4 v = m_load4(rec + (h * cap + j) * ns, R, d, r, k, fmt);
         reinterpret_cast<float4*>(m)[t] = v;
     }
 }
@@ -362,12 +388,12 @@ int workers_per_block(int R) {
 
 }  // namespace
 
-cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
-                            float* m, cudaStream_t st) {
+cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int32_t fmt,
+                            int64_t n, float* m, cudaStream_t st) {
     const int64_t total = (int64_t)Hkv * n * R * d / 4;
     if (total <= 0) return cudaSuccess;
     const int64_t blocks = std::min<int64_t>((total + 255) / 256, sm_count() * 16);
-    k_export_m<<<(unsigned)blocks, 256, 0, st>>>(rec, cap, ns, Hkv, R, d, n, m);
+    k_export_m<<<(unsigned)blocks, 256, 0, st>>>(rec, cap, ns, Hkv, R, d, fmt, n, m);
     return cudaGetLastError();
 }
 

@@ -13,14 +13,29 @@ namespace zha {
 
 constexpr int kMaxL = ZHA_MAX_LEVELS;
 
-// Node record layout in HBM (per level, per KV head, per node): m [R][d] f32 followed by
-// b [R] f32, stride `ns` floats = R*(d+1) rounded up to 8 floats (32-byte sectors).
-// lse [R] f32 is kept in a separate array per level (read only by merges and export).
-inline __host__ __device__ int32_t record_stride(int R, int d) { return ((R * (d + 1) + 7) / 8) * 8; }
+// Node record layout in HBM (per level, per KV head, per node): the R slopes m_r in the tree's
+// summary format, then b [R] f32; stride `ns` floats rounded up to 8 floats (32-byte
+// sectors).  lse [R] f32 is kept in a separate array per level (read by merges and export).
+//   format 0 (ZHA_SUMMARY_F16X2): m as fp16 planes hi [R][d] then lo [R][d] (4 bytes a value)
+//   format 1 (ZHA_SUMMARY_BF16):  m as one bf16 plane [R][d] (2 bytes a value)
+constexpr int kFmtF16x2 = 0;
+constexpr int kFmtBf16 = 1;
+inline __host__ __device__ int32_t record_stride(int R, int d, int fmt = kFmtF16x2) {
+    return fmt == kFmtBf16 ? ((R * d / 2 + R + 7) / 8) * 8 : ((R * (d + 1) + 7) / 8) * 8;
+}
+// Floats from the start of a record to its b values.
+inline __host__ __device__ int64_t b_offset(int R, int d, int fmt) {
+    return fmt == kFmtBf16 ? (int64_t)R * d / 2 : (int64_t)R * d;
+}
+// Bytes a scorer reads per node: the m planes and b.
+inline __host__ __device__ int64_t scored_node_bytes(int R, int d, int fmt) {
+    return (fmt == kFmtBf16 ? (int64_t)R * d * 2 : (int64_t)R * d * 4) + (int64_t)R * 4;
+}
 
 // One sequence of a decode batch, as the kernels see it.
 struct SeqDev {
     int32_t C, L, R, ns;
+    int32_t fmt;                     // summary format of the tree (kFmtF16x2 / kFmtBf16)
     int64_t N;                       // tokens present
     int64_t T;                       // complete top-level nodes = N / C^L
     int64_t top;                     // C^L
@@ -78,6 +93,7 @@ struct Batch {
     int32_t score_path;              // 0 auto, 1 CUDA cores, 2 tensor cores (R = 16 only)
     int32_t attn_path;               // 0 auto, 1 CUDA cores, 2 tensor cores
     int32_t all_r16;                 // every tree of the batch has R = 16
+    int32_t fmt = 0;                 // summary format shared by the batch's trees
     int32_t dense = 0;               // every lane attends every token (no routed sets, no lane masks)
     int32_t split_tok = 0;           // attention split size in tokens (0: split_tokens(n_gl))
 };
@@ -107,8 +123,17 @@ __device__ __forceinline__ float2 m_decode2(uint32_t hi, uint32_t lo) {
     const float2 lf = __half22float2(*reinterpret_cast<const __half2*>(&lo));
     return make_float2(hf.x + lf.x, hf.y + lf.y);
 }
-// Four consecutive m values (dims k..k+3 of plane r) of a record from its two planes.
-__device__ __forceinline__ float4 m_load4(const float* rec, int R, int D, int r, int k) {
+// The same for a one-plane bf16 record: two bf16 values of a 32-bit word.
+__device__ __forceinline__ float2 m_decode_bf16(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+}
+// Four consecutive m values (dims k..k+3 of slope r) of a record in format fmt.
+__device__ __forceinline__ float4 m_load4(const float* rec, int R, int D, int r, int k, int fmt) {
+    if (fmt == kFmtBf16) {
+        const uint2 a = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(rec) + (int64_t)r * D + k);
+        const float2 x = m_decode_bf16(a.x), y = m_decode_bf16(a.y);
+        return make_float4(x.x, x.y, y.x, y.y);
+    }
     const __half* h = reinterpret_cast<const __half*>(rec);
     const uint2 a = *reinterpret_cast<const uint2*>(h + (int64_t)r * D + k);
     const uint2 c = *reinterpret_cast<const uint2*>(h + (int64_t)R * D + (int64_t)r * D + k);
@@ -146,6 +171,12 @@ inline int sm_count() {
         cached[dev] = n;
     }
     return cached[dev];
+}
+
+// A tree's flag word as routing reports it: bit 0, a summary left the fp16 range (kStatusRange);
+// bit 1, a wait of the tensor-core build gave up (kStatusTimeout: the tree is incomplete).
+__device__ __forceinline__ void tree_flag_status(int32_t flag, int32_t* status) {
+    if (flag) atomicOr(status, ((flag & 1) ? kStatusRange : 0) | ((flag & 2) ? kStatusTimeout : 0));
 }
 
 // Split size (tokens) of the attention work for a call with n_gl lanes per group.

@@ -17,6 +17,7 @@ struct BuildArgs {
     const __nv_bfloat16* qref;   // [Hkv][R][d]
     int32_t* rflag;              // set when a summary leaves the fp16 range
     int32_t Hkv, R, C, ns, k_emit;
+    int32_t fmt;                 // summary format (kFmtF16x2 / kFmtBf16)
     int64_t u0, nu;
     float scale;
     float* rec[kMaxL + 1];
@@ -29,6 +30,7 @@ struct MergeArgs {
     const __nv_bfloat16* qref;
     int32_t* rflag;
     int32_t Hkv, R, C, ns;
+    int32_t fmt;
     int64_t p0, np;
     float scale;
     const float* child_rec;
@@ -39,11 +41,29 @@ struct MergeArgs {
     int64_t cap;
 };
 
+// Tensor-core build (C = 4, R = 16, d = 64 or 128): tiles [t0, t1) of 128 tokens of every KV
+// head; writes every complete node of levels 1..k_emit (k_emit <= 3) whose tokens lie in them.
+struct BuildTcArgs {
+    const __nv_bfloat16* K;      // [Hkv][ld][d]
+    int64_t ld, n_tokens;        // rows of the cache valid for this call
+    const __nv_bfloat16* qref;   // [Hkv][R][d]
+    int32_t* rflag;              // bit 0: a summary left the fp16 range; bit 1: a wait gave up
+    int32_t Hkv, ns, k_emit;
+    int64_t t0, t1;
+    int64_t n1, n2, n3;          // complete nodes of levels 1..3 (n_tokens / C^l)
+    float scale;
+    float* rec[4];
+    float* lse[4];
+    int64_t cap[4];
+};
+
 cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st);
+bool build_tc_supported(int C, int R, int d, int fmt);
+cudaError_t launch_build_tc(const BuildTcArgs& a, int d, cudaStream_t st);
 cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st);
 // m of nodes [0, n) of every KV head of one level, decoded to f32 [Hkv][n][R][d].
-cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int64_t n,
-                            float* m, cudaStream_t st);
+cudaError_t launch_export_m(const float* rec, int64_t cap, int32_t ns, int32_t Hkv, int32_t R, int32_t d, int32_t fmt,
+                            int64_t n, float* m, cudaStream_t st);
 
 // Decode (routing + attention).  `it` is the level iteration: sequence s works on level
 // L_s - it.  mode 0 of the union kernel prepares routing iteration it (union of the kept

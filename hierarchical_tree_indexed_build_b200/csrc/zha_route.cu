@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
 // Warp = 8 lanes x 4 quarter-threads; thread (lane, quarter) keeps its lane's query
 // dimensions {16 i + 4 quarter + c} in registers.  WB warps split a block of 8*WB lanes,
 // 8/WB node slots run concurrently.  Each node record is read with 16-byte loads.
-template <int D>
+template <int D, bool BF>
 __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float scale) {
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
     const int64_t nc = top ? sq.T : (int64_t)w.ucount[grp] * C;
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
-        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+        tree_flag_status(*sq.rflag, w.status);
     }
     if (nc == 0) return;
     const int WB = min(8, (b.n_gl + 7) / 8);
@@ -268,15 +268,23 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
         const float* rec = base + j * ns;
         const __half* rh = reinterpret_cast<const __half*>(rec);
         float best = -INFINITY;
+        const float* brow = rec + (BF ? (int64_t)R * D / 2 : (int64_t)R * D);
         for (int r = 0; r < R; ++r) {
-            const uint2* hrow = reinterpret_cast<const uint2*>(rh + (int64_t)r * D);
+            const uint2* hrow = reinterpret_cast<const uint2*>(rh + (int64_t)r * D);   // also the bf16 plane
             const uint2* lrow = reinterpret_cast<const uint2*>(rh + (int64_t)R * D + (int64_t)r * D);
             float dot = 0.0f;
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) {
-                const uint2 hv = __ldg(hrow + 4 * i + q), lv = __ldg(lrow + 4 * i + q);
-                const float2 m01 = m_decode2(hv.x, lv.x), m23 = m_decode2(hv.y, lv.y);
-                const float4 m = make_float4(m01.x, m01.y, m23.x, m23.y);
+                float4 m;
+                if constexpr (BF) {
+                    const uint2 hv = __ldg(hrow + 4 * i + q);
+                    const float2 m01 = m_decode_bf16(hv.x), m23 = m_decode_bf16(hv.y);
+                    m = make_float4(m01.x, m01.y, m23.x, m23.y);
+                } else {
+                    const uint2 hv = __ldg(hrow + 4 * i + q), lv = __ldg(lrow + 4 * i + q);
+                    const float2 m01 = m_decode2(hv.x, lv.x), m23 = m_decode2(hv.y, lv.y);
+                    m = make_float4(m01.x, m01.y, m23.x, m23.y);
+                }
                 dot = fmaf(qv[4 * i], m.x, dot);
                 dot = fmaf(qv[4 * i + 1], m.y, dot);
                 dot = fmaf(qv[4 * i + 2], m.z, dot);
@@ -284,7 +292,7 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
             }
             dot += __shfl_xor_sync(kFull, dot, 1);
             dot += __shfl_xor_sync(kFull, dot, 2);
-            best = fmaxf(best, fmaf(scale, dot, __ldg(rec + (int64_t)R * D + r)));
+            best = fmaxf(best, fmaf(scale, dot, __ldg(brow + r)));
         }
         if (lane_ok && q == 0) {
             bool mb = true;
@@ -313,7 +321,7 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
 // k_score: e = max_r (s q.m_r + b_r), -inf off the lane's frontier, in candidate order.
 constexpr int kFewLanes = 16;
 
-template <int D>
+template <int D, bool BF>
 __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, float scale) {
     constexpr int kHalf = D / 2;      // dims per thread
     constexpr int kV = kHalf / 8;     // 16-byte pieces per plane per thread
@@ -330,7 +338,7 @@ __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, f
     const int64_t nc = top ? sq.T : (int64_t)w.ucount[grp] * C;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
-        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+        tree_flag_status(*sq.rflag, w.status);
     }
     if (nc == 0) return;
     const int nl = b.n_gl;            // <= kFewLanes (checked by the launcher)
@@ -356,23 +364,28 @@ __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, f
         const int64_t j = top ? k : (int64_t)__ldg(ul + k / C) * C + k % C;
         const float* rec = base + j * ns;
         const __half* rh = reinterpret_cast<const __half*>(rec);
-        const uint4* hp = reinterpret_cast<const uint4*>(rh + (int64_t)r * D + hf * kHalf);
+        const uint4* hp = reinterpret_cast<const uint4*>(rh + (int64_t)r * D + hf * kHalf);   // also the bf16 plane
         const uint4* lp = reinterpret_cast<const uint4*>(rh + (int64_t)R * D + (int64_t)r * D + hf * kHalf);
         uint4 hv[kV], lv[kV];
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             hv[v] = __ldg(hp + v);
-            lv[v] = __ldg(lp + v);
+            if constexpr (!BF) lv[v] = __ldg(lp + v);
         }
-        const float br = __ldg(rec + (int64_t)R * D + r);
+        const float br = __ldg(rec + (BF ? (int64_t)R * D / 2 : (int64_t)R * D) + r);
         float m[kHalf];
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             const uint32_t hw[4] = {hv[v].x, hv[v].y, hv[v].z, hv[v].w};
-            const uint32_t lw[4] = {lv[v].x, lv[v].y, lv[v].z, lv[v].w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const float2 f = m_decode2(hw[c], lw[c]);
+                float2 f;
+                if constexpr (BF) {
+                    f = m_decode_bf16(hw[c]);
+                } else {
+                    const uint32_t lw[4] = {lv[v].x, lv[v].y, lv[v].z, lv[v].w};
+                    f = m_decode2(hw[c], lw[c]);
+                }
                 m[8 * v + 2 * c] = f.x;
                 m[8 * v + 2 * c + 1] = f.y;
             }
@@ -913,17 +926,24 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
         // the few-lane kernel is validated on; d = 64 takes k_score)
         const int bx = std::max(1, 2 * sm_count() / std::max(1, b.n_groups));
         ProfScope ps_("k_score", st);
-        k_score_few<128><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        if (b.fmt == kFmtBf16)
+            k_score_few<128, true><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        else
+            k_score_few<128, false><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
         return cudaGetLastError();
     }
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
     dim3 grid(score_blocks_x(lane_blocks, b.n_groups), lane_blocks, b.n_groups);
     ProfScope ps_("k_score", st);
-    if (b.d == 128)
-        k_score<128><<<grid, 256, 0, st>>>(b, w, it, scale);
-    else
-        k_score<64><<<grid, 256, 0, st>>>(b, w, it, scale);
+    const bool bf = b.fmt == kFmtBf16;
+    if (b.d == 128) {
+        if (bf) k_score<128, true><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else k_score<128, false><<<grid, 256, 0, st>>>(b, w, it, scale);
+    } else {
+        if (bf) k_score<64, true><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else k_score<64, false><<<grid, 256, 0, st>>>(b, w, it, scale);
+    }
     return cudaGetLastError();
 }
 

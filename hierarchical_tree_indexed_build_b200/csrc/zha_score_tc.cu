@@ -42,7 +42,7 @@
 
 namespace zha {
 
-size_t score_tc_smem_lt(int d, int lt);
+size_t score_tc_smem_lt(int d, int lt, int planes);
 
 namespace {
 
@@ -50,7 +50,7 @@ constexpr int kTileM = 128;          // lanes per tile (MMA M)
 constexpr int kTileN = 128;          // rows (node, plane) per tile (MMA N)
 constexpr int kR = 16;               // planes per node on this path
 constexpr int kNodes = kTileN / kR;  // nodes per tile
-constexpr int kPlanes = 2;           // fp16 terms of m
+// planes of m per record: two fp16 terms (hi, lo) or one bf16 plane
 constexpr float kHalfMax = 65504.0f; // largest finite fp16
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
 
@@ -69,17 +69,21 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: kind::f16 with fp16 A/B, f32 accumulate, both K-major, M x N.
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+// Instruction descriptor: kind::f16 with fp16 (or, with bf, bf16) A/B, f32 accumulate, both
+// K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_score(bool bf) {
+    return (1u << 4) | (bf ? (1u << 7) | (1u << 10) : 0u) | ((uint32_t)(kTileN >> 3) << 17) |
+           ((uint32_t)(kTileM >> 4) << 24);
+}
 
 // D (tensor memory) = or += A (tensor memory) x B (shared memory descriptor)
-__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t acc) {
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t id, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
         :
-        : "r"(tmem_d), "r"(tmem_a), "l"(b), "r"(kIdesc), "r"(acc));
+        : "r"(tmem_d), "r"(tmem_a), "l"(b), "r"(id), "r"(acc));
 }
 
 // Writes 32 consecutive 32-bit columns of this thread's tensor-memory lane.
@@ -296,13 +300,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
 
 constexpr int kStages = 3;           // shared-memory stages of node tiles
 
-template <int D, int LT>
+template <int D, int LT, bool BF>
 __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, int it, float scale) {
+    constexpr int kPlanes = BF ? 1 : 2;
     constexpr int kEpilogue = 128 * LT;
     constexpr int kLW = 4 * LT;                       // 32-lane membership words per CTA
-    constexpr int KB = D / 64;                        // 128-byte K blocks of fp16
-    constexpr int P_BYTES = KB * kTileN * 128;        // one fp16 plane of one stage
+    constexpr int KB = D / 64;                        // 128-byte K blocks of 16-bit values
+    constexpr int P_BYTES = KB * kTileN * 128;        // one plane of one stage
     constexpr int STAGE = kPlanes * P_BYTES;
+    constexpr uint32_t kId = idesc_score(BF);
+    constexpr int kBOff = BF ? kR * D / 2 : kR * D;   // floats from a record to its b values
     constexpr int kAcc = 3;                           // accumulator slots (columns 0, 128, 256)
     constexpr uint32_t kColA = kAcc * kTileN;         // queries after the accumulators
     constexpr uint32_t kCols = 512;
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     const int nc = (int)(top ? sq.T : (int64_t)w.ucount[grp] * C);   // < 2^31: level-1 nodes <= 2^24
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         atomicAdd(&w.ctr[kCtrUnionNodes + lev], (unsigned long long)nc);
-        if (*sq.rflag) atomicOr(w.status, kStatusRange);
+        tree_flag_status(*sq.rflag, w.status);
     }
     const int ntiles = (nc + kNodes - 1) / kNodes;
     if ((int)blockIdx.x >= ntiles) return;          // whole block leaves before any barrier
@@ -368,8 +375,8 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
     const int row = lt * kTileM + quad * 32 + lane;
     const uint32_t tlane = (uint32_t)(quad * 32) << 16;
     if (warp >= 2) {
-        // A: this lane's query row (bf16 -> fp16, exact in range) into tensor memory; zero
-        // rows past the group's lanes
+        // A: this lane's query row into tensor memory - as fp16 (exact in range) against
+        // fp16 planes, as its own bf16 bits against a bf16 plane; zero rows past the group's lanes
         const int y = y0 + row;
         const uint4* qp = reinterpret_cast<const uint4*>(b.Q + lane_of(b, s, g, y < b.n_gl ? y : 0) * D);
         float amax = 0.0f;
@@ -383,10 +390,14 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                 const uint32_t* bv = &v.x;
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(bv + t));
-                    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-                    const __half2 hh = __floats2half2_rn(f.x, f.y);
-                    hv[c * 4 + t] = *reinterpret_cast<const uint32_t*>(&hh);
+                    if constexpr (BF) {
+                        hv[c * 4 + t] = bv[t];
+                    } else {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(bv + t));
+                        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                        const __half2 hh = __floats2half2_rn(f.x, f.y);
+                        hv[c * 4 + t] = *reinterpret_cast<const uint32_t*>(&hh);
+                    }
                 }
             }
             tmem_st32(tmem + tlane + kColA + (uint32_t)(lt * (D / 2) + h * 32), hv);
@@ -470,7 +481,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                         if (runs)
                             tma_load_2d(smem_u32(sBv + st * kTileN + nl * kR), maps + 2, 0, wn, fb);
                         else
-                            bulk_load(smem_u32(sBv + st * kTileN + nl * kR), recb + (int64_t)wn * sq.ns + kR * D, kR * 4, fb);
+                            bulk_load(smem_u32(sBv + st * kTileN + nl * kR), recb + (int64_t)wn * sq.ns + kBOff, kR * 4, fb);
                     }
                 }
                 __syncwarp();
@@ -513,7 +524,7 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                     const uint32_t a1 = ta + (uint32_t)(kb * 32);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ts(d, a1 + (uint32_t)(kk * 8), b1 + (uint64_t)(kk * 2), (pk | kk) ? 1u : 0u);
+                        mma_f16_ts(d, a1 + (uint32_t)(kk * 8), b1 + (uint64_t)(kk * 2), kId, (pk | kk) ? 1u : 0u);
                 }
                 mma_commit(smem_u32(&bar_acc_full[slot]));
             }
@@ -604,25 +615,28 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
 }
 
-template <int D, int LT>
+template <int D, int LT, bool BF>
 cudaError_t launch_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st, int pairs) {
     int nb = sm_count() / max(1, pairs * b.n_groups);
     nb = nb < 1 ? 1 : nb;
     dim3 grid(nb, pairs, b.n_groups);
-    const size_t smem = score_tc_smem_lt(D, LT);
-    cudaFuncSetAttribute(k_score_tc<D, LT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_score_tc<D, LT><<<grid, 64 + 128 * LT, smem, st>>>(b, w, it, scale);
+    const size_t smem = score_tc_smem_lt(D, LT, BF ? 1 : 2);
+    cudaFuncSetAttribute(k_score_tc<D, LT, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_score_tc<D, LT, BF><<<grid, 64 + 128 * LT, smem, st>>>(b, w, it, scale);
     return cudaGetLastError();
+}
+
+template <int LT, bool BF>
+cudaError_t launch_tc_d(const Batch& b, const Work& w, int it, float scale, cudaStream_t st, int pairs) {
+    return b.d == 128 ? launch_tc<128, LT, BF>(b, w, it, scale, st, pairs) : launch_tc<64, LT, BF>(b, w, it, scale, st, pairs);
 }
 
 }  // namespace
 
-size_t score_tc_smem_lt(int d, int lt) {
-    return (size_t)kStages * kPlanes * (d / 64) * kTileN * 128 + (size_t)kStages * kTileN * 4 +
+size_t score_tc_smem_lt(int d, int lt, int planes) {
+    return (size_t)kStages * planes * (d / 64) * kTileN * 128 + (size_t)kStages * kTileN * 4 +
            (size_t)kStages * kNodes * 4 * lt * 4 + (size_t)kStages * kNodes * 4 + 1024;
 }
-
-size_t score_tc_smem(int d) { return score_tc_smem_lt(d, 2); }
 
 cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaStream_t st) {
     ProfScope ps_("k_member", st);
@@ -642,11 +656,12 @@ cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, 
     }
     ProfScope ps_("k_score_tc", st);
     const int lane_tiles = (b.n_gl + kTileM - 1) / kTileM;
+    const bool bf = b.fmt == kFmtBf16;
     if (lane_tiles >= 2) {
         const int pairs = (lane_tiles + 1) / 2;
-        return b.d == 128 ? launch_tc<128, 2>(b, w, it, scale, st, pairs) : launch_tc<64, 2>(b, w, it, scale, st, pairs);
+        return bf ? launch_tc_d<2, true>(b, w, it, scale, st, pairs) : launch_tc_d<2, false>(b, w, it, scale, st, pairs);
     }
-    return b.d == 128 ? launch_tc<128, 1>(b, w, it, scale, st, 1) : launch_tc<64, 1>(b, w, it, scale, st, 1);
+    return bf ? launch_tc_d<1, true>(b, w, it, scale, st, 1) : launch_tc_d<1, false>(b, w, it, scale, st, 1);
 }
 
 }  // namespace zha

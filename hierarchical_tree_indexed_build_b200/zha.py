@@ -36,10 +36,13 @@ class ZhaError(RuntimeError):
         self.status = status
 
 
+ZHA_SUMMARY_F16X2, ZHA_SUMMARY_BF16 = 0, 1
+
+
 class Geometry(ctypes.Structure):
     _fields_ = [("C", ctypes.c_int32), ("L", ctypes.c_int32), ("R", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
-                ("capacity", ctypes.c_int64)]
+                ("capacity", ctypes.c_int64), ("format", ctypes.c_int32)]
 
 
 class DecodeStats(ctypes.Structure):
@@ -240,8 +243,9 @@ def _need(t: torch.Tensor, dtype, what: str):
 class Tree:
     """A summary tree over one sequence's KV cache (device memory owned by libzha)."""
 
-    def __init__(self, C: int, L: int, R: int, d: int, n_q_heads: int, n_kv_heads: int, capacity: int):
-        self.geom = Geometry(C, L, R, d, n_q_heads, n_kv_heads, capacity)
+    def __init__(self, C: int, L: int, R: int, d: int, n_q_heads: int, n_kv_heads: int, capacity: int,
+                 format: int = ZHA_SUMMARY_F16X2):
+        self.geom = Geometry(C, L, R, d, n_q_heads, n_kv_heads, capacity, format)
         self.handle = zha_tree_create(self.geom)
 
     def close(self):

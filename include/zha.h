@@ -58,6 +58,18 @@ typedef enum zha_status {
     ZHA_ERR_DEVICE = 5     /* a kernel flagged an internal failure in the device status word */
 } zha_status;
 
+/* How a node record stores its R slopes m_r (b, lse and every computation stay f32).
+ * The pages test a router with reduced-precision summaries next to the full one (wqu.guru,
+ * summary bullets: an FP4 router variant); this library offers two formats:
+ *   ZHA_SUMMARY_F16X2  m as two fp16 planes hi + lo (m = hi + lo within 2^-22 |m| + 2^-25):
+ *                      float32-grade summaries, 4 bytes per value.  Keys must stay below
+ *                      65504 in magnitude.  The default.
+ *   ZHA_SUMMARY_BF16   m as one bf16 plane (relative rounding 2^-9): half the bytes every
+ *                      scored node costs, one tensor-core pass per node; routing decisions
+ *                      follow the rounded slopes, so kept sets differ from the float32-grade
+ *                      router's where estimates are close. */
+typedef enum zha_summary_format { ZHA_SUMMARY_F16X2 = 0, ZHA_SUMMARY_BF16 = 1 } zha_summary_format;
+
 /* Tree geometry and the shape of the KV cache it indexes. */
 typedef struct zha_geometry {
     int32_t C;            /* children per node = tokens per level-1 chunk, 2..1024 */
@@ -67,6 +79,7 @@ typedef struct zha_geometry {
     int32_t n_q_heads;    /* query heads Hq (multiple of n_kv_heads) */
     int32_t n_kv_heads;   /* KV heads Hkv; query head h reads KV head h*Hkv/Hq */
     int64_t capacity;     /* rows per KV head of the K/V buffers (max tokens) */
+    int32_t format;       /* zha_summary_format of the node records */
 } zha_geometry;
 
 typedef struct zha_tree zha_tree;        /* per-sequence summary tree (device memory) */
@@ -77,9 +90,10 @@ const char* zha_last_error(void);
 
 /* ------------------------------------------------------------------ tree */
 
-/* Allocates the tree for `g` (levels 1..L at capacity: node records of R*(d+1) f32
- * rounded up to 8 floats, plus lse [R] f32 per node, plus q_ref).  *out receives the
- * handle.  ZHA_ERR_ARG on invalid geometry, ZHA_ERR_CUDA on allocation failure. */
+/* Allocates the tree for `g` (levels 1..L at capacity: node records of the slopes in
+ * g->format plus b [R] f32, rounded up to 8 floats, plus lse [R] f32 per node, plus q_ref).
+ * *out receives the handle.  ZHA_ERR_ARG on invalid geometry, ZHA_ERR_CUDA on allocation
+ * failure. */
 zha_status zha_tree_create(const zha_geometry* g, zha_tree** out);
 
 /* Frees the tree (synchronises the device first).  NULL is accepted. */
@@ -111,9 +125,9 @@ zha_status zha_tree_export(const zha_tree* t, int32_t level, float* m, float* ls
 
 /* ------------------------------------------------------------------ decode */
 
-/* Creates a decoder for a batch of n_seq trees (same d, Hq, Hkv; C, L, R may differ per
- * tree) and up to max_queries query tokens per sequence per call.  Workspace is sized
- * from the trees' capacities; trees must outlive the decoder. */
+/* Creates a decoder for a batch of n_seq trees (same d, Hq, Hkv and summary format; C, L,
+ * R may differ per tree) and up to max_queries query tokens per sequence per call.
+ * Workspace is sized from the trees' capacities; trees must outlive the decoder. */
 zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n_seq, int32_t max_queries,
                               zha_decoder** out);
 zha_status zha_decoder_destroy(zha_decoder* dec);
@@ -151,12 +165,13 @@ zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* c
  * rounding).  ZHA_KERNELS_AUTO picks the tensor cores (tcgen05) when a (sequence, KV
  * head) group has >= 64 lanes - for scoring only if every tree has R = 16 - and the CUDA
  * cores otherwise; SIMT and TENSOR force one kind.
- *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::f16 with Q in fp16 and
- *          each summary split into fp16 hi + lo passes (ZHA_ERR_ARG for TENSOR unless
- *          every tree has R = 16).  The tensor path needs every entry of Q and of the
- *          cache's keys below 65504 in magnitude (the fp16 range); otherwise it sets
- *          bit 8 of the device status word (see zha_decoder_stats) and its plane
- *          estimates are not valid - select SIMT for such data.
+ *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::f16 (ZHA_ERR_ARG for
+ *          TENSOR unless every tree has R = 16).  With ZHA_SUMMARY_F16X2 records Q is
+ *          taken in fp16 and each summary in two passes (hi, lo); the tensor path then
+ *          needs every entry of Q and of the cache's keys below 65504 in magnitude (the
+ *          fp16 range), else it sets bit 8 of the device status word (see
+ *          zha_decoder_stats) and its plane estimates are not valid - select SIMT for such
+ *          data.  With ZHA_SUMMARY_BF16 records Q stays bf16 and one pass is made.
  *   attn   exact attention: CUDA-core split-KV, or tcgen05 kind::f16 (S = Q K^T exact
  *          products, P split into bf16 hi + lo for P V) */
 typedef enum zha_kernels { ZHA_KERNELS_AUTO = 0, ZHA_KERNELS_SIMT = 1, ZHA_KERNELS_TENSOR = 2 } zha_kernels;
@@ -232,7 +247,7 @@ typedef struct zha_decode_stats {
     int64_t lane_nodes[ZHA_MAX_LEVELS];
     int64_t union_tokens;
     int64_t lane_tokens;
-    int64_t node_bytes;                       /* bytes read per scored node (m and b, f32) */
+    int64_t node_bytes;                       /* bytes read per scored node (m planes and b) */
     int32_t status;
 } zha_decode_stats;
 zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats* out, void* stream);

@@ -15,6 +15,11 @@ def pytest_terminal_summary(terminalreporter):
     logged mass / score near-ties) and the output errors, one line each."""
     tl = sys.modules.get("zha_testlib")
     log = getattr(tl, "TIE_LOG", None) if tl else None
+    notes = getattr(tl, "NOTES", None) if tl else None
+    if notes:
+        terminalreporter.section("measured rates")
+        for line in notes:
+            terminalreporter.write_line(line)
     if not log:
         return
     tr = terminalreporter

@@ -46,7 +46,7 @@ def test_build_targets_sm100a_only():
 
 @pytest.mark.parametrize("field,value", [("C", 1), ("C", 2048), ("L", 0), ("L", 17), ("R", 3), ("R", 64),
                                          ("d", 96), ("n_kv_heads", 0), ("n_q_heads", 3), ("capacity", 0),
-                                         ("capacity", 1 << 31)])
+                                         ("capacity", 1 << 31), ("format", 2), ("format", -1)])
 def test_tree_create_rejects_bad_geometry(libzha, field, value):
     g = zha.Geometry(4, 6, 16, 128, 16, 2, 65536)
     setattr(g, field, value)

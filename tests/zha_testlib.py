@@ -40,6 +40,8 @@ TIE_FLOOR = 2
 # max error vs the oracle on the GPU's set, max error end to end); printed as a table at
 # the end of the run (tests/conftest.py), also under -q.
 TIE_LOG: List[tuple] = []
+# Free-form measured rates of the session, printed after that table.
+NOTES: List[str] = []
 
 
 def record(name: str, rep, e1, e2) -> str:
