@@ -130,8 +130,9 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-__device__ __forceinline__ void tld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// Starts the load of 32 consecutive columns of this thread's tensor-memory lane into r; the
+// registers hold the values only after tld_wait().
+__device__ __forceinline__ void tld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -139,8 +140,26 @@ __device__ __forceinline__ void tld32(uint32_t taddr, float (&v)[32]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The same wait, with the loaded registers as its operands, so that no use of them can be
+// scheduled before it.
+__device__ __forceinline__ void tld_wait(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                   "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ void tld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    tld32_issue(taddr, r);
+    tld_wait(r);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -163,10 +182,11 @@ __device__ __forceinline__ void split3_bf16x2(float a, float b, uint32_t (&t)[3]
     }
 }
 
-// log(exp a + exp b), the same bits for (a, b) and (b, a).
+// log(exp a + exp b), the same bits for (a, b) and (b, a).  The fast intrinsics (relative
+// error about 2^-21) are far inside the summaries' 1e-4 bar.
 __device__ __forceinline__ float lse2f(float a, float b) {
     const float m = fmaxf(a, b);
-    return m + logf(expf(a - m) + expf(b - m));
+    return m + __logf(__expf(a - m) + __expf(b - m));
 }
 
 // fp16 hi and lo planes of n consecutive m values at hp / lp (n = 8: 16 bytes each;
@@ -390,14 +410,18 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                 av[c] *= a.scale;
                 mx = fmaxf(mx, av[c]);
             }
-            float z = 0.0f;
+            float z = 0.0f, ev[kC];
 #pragma unroll
-            for (int c = 0; c < kC; ++c) z += expf(av[c] - mx);
-            const float l1 = mx + logf(z);
+            for (int c = 0; c < kC; ++c) {
+                ev[c] = __expf(av[c] - mx);
+                z += ev[c];
+            }
+            const float l1 = mx + __logf(z);
+            const float iz = 1.0f / z;
             float wv[kC], wa = 0.0f;                        // wa = s q_r.m_r = sum_t w_t a_t
 #pragma unroll
             for (int c = 0; c < kC; ++c) {
-                wv[c] = expf(av[c] - l1);
+                wv[c] = ev[c] * iz;
                 wa = fmaf(wv[c], av[c], wa);
             }
             uint32_t t01[3], t23[3];
@@ -417,7 +441,7 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
             const bool st1 = j1 < a.n1, st2 = a.k_emit >= 2 && j2 < a.n2, st3 = a.k_emit >= 3 && j3 < a.n3;
             float l2 = lse2f(l1, __shfl_xor_sync(0xffffffffu, l1, 1));
             l2 = lse2f(l2, __shfl_xor_sync(0xffffffffu, l2, 2));
-            const float w21 = expf(l1 - l2);
+            const float w21 = __expf(l1 - l2);
             float wa2 = w21 * wa;                            // s q_r.m_r of the level-2 node
             wa2 += __shfl_xor_sync(0xffffffffu, wa2, 1);
             wa2 += __shfl_xor_sync(0xffffffffu, wa2, 2);
@@ -429,9 +453,9 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                 const float la0 = sXl[(r * 2 + 0) * 2], la1 = sXl[(r * 2 + 1) * 2];
                 const float lo = __shfl_xor_sync(0xffffffffu, l2, 4);   // this group's other level-2 node
                 l3 = lse2f(lse2f(la0, la1), lse2f(l2, lo));
-                wX0 = expf(la0 - l3);
-                wX1 = expf(la1 - l3);
-                w32 = expf(l2 - l3);
+                wX0 = __expf(la0 - l3);
+                wX1 = __expf(la1 - l3);
+                w32 = __expf(l2 - l3);
                 float y = w32 * wa2;
                 y += __shfl_xor_sync(0xffffffffu, y, 4);
                 wa3 = fmaf(wX0, sXl[(r * 2 + 0) * 2 + 1], wX1 * sXl[(r * 2 + 1) * 2 + 1]) + y;
@@ -447,10 +471,16 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
             __half* r2 = a.k_emit >= 2 ? reinterpret_cast<__half*>(a.rec[2] + ((int64_t)hg * a.cap[2] + j2) * a.ns) : nullptr;
             __half* r3 = lv3 ? reinterpret_cast<__half*>(a.rec[3] + ((int64_t)hg * a.cap[3] + j3) * a.ns) : nullptr;
             const bool lo2 = (c4 & 2) == 0, lo1 = (c4 & 1) == 0;
+            // pieces of 32 columns: the load of piece p + 1 is in flight while piece p is used
+            uint32_t nx[32];
+            tld32_issue(tM, nx);
+            tld_wait(nx);
 #pragma unroll 1
             for (int p = 0; p < D / 32; ++p) {
                 float v[32];
-                tld32(tM + p * 32, v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(nx[k]);
+                if (p + 1 < D / 32) tld32_issue(tM + (p + 1) * 32, nx);
                 if (st1) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
@@ -488,10 +518,15 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                             yy += __shfl_xor_sync(0xffffffffu, yy, 4);
                             m3[k] = fmaf(wX0, x0[k], wX1 * x1[k]) + yy;
                         }
-                        // lanes of node 0 store dims +0..3, lanes of node 1 dims +4..7
-                        if (st3) store_planes<4>(m3 + 4 * P, r3 + r * D + dim + 4 * P, r3 + kR * D + r * D + dim + 4 * P, bad);
+                        // lanes of node 0 store dims +0..3, lanes of node 1 dims +4..7 (static
+                        // offsets: the array stays in registers)
+                        if (st3) {
+                            if (P == 0) store_planes<4>(m3, r3 + r * D + dim, r3 + kR * D + r * D + dim, bad);
+                            else store_planes<4>(m3 + 4, r3 + r * D + dim + 4, r3 + kR * D + r * D + dim + 4, bad);
+                        }
                     }
                 }
+                tld_wait(nx);                                // piece p + 1 has landed
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             mbar_arrive(su32(&bM_empty[w]));
