@@ -642,7 +642,7 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     b.attn_path = dec->attn_path;
     b.all_r16 = dec->all_r16;
     b.fmt = dec->trees[0]->g.format;
-    b.split_tok = decoder_split_tokens(b.n_gl);
+    b.split_tok = attn_on_tensor_cores(b) ? split_tokens(b.n_gl) : decoder_split_tokens(b.n_gl);
     return b;
 }
 

@@ -275,7 +275,7 @@ cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float
     if (max_splits <= 0) return cudaSuccess;
     // the tensor-core kernel's grid holds the splits in y (at most 65,535: caches of up to
     // ~268M tokens); longer caches use the CUDA-core kernel
-    if ((b.attn_path == 2 || (b.attn_path == 0 && b.n_gl >= kTensorAttnMinLanes)) && max_splits <= 65535)
+    if (attn_on_tensor_cores(b) && max_splits <= 65535)
         return launch_attn_tc(b, w, max_splits, scale, st);
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);

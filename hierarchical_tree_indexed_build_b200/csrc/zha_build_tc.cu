@@ -191,6 +191,29 @@ __device__ __forceinline__ float lse2f(float a, float b) {
 
 // fp16 hi and lo planes of n consecutive m values at hp / lp (n = 8: 16 bytes each;
 // n = 4: 8 bytes each); `bad` for |m| >= 65504.
+// One 32-byte store (a whole sector) of 8 32-bit words.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
+// fp16 hi and lo planes of 16 consecutive m values at hp / lp (32 bytes each, 32-byte aligned).
+__device__ __forceinline__ void store_planes16(const float* v, __half* hp, __half* lp, bool& bad) {
+    uint32_t h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __half2 hh = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+        const float2 hf = __half22float2(hh);
+        const __half2 ll = __floats2half2_rn(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+        h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+        l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+        bad |= !(fabsf(v[2 * i]) < 65504.0f) || !(fabsf(v[2 * i + 1]) < 65504.0f);
+    }
+    st_global_v8(hp, h);
+    st_global_v8(lp, l);
+}
+
 template <int n>
 __device__ __forceinline__ void store_planes(const float* v, __half* hp, __half* lp, bool& bad) {
     uint32_t h[n / 2], l[n / 2];
@@ -483,8 +506,8 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                 if (p + 1 < D / 32) tld32_issue(tM + (p + 1) * 32, nx);
                 if (st1) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        store_planes<8>(v + 8 * e, r1 + r * D + p * 32 + 8 * e, r1 + kR * D + r * D + p * 32 + 8 * e, bad);
+                    for (int e = 0; e < 2; ++e)
+                        store_planes16(v + 16 * e, r1 + r * D + p * 32 + 16 * e, r1 + kR * D + r * D + p * 32 + 16 * e, bad);
                 }
                 // level 2: sum over the 4 chunks of w21 * m, reduce-scattered so that lane c4
                 // keeps dims 8 c4 .. 8 c4 + 7 of this piece

@@ -185,8 +185,10 @@ inline __host__ __device__ int64_t segs_per_split(int n_gl, int C) {
     const int64_t s = split_tokens(n_gl) / C;
     return s > 0 ? s : 1;
 }
-// Split size of a decoder call: groups of a few lanes take short splits (more warps in flight
-// over a small kept set); the partials workspace is sized by lanes x splits.
+// Split size of a decoder call: on the CUDA-core attention, groups of a few lanes take short
+// splits (more warps in flight over a small kept set); the tensor-core attention keeps
+// split_tokens (its CTAs gather 128-position tiles, so longer splits amortise each CTA's
+// set-up).  The partials workspace is sized by lanes x splits.
 inline __host__ __device__ int decoder_split_tokens(int n_gl) { return n_gl <= 16 ? 256 : split_tokens(n_gl); }
 inline __host__ __device__ int64_t batch_segs(const Batch& b, int C) {
     const int64_t s = (b.split_tok > 0 ? b.split_tok : split_tokens(b.n_gl)) / C;

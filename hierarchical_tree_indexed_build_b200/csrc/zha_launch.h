@@ -80,8 +80,11 @@ constexpr int kTensorScoreMinLanes = 64;
 cudaError_t launch_select(const Batch& b, const Work& w, int it, int64_t max_cands, cudaStream_t st);
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);
-// Lanes per group from which the automatic choice attends on tensor cores.
-constexpr int kTensorAttnMinLanes = 64;
+// Whether a call's attention runs on the tensor cores: forced, or the automatic choice, which
+// takes them at every lane count (a padded 128-lane tile measured faster than the CUDA-core
+// split-KV kernel even for one query token).  Calls with more than 65,535 splits use the
+// CUDA-core kernel either way.
+inline bool attn_on_tensor_cores(const Batch& b) { return b.attn_path == 2 || b.attn_path == 0; }
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);
 
 // Records the message returned by zha_last_error() on this thread; returns s.

@@ -328,7 +328,8 @@ def test_tensor_core_and_cuda_core_attention_agree(n_q, p):
 
 @needs_cuda
 @pytest.mark.parametrize("geom,n_tokens,n_q,attn", [
-    (inputs.TINY, 4096 + 77, 16, zha.ZHA_KERNELS_AUTO),      # 16 lanes: CUDA-core split-KV
+    (inputs.TINY, 4096 + 77, 16, zha.ZHA_KERNELS_SIMT),      # 16 lanes: CUDA-core split-KV
+    (inputs.TINY, 4096 + 77, 16, zha.ZHA_KERNELS_AUTO),      # 16 lanes, d = 64: tcgen05 with a padded lane tile
     (inputs.DEEP, 3 * 4096 + 1234, 8, zha.ZHA_KERNELS_AUTO),  # 64 lanes per group: tcgen05
     (inputs.DEEP, 3 * 4096 + 1234, 8, zha.ZHA_KERNELS_SIMT),
     (inputs.MID, 2 * 4096 + 700, 3, zha.ZHA_KERNELS_TENSOR),  # 24 lanes: a ragged lane tile on tcgen05
