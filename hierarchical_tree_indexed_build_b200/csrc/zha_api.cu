@@ -118,6 +118,15 @@ struct zha_decoder {
     cudaEvent_t status_ev;
     bool status_pending;     // a copy was enqueued and not yet looked at
     int32_t sync;            // calls wait for their own work and report its status
+    // Sequence-sharded decode (zha_shard_*); sh_world = 0 on a plain decoder.
+    int32_t sh_rank = 0, sh_world = 0;
+    int64_t sh_tok0 = 0;             // global index of the shard's first token
+    unsigned long long* sh_need = nullptr;   // [lanes_cap] (workspace)
+    const void* sh_Q = nullptr;
+    int32_t sh_nq = 0;
+    float sh_p = 1.0f;
+    int32_t sh_level = 0;            // level of the next protocol step (0: attention)
+    int32_t sh_step = -1;            // next step: 0 score, 1 hist, 2 cut, 3 finish, 4 attend, 5 combine; -1 none
 };
 
 extern "C" const char* zha_last_error(void) { return g_err.c_str(); }
@@ -482,6 +491,8 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     off += up256(4);
     const size_t seq_off = off;
     off += up256((size_t)n_seq * sizeof(SeqDev));
+    const size_t need_off = off;
+    off += up256((size_t)dec->lanes_cap * 8);
     cudaError_t e = cudaMalloc(&dec->block, off);
     if (e != cudaSuccess) {
         delete dec;
@@ -502,6 +513,7 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     w.ctr = reinterpret_cast<unsigned long long*>(base + ctr_off);
     w.status = reinterpret_cast<int32_t*>(base + status_off);
     dec->seq_dev = reinterpret_cast<SeqDev*>(base + seq_off);
+    dec->sh_need = reinterpret_cast<unsigned long long*>(base + need_off);
     dec->seq_host.resize(n_seq);
     // TMA maps of the trees' fp16 planes, one per (sequence, level), for the tensor scorer
     w.tmaps = nullptr;
@@ -560,6 +572,7 @@ static std::string status_text(int32_t st) {
     if (st & kStatusCapacity) t += " a union list reached its capacity;";
     if (st & kStatusTimeout) t += " a tensor-core pipeline wait gave up;";
     if (st & kStatusRange) t += " an input or summary outside the fp16 range reached the tensor-core scorer;";
+    if (st & kStatusShardKeys) t += " a sharded cut's boundary bin held more keys than the ranks can exchange;";
     return t;
 }
 
@@ -618,6 +631,7 @@ static zha_status fill_seqs(zha_decoder* dec, const void* const* K, const void* 
             sd.rec[l] = t->rec[l];
         }
         sd.rflag = t->rflag;
+        sd.no_sink = (dec->sh_world > 0 && dec->sh_tok0 != 0) ? 1 : 0;
         if (K) sd.K = static_cast<const __nv_bfloat16*>(K[s]);
         if (V) sd.V = static_cast<const __nv_bfloat16*>(V[s]);
     }
@@ -646,23 +660,32 @@ static Batch make_batch(const zha_decoder* dec, const void* Q, int32_t n_q, floa
     return b;
 }
 
-static zha_status route_impl(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
+// Checks of a routing call and the reset of its workspace (kept bitmaps, counters, status,
+// frontier maxima and sizes).
+static zha_status route_prepare(zha_decoder* dec, const void* Q, int32_t n_q, float p, cudaStream_t st) {
     if (!Q || !aligned16(Q)) return fail(ZHA_ERR_ARG, "Q must be a 16-byte aligned device pointer");
     if (n_q < 1 || n_q > dec->max_q) return fail(ZHA_ERR_CAPACITY, "n_q must be in [1, max_queries]");
     if (!(p > 0.0f) || isnan(p)) return fail(ZHA_ERR_ARG, "p must be > 0");
     zha_status s = fill_seqs(dec, nullptr, nullptr);
     if (s != ZHA_OK) return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     ZHA_CUDA(cudaMemcpyAsync(dec->seq_dev, dec->seq_host.data(), sizeof(SeqDev) * dec->n_seq,
                              cudaMemcpyHostToDevice, st));
-    const Batch b = make_batch(dec, Q, n_q, p);
+    const int64_t n_lanes = (int64_t)dec->n_seq * n_q * dec->Hq;
     for (int l = 1; l <= dec->Lmax; ++l)
-        ZHA_CUDA(cudaMemsetAsync(dec->w.kept[l], 0, (size_t)b.n_lanes * dec->w.W[l] * 4, st));
+        ZHA_CUDA(cudaMemsetAsync(dec->w.kept[l], 0, (size_t)n_lanes * dec->w.W[l] * 4, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.ctr, 0, (size_t)kCtrCount * 8, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.status, 0, 4, st));
     // ordered-bits 0 is below every float; counts start at 0
     ZHA_CUDA(cudaMemsetAsync(dec->w.lane_max, 0, (size_t)(kMaxL + 1) * dec->lanes_cap * 4, st));
     ZHA_CUDA(cudaMemsetAsync(dec->w.lane_cnt, 0, (size_t)(kMaxL + 1) * dec->lanes_cap * 4, st));
+    return ZHA_OK;
+}
+
+static zha_status route_impl(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    zha_status s = route_prepare(dec, Q, n_q, p, st);
+    if (s != ZHA_OK) return s;
+    const Batch b = make_batch(dec, Q, n_q, p);
     const float scale = score_scale(dec->d);
     for (int it = 0; it < dec->Lmax; ++it) {
         if (it > 0) ZHA_CUDA(launch_union(b, dec->w, it, 0, st));
@@ -681,8 +704,14 @@ static zha_status route_impl(zha_decoder* dec, const void* Q, int32_t n_q, float
     return ZHA_OK;
 }
 
+static zha_status refuse_shard(const zha_decoder* dec) {
+    if (dec->sh_world > 0) return fail(ZHA_ERR_STATE, "a shard decoder routes through the zha_shard_* calls");
+    return ZHA_OK;
+}
+
 extern "C" zha_status zha_route(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (refuse_shard(dec) != ZHA_OK) return ZHA_ERR_STATE;
     zha_status s = check_previous(dec);
     if (s != ZHA_OK) return s;
     s = route_impl(dec, Q, n_q, p, stream);
@@ -724,6 +753,7 @@ static zha_status sparse_attn_impl(zha_decoder* dec, const void* const* K, const
 extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* const* V,
                                       const void* Q, int32_t n_q, float* out, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (refuse_shard(dec) != ZHA_OK) return ZHA_ERR_STATE;
     zha_status s = check_previous(dec);
     if (s != ZHA_OK) return s;
     s = sparse_attn_impl(dec, K, V, Q, n_q, out, stream);
@@ -734,6 +764,7 @@ extern "C" zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, co
 extern "C" zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, const void* const* V,
                                      const void* Q, int32_t n_q, float* out, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (refuse_shard(dec) != ZHA_OK) return ZHA_ERR_STATE;
     {
         const zha_status s0 = check_previous(dec);
         if (s0 != ZHA_OK) return s0;
@@ -774,6 +805,7 @@ extern "C" zha_status zha_dense_attn(zha_decoder* dec, const void* const* K, con
 extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const void* const* V,
                                  const void* Q, int32_t n_q, float p, float* out, void* stream) {
     if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (refuse_shard(dec) != ZHA_OK) return ZHA_ERR_STATE;
     zha_status s = check_previous(dec);
     if (s != ZHA_OK) return s;
     s = route_impl(dec, Q, n_q, p, stream);
@@ -781,6 +813,188 @@ extern "C" zha_status zha_decode(zha_decoder* dec, const void* const* K, const v
     s = sparse_attn_impl(dec, K, V, Q, n_q, out, stream);
     if (s != ZHA_OK) return s;
     return finish_call(dec, static_cast<cudaStream_t>(stream));
+}
+
+
+// ------------------------------------------------------------------------------ sharded sequence
+static_assert(ZHA_SHARD_BINS == kShardBins && ZHA_SHARD_KEYS == kShardKeys, "exchange sizes of zha.h");
+static_assert(kStatusShardKeys == 16, "status bit of zha.h");
+//
+// One sequence split over ranks: each level's cut over the union of the ranks' frontiers,
+// taken by k_select in three phases around the caller's collectives (histogram out; cut on
+// the summed histogram with the boundary keys out; finish on every rank's keys).
+
+extern "C" zha_status zha_shard_decoder_create(const zha_tree* tree, int32_t max_queries, int32_t rank,
+                                               int32_t world, int64_t token_offset, zha_decoder** out) {
+    if (!tree) return fail(ZHA_ERR_ARG, "tree is NULL");
+    if (!out) return fail(ZHA_ERR_ARG, "out is NULL");
+    if (world < 1 || rank < 0 || rank >= world) return fail(ZHA_ERR_ARG, "rank must be in [0, world)");
+    const int64_t top = ipow(tree->g.C, tree->g.L);
+    if (token_offset < 0 || token_offset % top != 0)
+        return fail(ZHA_ERR_ARG, "token_offset must be a non-negative multiple of C^L");
+    if ((rank == 0) != (token_offset == 0)) return fail(ZHA_ERR_ARG, "rank 0, and only rank 0, starts at token 0");
+    const zha_tree* one[1] = {tree};
+    zha_decoder* dec = nullptr;
+    const zha_status s = zha_decoder_create(one, 1, max_queries, &dec);
+    if (s != ZHA_OK) return s;
+    dec->sh_rank = rank;
+    dec->sh_world = world;
+    dec->sh_tok0 = token_offset;
+    dec->sh_step = -1;
+    *out = dec;
+    return ZHA_OK;
+}
+
+// The protocol position a call must find, and the exchange pointers it uses.
+static zha_status shard_check(const zha_decoder* dec, int32_t level, int step, const zha_shard_exchange* ex) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (dec->sh_world < 1) return fail(ZHA_ERR_STATE, "not a shard decoder (zha_shard_decoder_create)");
+    if (dec->sh_step != step || dec->sh_level != level)
+        return fail(ZHA_ERR_STATE, "sharded decode call out of order (see the protocol in zha.h)");
+    if (!ex) return fail(ZHA_ERR_ARG, "exchange is NULL");
+    auto ok = [](const void* q) { return q && aligned16(q); };
+    bool good = true;
+    switch (step) {
+        case 0: case 1: good = ok(ex->lane_max) && ok(ex->lane_cnt) && (step == 0 || ok(ex->hist)); break;
+        case 2: good = ok(ex->hist) && ok(ex->keys) && ok(ex->nkeys); break;
+        case 3: good = ok(ex->keys_all) && ok(ex->nkeys_all); break;
+        case 4: good = ok(ex->out) && ok(ex->lse); break;
+        case 5: good = ok(ex->out_all) && ok(ex->lse_all); break;
+        default: break;
+    }
+    if (!good) return fail(ZHA_ERR_ARG, "an exchange buffer this step uses is NULL or not 16-byte aligned");
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_shard_begin(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream) {
+    if (!dec) return fail(ZHA_ERR_ARG, "decoder is NULL");
+    if (dec->sh_world < 1) return fail(ZHA_ERR_STATE, "not a shard decoder (zha_shard_decoder_create)");
+    const zha_tree* t = dec->trees[0];
+    const int64_t top = ipow(t->g.C, t->g.L);
+    if (t->built && dec->sh_rank < dec->sh_world - 1 && t->n_tokens % top != 0)
+        return fail(ZHA_ERR_STATE, "every shard but the last must hold a multiple of C^L tokens");
+    if (t->built && (dec->sh_tok0 + t->n_tokens) / t->g.C > (int64_t(1) << 24))
+        return fail(ZHA_ERR_CAPACITY, "a sharded sequence holds at most 2^24 level-1 nodes");
+    zha_status s = check_previous(dec);
+    if (s != ZHA_OK) return s;
+    s = route_prepare(dec, Q, n_q, p, static_cast<cudaStream_t>(stream));
+    if (s != ZHA_OK) return s;
+    dec->sh_Q = Q;
+    dec->sh_nq = n_q;
+    dec->sh_p = p;
+    dec->sh_level = t->g.L;
+    dec->sh_step = 0;
+    dec->routed = false;
+    return ZHA_OK;
+}
+
+// Work of one select phase of the sharded cut at `level`.
+static Work shard_work(const zha_decoder* dec, int phase, int32_t level, const zha_shard_exchange* ex) {
+    Work w = dec->w;
+    const zha_tree* t = dec->trees[0];
+    w.sh_phase = phase;
+    w.sh_world = dec->sh_world;
+    w.sh_off = dec->sh_tok0 / ipow(t->g.C, level);
+    w.sh_hist = reinterpret_cast<unsigned long long*>(ex->hist);
+    w.sh_keys = reinterpret_cast<unsigned long long*>(ex->keys);
+    w.sh_nkeys = ex->nkeys;
+    w.sh_keys_all = reinterpret_cast<const unsigned long long*>(ex->keys_all);
+    w.sh_nkeys_all = ex->nkeys_all;
+    w.sh_need = dec->sh_need;
+    return w;
+}
+
+extern "C" zha_status zha_shard_score(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream) {
+    zha_status s = shard_check(dec, level, 0, ex);
+    if (s != ZHA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Batch b = make_batch(dec, dec->sh_Q, dec->sh_nq, dec->sh_p);
+    const int it = dec->trees[0]->g.L - level;
+    if (it > 0) ZHA_CUDA(launch_union(b, dec->w, it, 0, st));
+    ZHA_CUDA(launch_score(b, dec->w, it, score_scale(dec->d), st));
+    ZHA_CUDA(launch_shard_lanes(dec->w.lane_max + (int64_t)level * dec->w.lanes_cap,
+                                dec->w.lane_cnt + (int64_t)level * dec->w.lanes_cap, ex->lane_max, ex->lane_cnt,
+                                b.n_lanes, true, st));
+    dec->sh_step = 1;
+    return ZHA_OK;
+}
+
+// One select phase (1, 2 or 3) of the sharded cut at `level`.
+static zha_status shard_select(zha_decoder* dec, int32_t level, int phase, const zha_shard_exchange* ex,
+                               cudaStream_t st) {
+    const Batch b = make_batch(dec, dec->sh_Q, dec->sh_nq, dec->sh_p);
+    const int it = dec->trees[0]->g.L - level;
+    const Work w = shard_work(dec, phase, level, ex);
+    ZHA_CUDA(launch_select(b, w, it, dec->seq_host[0].n[level], st));
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_shard_hist(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream) {
+    zha_status s = shard_check(dec, level, 1, ex);
+    if (s != ZHA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the frontier maxima and sizes over all ranks back into the decoder's arrays
+    ZHA_CUDA(launch_shard_lanes(dec->w.lane_max + (int64_t)level * dec->w.lanes_cap,
+                                dec->w.lane_cnt + (int64_t)level * dec->w.lanes_cap, ex->lane_max, ex->lane_cnt,
+                                (int64_t)dec->sh_nq * dec->Hq, false, st));
+    s = shard_select(dec, level, 1, ex, st);
+    if (s != ZHA_OK) return s;
+    dec->sh_step = 2;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_shard_cut(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream) {
+    zha_status s = shard_check(dec, level, 2, ex);
+    if (s != ZHA_OK) return s;
+    s = shard_select(dec, level, 2, ex, static_cast<cudaStream_t>(stream));
+    if (s != ZHA_OK) return s;
+    dec->sh_step = 3;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_shard_finish(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream) {
+    zha_status s = shard_check(dec, level, 3, ex);
+    if (s != ZHA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = shard_select(dec, level, 3, ex, st);
+    if (s != ZHA_OK) return s;
+    if (level > 1) {
+        dec->sh_level = level - 1;
+        dec->sh_step = 0;
+        return ZHA_OK;
+    }
+    dec->sh_level = 0;
+    dec->sh_step = 4;
+    dec->routed = true;
+    dec->last_n_q = dec->sh_nq;
+    return finish_call(dec, st);
+}
+
+extern "C" zha_status zha_shard_attend(zha_decoder* dec, const void* K, const void* V, const zha_shard_exchange* ex,
+                                       void* stream) {
+    zha_status s = shard_check(dec, 0, 4, ex);
+    if (s != ZHA_OK) return s;
+    s = check_previous(dec);
+    if (s != ZHA_OK) return s;
+    const void* Ks[1] = {K};
+    const void* Vs[1] = {V};
+    dec->w.lse_out = ex->lse;
+    s = sparse_attn_impl(dec, Ks, Vs, dec->sh_Q, dec->sh_nq, ex->out, stream);
+    dec->w.lse_out = nullptr;
+    if (s != ZHA_OK) return s;
+    dec->sh_step = 5;
+    return ZHA_OK;
+}
+
+extern "C" zha_status zha_shard_combine(zha_decoder* dec, const zha_shard_exchange* ex, float* out, void* stream) {
+    zha_status s = shard_check(dec, 0, 5, ex);
+    if (s != ZHA_OK) return s;
+    if (!out || !aligned16(out)) return fail(ZHA_ERR_ARG, "out must be a 16-byte aligned device pointer");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ZHA_CUDA(launch_shard_combine(ex->out_all, ex->lse_all, (int64_t)dec->sh_nq * dec->Hq, dec->sh_world, dec->d,
+                                  out, st));
+    dec->sh_step = -1;
+    return finish_call(dec, st);
 }
 
 extern "C" zha_status zha_decoder_set_sync(zha_decoder* dec, int32_t on) {

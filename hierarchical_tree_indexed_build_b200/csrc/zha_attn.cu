@@ -49,8 +49,8 @@ __global__ void __launch_bounds__(256) k_attn(Batch b, Work w, float scale) {
     const int64_t T = sq.T, N = sq.N;
     const int64_t tail0 = T * sq.top;
     const int64_t tail = N - tail0;
-    const int has_sink = T >= 1 ? 1 : 0;
-    const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
+    const int has_sink = seq_has_sink(sq);
+    const int64_t nu = T >= 1 ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
     const int64_t SEGS = batch_segs(b, (int)C);
     const int64_t split = blockIdx.x;
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(256) k_attn(Batch b, Work w, float scale) {
                     if (k < nu) {
                         const int64_t j = ul[k];
                         const int64_t t = j * C + off;
-                        tok = t == 0 ? -1 : t;
+                        tok = (t == 0 && has_sink) ? -1 : t;
                         cid = (int32_t)j;
                     } else {
                         const int64_t t = tail0 + (k - nu) * C + off;
@@ -191,6 +191,13 @@ __global__ void __launch_bounds__(256) k_attn(Batch b, Work w, float scale) {
 // order, so the result does not depend on scheduling.
 constexpr int kCombThreads = 256;
 
+// Sum of the warps' weighted denominators, in the order the output's division uses.
+__device__ __forceinline__ float dd_all(const float* s_den, int nw) {
+    float dd = 0.0f;
+    for (int i = 0; i < nw; ++i) dd += s_den[i];
+    return dd;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kCombThreads) k_combine(Batch b, Work w, float* out) {
     constexpr int PR = D + 4;
@@ -208,8 +215,8 @@ __global__ void __launch_bounds__(kCombThreads) k_combine(Batch b, Work w, float
     const SeqDev& sq = b.seqs[s];
     const int64_t C = sq.C, T = sq.T;
     const int64_t tail = sq.N - T * sq.top;
-    const int has_sink = T >= 1 ? 1 : 0;
-    const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
+    const int has_sink = seq_has_sink(sq);
+    const int64_t nu = T >= 1 ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
     const int64_t SEGS = batch_segs(b, (int)C);
     const int64_t nsplit = (nseg + SEGS - 1) / SEGS;
@@ -257,13 +264,19 @@ __global__ void __launch_bounds__(kCombThreads) k_combine(Batch b, Work w, float
             nn += s_num[i][tid];
             dd += s_den[i];
         }
-        out[x * D + tid] = nn / dd;
+        // a lane with no attended token (possible only on one shard of a sharded sequence)
+        // gets 0 and a log-sum-exp of -inf, so that the ranks' combine ignores it
+        out[x * D + tid] = dd > 0.0f ? nn / dd : 0.0f;
     }
     if (tid == 0) {
+        if (w.lse_out) w.lse_out[x] = dd_all(s_den, NW) > 0.0f ? M + logf(dd_all(s_den, NW)) : -INFINITY;
         int64_t a = tail;
-        if (has_sink) {
-            const uint32_t first = w.kept[1][x * w.W[1]];
-            a += 1 + (int64_t)w.kcount[(int64_t)1 * w.lanes_cap + x] * C - (int64_t)(first & 1u);
+        if (T >= 1) {
+            a += (int64_t)w.kcount[(int64_t)1 * w.lanes_cap + x] * C;
+            if (has_sink) {
+                const uint32_t first = w.kept[1][x * w.W[1]];
+                a += 1 - (int64_t)(first & 1u);
+            }
         }
         atomicAdd(&w.ctr[kCtrLaneTokens], (unsigned long long)a);
     }

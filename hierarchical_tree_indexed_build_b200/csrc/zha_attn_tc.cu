@@ -162,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int64_t C = sq.C, T = sq.T, N = sq.N;
     const int64_t tail0 = T * sq.top;
     const int64_t tail = N - tail0;
-    const int has_sink = T >= 1 ? 1 : 0;
-    const int64_t nu = has_sink ? (int64_t)w.ucount[grp] : 0;
+    const int has_sink = seq_has_sink(sq);
+    const int64_t nu = T >= 1 ? (int64_t)w.ucount[grp] : 0;
     const int64_t nseg = has_sink + nu + (tail + C - 1) / C;
     const int64_t SEGS = batch_segs(b, (int)C);
     // grid (lane tiles, splits, groups): the lane tiles of one split run together, so each
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                     if (k < nu) {
                         const int t = ul[k] * (int)C + off;
                         code = k;
-                        if (t != 0) tok = t;
+                        if (t != 0 || !has_sink) tok = t;
                     } else {
                         const int64_t t = tail0 + (int64_t)(k - nu) * C + off;
                         code = -1;

@@ -46,7 +46,13 @@ struct SeqDev {
     const int32_t* rflag;            // tree's range flag: a summary left the fp16 range
     const __nv_bfloat16* K;          // [Hkv][ld][d]
     const __nv_bfloat16* V;
+    int32_t no_sink;                 // 1: token 0 of this tree is not the sequence's first token
+                                     // (a later shard of a sharded sequence): no sink segment
 };
+
+// Whether attention over the tree has the sink segment (token 0, attended every time): the
+// tree holds a complete top node and starts the sequence.
+__host__ __device__ inline int seq_has_sink(const SeqDev& sq) { return (sq.T >= 1 && !sq.no_sink) ? 1 : 0; }
 
 constexpr int kMapsPerLevel = 3;     // planes by 1 node, planes by 4 nodes, b by 4 nodes
 
@@ -80,7 +86,25 @@ struct Work {
     int32_t* lane_cnt;               // [(kMaxL+1)][lanes_cap] frontier size per lane
     unsigned long long* ctr;         // kCtrCount counters
     int32_t* status;                 // device status word (0 = ok)
+    // Sequence-sharded routing (one sequence whose tokens are split over ranks; null / 0 on
+    // every other path).  k_select then runs in one of three phases around the collectives:
+    // 1 writes the lane's mass histogram, 2 cuts on the summed histogram and writes the
+    // boundary bin's keys, 3 finishes the cut on every rank's keys.
+    int32_t sh_phase;                // 0: the whole cut in one kernel
+    int32_t sh_world;                // ranks
+    int64_t sh_off;                  // global index of this rank's first node of the level
+    unsigned long long* sh_hist;     // [lanes][kShardBins] fixed-point bin masses
+    unsigned long long* sh_keys;     // [lanes][kShardKeys] boundary-bin keys (global node ids)
+    int32_t* sh_nkeys;               // [lanes]
+    const unsigned long long* sh_keys_all;   // [world][lanes][kShardKeys]
+    const int32_t* sh_nkeys_all;     // [world][lanes]
+    unsigned long long* sh_need;     // [lanes_cap] mass still needed from the boundary bin
+    float* lse_out;                  // [lanes] log-sum-exp of each lane's attention (or null)
 };
+
+constexpr int kShardBins = 2048;     // histogram bins of the sharded cut (those of k_select)
+constexpr int kShardKeys = 2048;     // boundary-bin keys one rank contributes per lane
+constexpr int kShardMergeKeys = 4096;   // keys of all ranks one lane's finish can sort
 
 // A decode call's shape.
 struct Batch {
@@ -158,6 +182,7 @@ constexpr int32_t kStatusSelectFallbackLimit = 1;
 constexpr int32_t kStatusCapacity = 2;
 constexpr int32_t kStatusTimeout = 4;        // a bounded wait on the tensor-core pipeline gave up
 constexpr int32_t kStatusRange = 8;          // an entry of Q or of a summary exceeds the fp16 range
+constexpr int32_t kStatusShardKeys = 16;     // a sharded cut's boundary bin held more keys than it can exchange
 
 // Streaming multiprocessors of the current device (grids are sized in multiples of it);
 // looked up once per device ordinal.

@@ -87,6 +87,14 @@ cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, fl
 inline bool attn_on_tensor_cores(const Batch& b) { return b.attn_path == 2 || b.attn_path == 0; }
 cudaError_t launch_combine(const Batch& b, const Work& w, float* out, cudaStream_t st);
 
+// Sharded sequence: a level's frontier maximum and size between the decoder's arrays and the
+// exchange (to_exchange: ordered bits -> ordered int32; else back), and the ranks' merge of
+// their attention outputs by log-sum-exp.
+cudaError_t launch_shard_lanes(uint32_t* lane_max, int32_t* lane_cnt, int32_t* ex_max, int32_t* ex_cnt,
+                               int64_t lanes, bool to_exchange, cudaStream_t st);
+cudaError_t launch_shard_combine(const float* out_all, const float* lse_all, int64_t lanes, int world, int d,
+                                 float* out, cudaStream_t st);
+
 // Records the message returned by zha_last_error() on this thread; returns s.
 zha_status set_last_error(zha_status s, const char* msg);
 

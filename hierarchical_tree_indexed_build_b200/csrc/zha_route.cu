@@ -205,10 +205,12 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
     if (threadIdx.x == 0) {
         w.ucount[grp] = base;
         if (mode == 1) {
-            // attended tokens of the group: sink + kept chunks (token 0 once) + tail
+            // attended tokens of the group: sink + kept chunks (token 0 once) + tail; a later
+            // shard of a sharded sequence has no sink and attends its token 0 with chunk 0
             const int64_t tail = sq.N - sq.T * sq.top;
             const int has0 = nwords > 0 ? (int)(uwp[0] & 1u) : 0;
-            atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)(tail + 1 + (int64_t)base * sq.C - has0));
+            const int64_t s0 = sq.no_sink ? 0 : 1;
+            atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)(tail + s0 + (int64_t)base * sq.C - s0 * has0));
         }
     }
 }
@@ -437,6 +439,8 @@ constexpr int64_t kSelSmallCands = 16384;
 constexpr int kNB = 2048;            // bins over (max e - e) * kBinScale
 constexpr float kBinScale = 64.0f;
 constexpr int kCap = 2048;           // boundary-bin candidates sorted in shared memory
+static_assert(kShardBins == kNB && kShardKeys == kCap, "the sharded cut exchanges k_select's own bins and keys");
+static_assert(kShardMergeKeys * 8 <= kNB * 8 + kCap * 8, "the sharded finish sorts in the histogram and key areas");
 constexpr int kUn = 2;               // 128-candidate blocks per warp in flight (gather path)
 constexpr int kPD = 4;               // per-thread prefetch ring depth (cp.async), a power of two
 
@@ -542,11 +546,19 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
     if (lev < 1) return;
     int32_t* kcount = w.kcount + (int64_t)lev * w.lanes_cap + x;
     const int64_t F = w.lane_cnt[(int64_t)lev * w.lanes_cap + x];
-    if (threadIdx.x == 0) atomicAdd(&w.ctr[kCtrLaneNodes + lev], (unsigned long long)F);
+    const int phase = w.sh_phase;
+    if (threadIdx.x == 0 && phase <= 1) atomicAdd(&w.ctr[kCtrLaneNodes + lev], (unsigned long long)F);
     if (F == 0) {
-        if (threadIdx.x == 0) *kcount = 0;
+        if (threadIdx.x == 0 && phase != 3) {
+            *kcount = 0;
+            if (phase == 2) {
+                w.sh_nkeys[x] = 0;
+                w.sh_need[x] = 0;
+            }
+        }
         return;
     }
+    if (phase == 1 && !(b.p < 1.0f)) return;      // p >= 1 keeps the whole frontier: no histogram
     const float M = unord_bits(w.lane_max[(int64_t)lev * w.lanes_cap + x]);
     SelMath sm;
     sm.nl2M = -M * 1.4426950408889634f;
@@ -563,6 +575,89 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
     uint32_t* outw = w.kept[lev] + x * w.W[lev];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int nblk = (nc + 127) / 128;
+
+    // Sorts kk[0 .. n) by (e desc, j asc) and returns the index of the last key of the
+    // shortest prefix whose mass reaches `need` (n - 1 if none does).  Block-uniform.
+    auto sort_prefix = [&](unsigned long long* kk, int n, unsigned long long need_) -> int {
+        int npow = 1;
+        while (npow < n) npow <<= 1;
+        for (int i = threadIdx.x; i < npow; i += blockDim.x)
+            if (i >= n) kk[i] = ~0ull;
+        __syncthreads();
+        for (int k = 2; k <= npow; k <<= 1) {
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int i = threadIdx.x; i < npow; i += blockDim.x) {
+                    const int ixj = i ^ jj;
+                    if (ixj > i) {
+                        const unsigned long long a0 = kk[i], a1 = kk[ixj];
+                        const bool asc = (i & k) == 0;
+                        if ((a0 > a1) == asc) {
+                            kk[i] = a1;
+                            kk[ixj] = a0;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        const int per = (n + blockDim.x - 1) / blockDim.x;
+        const int i0 = threadIdx.x * per;
+        unsigned long long run = 0;
+        for (int i = i0; i < min(n, i0 + per); ++i) run += sm.mass(key_score(kk[i]));
+        unsigned long long tot;
+        unsigned long long cum = block_excl_scan<unsigned long long>(run, red_u, tot);
+        int found = n;
+        for (int i = i0; i < min(n, i0 + per); ++i) {
+            cum += sm.mass(key_score(kk[i]));
+            if (cum >= need_) {
+                found = i;
+                break;
+            }
+        }
+        found = block_min_t<int>(found, red_i);
+        return found >= n ? n - 1 : found;
+    };
+
+    if (phase == 3) {
+        // sharded cut, last step: every rank's boundary-bin keys (global node ids) for this
+        // lane, sorted together; the prefix reaching the needed mass is the same on every
+        // rank, and each rank sets the bits of its own nodes
+        const unsigned long long need3 = w.sh_need[x];
+        if (need3 == 0) return;
+        int tot = 0;
+        bool over = false;
+        for (int r = 0; r < w.sh_world; ++r) {
+            const int nr = w.sh_nkeys_all[(int64_t)r * b.n_lanes + x];
+            over |= nr > kShardKeys;
+            tot += nr;
+        }
+        if (over || tot > kShardMergeKeys || tot == 0) {
+            if (threadIdx.x == 0) atomicOr(w.status, kStatusShardKeys);
+            return;
+        }
+        unsigned long long* kk = sel_smem;                  // the histogram and key areas: 4,096 keys
+        int o = 0;
+        for (int r = 0; r < w.sh_world; ++r) {
+            const int nr = w.sh_nkeys_all[(int64_t)r * b.n_lanes + x];
+            const unsigned long long* src = w.sh_keys_all + ((int64_t)r * b.n_lanes + x) * kShardKeys;
+            for (int i = threadIdx.x; i < nr; i += blockDim.x) kk[o + i] = src[i];
+            o += nr;
+        }
+        __syncthreads();
+        const int found = sort_prefix(kk, tot, need3);
+        const int64_t own = sq.n[lev];
+        int mine = 0;
+        for (int i = threadIdx.x; i <= found; i += blockDim.x) {
+            const int64_t jl = (int64_t)(uint32_t)kk[i] - w.sh_off;
+            if (jl >= 0 && jl < own) {
+                atomicOr(outw + (jl >> 5), 1u << (jl & 31));
+                ++mine;
+            }
+        }
+        mine = (int)block_sum<unsigned long long>((unsigned long long)mine, red_u);
+        if (threadIdx.x == 0) *kcount += mine;
+        return;
+    }
 
     // candidate k -> node index (shifts when C is a power of two)
     const int cs = (C & (C - 1)) == 0 ? __ffs(C) - 1 : -1;
@@ -698,18 +793,32 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
         }
         if (threadIdx.x == 0) s_nkeys = 0;
         __syncthreads();
-        for_cands(std::false_type{}, [&](int bk, const float4 ev4, int j0) {
-            const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
-            // -inf (off the frontier) gives mass 0 and the last bin: computed without branches,
-            // the atomics are predicated
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t lo, hi;
-                sm.mass2(v[c], lo, hi);
-                hist_add(smem_u32(hlo + sm.bin(v[c])), smem_u32(hhi + sm.bin(v[c])), lo, hi);
+        if (phase == 2) {
+            // sharded cut: the histogram summed over the ranks replaces this rank's own
+            for (int i = threadIdx.x; i < kNB; i += blockDim.x) {
+                const unsigned long long hv = w.sh_hist[x * kShardBins + i];
+                hlo[i] = (uint32_t)hv;
+                hhi[i] = (uint32_t)(hv >> 32);
             }
-        });
+        } else {
+            for_cands(std::false_type{}, [&](int bk, const float4 ev4, int j0) {
+                const float v[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+                // -inf (off the frontier) gives mass 0 and the last bin: computed without
+                // branches, the atomics are predicated
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t lo, hi;
+                    sm.mass2(v[c], lo, hi);
+                    hist_add(smem_u32(hlo + sm.bin(v[c])), smem_u32(hhi + sm.bin(v[c])), lo, hi);
+                }
+            });
+        }
         __syncthreads();
+        if (phase == 1) {
+            // sharded cut, first step: this rank's histogram out, to be summed over the ranks
+            for (int i = threadIdx.x; i < kNB; i += blockDim.x) w.sh_hist[x * kShardBins + i] = hist(i);
+            return;
+        }
         // boundary bin b*: cum(bins < b*) < target <= cum(bins <= b*).  Thread t owns the BPT
         // bins from BPT t; one block-wide exclusive scan of the per-thread sums gives Z and
         // each thread's prefix, and the thread whose range holds the target finds b* there.
@@ -786,7 +895,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 if ((col >> c) & 1u) {
-                    if (idx < (unsigned)kCap) keys[idx] = sel_key(v[c], jof(bk, j0, c));
+                    if (idx < (unsigned)kCap) keys[idx] = sel_key(v[c], (int)(jof(bk, j0, c) + w.sh_off));
                     ++idx;
                 }
         }
@@ -795,52 +904,33 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_select(Batch b, Work w, int i
     });
     cnt = block_sum<unsigned long long>(cnt, red_u);
     if (bstar == kNB) {
-        if (threadIdx.x == 0) *kcount = (int32_t)cnt;
+        if (threadIdx.x == 0) {
+            *kcount = (int32_t)cnt;
+            if (phase == 2) {
+                w.sh_nkeys[x] = 0;
+                w.sh_need[x] = 0;
+            }
+        }
         return;
     }
     __syncthreads();
 
     const unsigned nkeys = s_nkeys;
+    if (phase == 2) {
+        // sharded cut, second step: this rank's boundary-bin keys out, to be gathered from
+        // every rank (more than kShardKeys cannot be exchanged: the last step flags it)
+        const int nk = (int)min(nkeys, (unsigned)kShardKeys);
+        for (int i = threadIdx.x; i < nk; i += blockDim.x) w.sh_keys[x * kShardKeys + i] = keys[i];
+        if (threadIdx.x == 0) {
+            w.sh_nkeys[x] = (int32_t)nkeys;
+            w.sh_need[x] = need;
+            *kcount = (int32_t)cnt;
+        }
+        return;
+    }
     if (nkeys <= (unsigned)kCap) {
         // sort the boundary bin by (e desc, j asc) and take the prefix reaching the target
-        const int n = (int)nkeys;
-        int npow = 1;
-        while (npow < n) npow <<= 1;
-        for (int i = threadIdx.x; i < npow; i += blockDim.x)
-            if (i >= n) keys[i] = ~0ull;
-        __syncthreads();
-        for (int k = 2; k <= npow; k <<= 1) {
-            for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                for (int i = threadIdx.x; i < npow; i += blockDim.x) {
-                    const int ixj = i ^ jj;
-                    if (ixj > i) {
-                        const unsigned long long a0 = keys[i], a1 = keys[ixj];
-                        const bool asc = (i & k) == 0;
-                        if ((a0 > a1) == asc) {
-                            keys[i] = a1;
-                            keys[ixj] = a0;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-        }
-        const int per = (n + blockDim.x - 1) / blockDim.x;
-        const int i0 = threadIdx.x * per;
-        unsigned long long run = 0;
-        for (int i = i0; i < min(n, i0 + per); ++i) run += sm.mass(key_score(keys[i]));
-        unsigned long long tot;
-        unsigned long long cum = block_excl_scan<unsigned long long>(run, red_u, tot);
-        int found = n;
-        for (int i = i0; i < min(n, i0 + per); ++i) {
-            cum += sm.mass(key_score(keys[i]));
-            if (cum >= need) {
-                found = i;
-                break;
-            }
-        }
-        found = block_min_t<int>(found, red_i);
-        if (found >= n) found = n - 1;
+        const int found = sort_prefix(keys, (int)nkeys, need);
         for (int i = threadIdx.x; i <= found; i += blockDim.x) {
             const uint32_t jk = (uint32_t)keys[i];
             atomicOr(outw + (jk >> 5), 1u << (jk & 31));

@@ -240,7 +240,8 @@ int64_t zha_decoder_words(const zha_decoder* dec, int32_t level);
  * as the per-lane sum, attended tokens (union per group and per-lane sum), and the
  * device status word (0 = ok; bit 1: the top-p select ran out of bisection steps,
  * bit 2: a union list reached its capacity, bit 4: a tensor-core wait gave up after 2 s,
- * bit 8: an input outside the fp16 range reached the tensor-core scorer).
+ * bit 8: an input outside the fp16 range reached the tensor-core scorer, bit 16: a
+ * sharded cut's boundary bin held more keys than the ranks can exchange).
  * Returns ZHA_ERR_DEVICE when the status word is not 0. */
 typedef struct zha_decode_stats {
     int64_t union_nodes[ZHA_MAX_LEVELS];      /* index l-1 */
@@ -251,6 +252,81 @@ typedef struct zha_decode_stats {
     int32_t status;
 } zha_decode_stats;
 zha_status zha_decoder_stats(const zha_decoder* dec, zha_decode_stats* out, void* stream);
+
+
+/* ------------------------------------------------------------------ sharded sequence */
+
+/* One sequence whose tokens are split over `world` ranks (one GPU each, one process per
+ * GPU), for contexts whose KV cache and tree do not fit one GPU: the tree is stored on top
+ * of the whole raw cache, so it saves bandwidth, not capacity (ic.work, section
+ * "四百倍加速只是纸面推演，局部改装与位置编码暗藏边界", bullet "风险"), while the pages aim the
+ * method at contexts of hundreds of millions of tokens (fluxbbs.com, section "换架构与后续展望").
+ *
+ * Layout: rank r holds tokens [token_offset_r, token_offset_r + n_r) of the sequence in its
+ * own K, V (same layout as zha_build_tree, row 0 = the shard's first token) and its own
+ * tree built over those rows; token_offset_0 = 0, the ranges are consecutive in rank order,
+ * every token_offset is a multiple of C^L, and every rank but the last holds a multiple of
+ * C^L tokens (the sequence's tail lives on the last rank).  The sequence's level-1 nodes
+ * must number at most 2^24 (the fixed-point masses of one level then sum below 2^63).
+ *
+ * Result: the same routing and attention as one tree over the whole sequence.  Every level's
+ * top-p cut is taken over the union of all ranks' frontiers: each rank sums the same exact
+ * fixed-point mass histogram, and the boundary bin is ordered by (score desc, GLOBAL node
+ * index asc), so the kept nodes in each rank's range are exactly the single-tree kept nodes
+ * there; attention runs per rank over its kept chunks (token 0 of the sequence, the sink,
+ * on rank 0; the tail on the last rank) and the ranks' results are merged by their
+ * log-sum-exp.
+ *
+ * Protocol (every rank makes the same calls and collectives in the same order; `lanes` =
+ * n_q * n_q_heads):
+ *   zha_shard_begin
+ *   for level = L down to 1:
+ *     zha_shard_score   then  all-reduce MAX ex.lane_max (int32), SUM ex.lane_cnt (int32)
+ *     zha_shard_hist    then  all-reduce SUM ex.hist (64-bit integers)
+ *     zha_shard_cut     then  all-gather ex.keys -> ex.keys_all, ex.nkeys -> ex.nkeys_all
+ *     zha_shard_finish
+ *   zha_shard_attend    then  all-gather ex.out -> ex.out_all, ex.lse -> ex.lse_all
+ *   zha_shard_combine
+ * A call out of this order returns ZHA_ERR_STATE and enqueues nothing.  The exchange
+ * buffers are device memory owned by the caller (all 16-byte aligned); all-gathers are
+ * rank-major ([world][...] with rank r's block at r). */
+#define ZHA_SHARD_BINS 2048
+#define ZHA_SHARD_KEYS 2048
+typedef struct zha_shard_exchange {
+    int32_t* lane_max;          /* [lanes] frontier maximum score, as ordered int32 (MAX over ranks) */
+    int32_t* lane_cnt;          /* [lanes] frontier size (SUM over ranks) */
+    uint64_t* hist;             /* [lanes][ZHA_SHARD_BINS] fixed-point bin masses (SUM over ranks) */
+    uint64_t* keys;             /* [lanes][ZHA_SHARD_KEYS] this rank's boundary-bin keys */
+    int32_t* nkeys;             /* [lanes] their number (may exceed ZHA_SHARD_KEYS: reported) */
+    const uint64_t* keys_all;   /* [world][lanes][ZHA_SHARD_KEYS] gathered keys */
+    const int32_t* nkeys_all;   /* [world][lanes] */
+    float* out;                 /* [lanes][d] this rank's attention output (normalised) */
+    float* lse;                 /* [lanes] its log-sum-exp of scaled scores (-inf: no token) */
+    const float* out_all;       /* [world][lanes][d] */
+    const float* lse_all;       /* [world][lanes] */
+} zha_shard_exchange;
+
+/* A decoder for this rank's shard: tree = the shard's tree; rank in [0, world);
+ * token_offset = global index of the shard's first token (0 exactly for rank 0, else a
+ * positive multiple of C^L).  Destroy with zha_decoder_destroy.  The routing calls of a
+ * plain decoder (zha_route, zha_decode, ...) are refused on it (ZHA_ERR_STATE). */
+zha_status zha_shard_decoder_create(const zha_tree* tree, int32_t max_queries, int32_t rank, int32_t world,
+                                    int64_t token_offset, zha_decoder** out);
+/* Q bf16 [n_q][n_q_heads][d] (device; kept until zha_shard_combine), p as in zha_route. */
+zha_status zha_shard_begin(zha_decoder* dec, const void* Q, int32_t n_q, float p, void* stream);
+zha_status zha_shard_score(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream);
+zha_status zha_shard_hist(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream);
+zha_status zha_shard_cut(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream);
+/* The last step of a level.  A lane whose boundary bin held more than ZHA_SHARD_KEYS keys on
+ * one rank, or more than 4,096 over all ranks, cannot be finished: bit 16 of the device
+ * status word is set (reported by the level-1 finish and by zha_shard_combine, see
+ * zha_decoder_set_sync). */
+zha_status zha_shard_finish(zha_decoder* dec, int32_t level, const zha_shard_exchange* ex, void* stream);
+/* K, V: this shard's rows (as zha_build_tree). */
+zha_status zha_shard_attend(zha_decoder* dec, const void* K, const void* V, const zha_shard_exchange* ex,
+                            void* stream);
+/* out f32 [n_q][n_q_heads][d] (device): the sequence's attention output. */
+zha_status zha_shard_combine(zha_decoder* dec, const zha_shard_exchange* ex, float* out, void* stream);
 
 
 /* ------------------------------------------------------------------ profile */
