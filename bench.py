@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparison")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16-record router measurement")
+    ap.add_argument("--no-fp4", action="store_true", help="skip the MXFP4-record router measurement")
+    ap.add_argument("--no-shard", action="store_true",
+                    help="skip the sequence-sharded decode measurement (shards held on this one GPU)")
+    ap.add_argument("--shards", type=int, default=2, help="shards of the sharded decode measurement")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the wide 256K and batched 32 x 128K measurements")
     ap.add_argument("--n-q", type=int, default=0, help="decode only the workload's first n query tokens (profiling)")
@@ -378,6 +382,19 @@ def run_ours(args, rank, world, dev):
         dec16.close()
         tree16.close()
 
+    # The reduced-precision records where their bytes matter most, the one-query-token decode
+    # (16 lanes per sequence: the node scan is a byte stream): the same grown cache indexed by
+    # two-plane, bf16 and MXFP4 trees, one query token decoded on each.
+    if not args.no_fp4:
+        res["fp4_router"] = fp4_measure(args, dev, stream, zha, seq, K, V, qref, Q, N0, n_app, dec, out)
+
+    # The sequence-sharded decode (one sequence split over ranks): the same grown cache cut into
+    # shards on whole top nodes, each with its own tree, decoded by the sharded protocol with
+    # the shards held by this process on this GPU in lockstep (the collectives become copies
+    # on the device); against the single-tree decode of the same queries.
+    if not args.no_shard and args.shards >= 2:
+        res["sharded"] = sharded_measure(args, dev, stream, zha, seq, K, V, qref, Q, N0 + n_app, dec, out)
+
     # end to end through the public API with host buffers
     if not args.no_e2e:
         Kh = seq.K.pin_memory()
@@ -421,6 +438,130 @@ def run_ours(args, rank, world, dev):
         res["per_workload"] = per_workload(args, dev, stream)
     res["wl"] = wl
     return res
+
+
+def fp4_measure(args, dev, stream, zha, seq, K, V, qref, Q, N0, n_app, dec, out):
+    g = seq.geom
+    Q1 = Q[:, :1].contiguous()
+    out1 = torch.empty(Q1.shape, dtype=torch.float32, device=dev)
+    trees = {"f16x2": None, "bf16": zha.ZHA_SUMMARY_BF16, "fp4": zha.ZHA_SUMMARY_FP4}
+    decs, own = {"f16x2": dec}, []
+    for name, fmt in trees.items():
+        if fmt is None:
+            continue
+        t = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, seq.capacity, fmt)
+        t.build(K, N0, qref)
+        if n_app:
+            t.append(K, N0, n_app)
+        decs[name] = zha.Decoder([t], Q.shape[1])
+        own.append((t, decs[name]))
+    hbm_peak, src = measured_peaks()
+    obj = {"format": "MXFP4 slopes (E2M1 codes, one E8M0 scale per 32 dims)", "query_tokens": 1,
+           "one_query_decode_ms": {}, "node_bytes": {}, "scorer": {}}
+    kept = {}
+    for name, d in decs.items():
+        for _ in range(max(3, args.warmup)):
+            d.decode([K], [V], Q1, args.p, out1)
+        torch.cuda.synchronize()
+        zha.zha_profile_reset()
+        zha.zha_profile_enable(True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            d.decode([K], [V], Q1, args.p, out1)
+        b.record(stream)
+        torch.cuda.synchronize()
+        zha.zha_profile_enable(False)
+        pr = zha.zha_profile_read()
+        st = d.stats()
+        obj["one_query_decode_ms"][name] = a.elapsed_time(b) / args.steps
+        obj["node_bytes"][name] = st.node_bytes
+        for kn in ("k_score_few", "k_score"):
+            if kn in pr:
+                la, tms = pr[kn]
+                nb = sum(st.union_nodes) * st.node_bytes
+                obj["scorer"][name] = {"kernel": kn, "ms_per_decode": tms / args.steps,
+                                       "union_node_gb": nb / 1e9,
+                                       "hbm_frac_of_%s" % src: nb / (tms / args.steps / 1e3) / 1e9 / hbm_peak}
+                break
+        kept[name] = d.export_kept(1)[0].cpu().numpy()
+    # the float32-grade router's attended level-1 chunks that each reduced router also attends
+    base = np.unpackbits(np.ascontiguousarray(kept["f16x2"]).view(np.uint8), axis=1, bitorder="little").astype(bool)
+    for name in ("bf16", "fp4"):
+        other = np.unpackbits(np.ascontiguousarray(kept[name]).view(np.uint8), axis=1, bitorder="little").astype(bool)
+        rec = [(base[x] & other[x]).sum() / max(1, base[x].sum()) for x in range(base.shape[0])]
+        obj.setdefault("kept_chunk_recall_vs_f16x2", {})[name] = {"min": float(min(rec)), "mean": float(np.mean(rec))}
+    for t, d in own:
+        d.close()
+        t.close()
+    return obj
+
+
+def sharded_measure(args, dev, stream, zha, seq, K, V, qref, Q, n_tok, dec, out):
+    g = seq.geom
+    world = args.shards
+    ranges = zha.shard_ranges(n_tok, g.C, g.L, world)
+    n_q = Q.shape[1]
+    shards = []
+    for r, (off, cnt) in enumerate(ranges):
+        Ks = K[:, off:off + cnt].contiguous()
+        Vs = V[:, off:off + cnt].contiguous()
+        t = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, cnt)
+        t.build(Ks, cnt, qref)
+        shards.append((t, Ks, Vs, zha.ShardedDecoder(t, n_q, r, world, off)))
+    outs = [torch.empty((n_q, g.Hq, g.d), dtype=torch.float32, device=dev) for _ in shards]
+    Q3 = Q[0]
+
+    def run():
+        zha.decode_local_shards([s[3] for s in shards], [s[1] for s in shards], [s[2] for s in shards],
+                                Q3, args.p, outs)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    sh_ms = timed(run)
+    one_ms = timed(lambda: dec.decode([K], [V], Q, args.p, out))
+    diff = float((outs[0] - out[0]).abs().max().item())
+    # kept sets of every shard against the single tree's, at every level (must be identical)
+    same = True
+    for lev in range(1, g.L + 1):
+        bits1, _ = dec.export_kept(lev)
+        span = g.C ** lev
+        for (t, _, _, e), (off, cnt) in zip(shards, ranges):
+            n_l = cnt // span
+            b = e.export_kept(lev)[0]
+            w1 = torch.from_numpy(_bits_slice(bits1.cpu().numpy(), off // span, n_l))
+            w2 = torch.from_numpy(_bits_slice(b.cpu().numpy(), 0, n_l))
+            same &= bool(torch.equal(w1, w2))
+    lanes = n_q * g.Hq
+    ex_level = lanes * (4 + 4 + zha.SHARD_BINS * 8 + world * (zha.SHARD_KEYS * 8 + 4))
+    ex_attn = world * lanes * (g.d + 1) * 4
+    obj = {"shards": world, "token_ranges": ranges, "decode_ms": sh_ms, "single_tree_decode_ms": one_ms,
+           "overhead": sh_ms / one_ms, "kept_sets_identical_to_single_tree": same,
+           "max_abs_out_diff_vs_single_tree": diff,
+           "exchange_bytes_per_rank_per_decode": g.L * ex_level + ex_attn,
+           "collectives_per_decode": 5 * g.L + 2,
+           "note": "shards held by one process on one GPU in lockstep: the collectives are device copies"}
+    for t, _, _, e in shards:
+        e.close()
+        t.close()
+    return obj
+
+
+def _bits_slice(bits, start, n):
+    """Bits [start, start + n) of each row of a uint32-word bitmap, as a bool array."""
+    b = np.ascontiguousarray(bits).view(np.uint8).reshape(bits.shape[0], -1)
+    u = np.unpackbits(b, axis=1, bitorder="little")
+    return u[:, start:start + n].astype(bool)
 
 
 def build_bytes(g, n_tokens):
@@ -684,6 +825,10 @@ def main():
             line["per_workload"] = res["per_workload"]
         if "bf16_router" in res:
             line["bf16_router"] = res["bf16_router"]
+        if "sharded" in res:
+            line["sharded"] = res["sharded"]
+        if "fp4_router" in res:
+            line["fp4_router"] = res["fp4_router"]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.p)
         print(json.dumps(line))

@@ -150,8 +150,8 @@ static zha_status check_geometry(const zha_geometry* g) {
         return fail(ZHA_ERR_ARG, "capacity / C must be <= 2^24 level-1 nodes");
     double top = pow((double)g->C, (double)g->L);
     if (top > 4.0e15) return fail(ZHA_ERR_ARG, "C^L too large");
-    if (g->format != ZHA_SUMMARY_F16X2 && g->format != ZHA_SUMMARY_BF16)
-        return fail(ZHA_ERR_ARG, "format must be ZHA_SUMMARY_F16X2 or ZHA_SUMMARY_BF16");
+    if (g->format != ZHA_SUMMARY_F16X2 && g->format != ZHA_SUMMARY_BF16 && g->format != ZHA_SUMMARY_FP4)
+        return fail(ZHA_ERR_ARG, "format must be ZHA_SUMMARY_F16X2, ZHA_SUMMARY_BF16 or ZHA_SUMMARY_FP4");
     return ZHA_OK;
 }
 
@@ -515,9 +515,10 @@ extern "C" zha_status zha_decoder_create(const zha_tree* const* trees, int32_t n
     dec->seq_dev = reinterpret_cast<SeqDev*>(base + seq_off);
     dec->sh_need = reinterpret_cast<unsigned long long*>(base + need_off);
     dec->seq_host.resize(n_seq);
-    // TMA maps of the trees' fp16 planes, one per (sequence, level), for the tensor scorer
+    // TMA maps of the trees' fp16 (or bf16) planes, one per (sequence, level), for the tensor
+    // scorer; MXFP4 records are scored on the CUDA cores only
     w.tmaps = nullptr;
-    if (dec->all_r16) {
+    if (dec->all_r16 && g0.format != ZHA_SUMMARY_FP4) {
         std::vector<CUtensorMap> maps((size_t)n_seq * (kMaxL + 1) * kMapsPerLevel);
         memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
         bool ok = true;
@@ -1009,6 +1010,8 @@ extern "C" zha_status zha_decoder_set_kernels(zha_decoder* dec, int32_t score, i
     if (!ok(score) || !ok(attn)) return fail(ZHA_ERR_ARG, "unknown kernel choice");
     if (score == ZHA_KERNELS_TENSOR && !dec->all_r16)
         return fail(ZHA_ERR_ARG, "the tensor-core scorer needs R = 16 in every tree");
+    if (score == ZHA_KERNELS_TENSOR && dec->trees[0]->g.format == ZHA_SUMMARY_FP4)
+        return fail(ZHA_ERR_ARG, "MXFP4 records are scored on the CUDA cores only");
     if (score == ZHA_KERNELS_TENSOR && !dec->w.tmaps)
         return fail(ZHA_ERR_CUDA, "the tensor-core scorer's TMA maps could not be encoded");
     dec->score_path = score;

@@ -51,6 +51,17 @@ __device__ __forceinline__ float quad_sum(float v) {
 // m values of slope r held by thread quarter q (dims 16 i + 4 q + c) of a stored record.
 template <int D>
 __device__ __forceinline__ void load_row_m(const float* rec, int R, int r, int q, float (&v)[D / 4], int fmt) {
+    if (fmt == kFmtFp4) {
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+            const float4 x = fp4_load4(rec, R, D, r, 16 * i + 4 * q);
+            v[4 * i + 0] = x.x;
+            v[4 * i + 1] = x.y;
+            v[4 * i + 2] = x.z;
+            v[4 * i + 3] = x.w;
+        }
+        return;
+    }
     if (fmt == kFmtBf16) {
         const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(rec) + (int64_t)r * D;
 #pragma unroll
@@ -91,6 +102,48 @@ __device__ __forceinline__ float finalize_store(float mx, float z, const float (
     bool bad = false;
     __half* hp = reinterpret_cast<__half*>(rec);
     __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(rec);
+    if (fmt == kFmtFp4) {
+        // MXFP4: block k of 32 dims is held 8 dims per quarter-thread (i = 2k, 2k + 1); its
+        // largest magnitude over the quad sets the scale, then every value gets its code
+        uint8_t* cp = reinterpret_cast<uint8_t*>(rec);
+        uint8_t* sp = cp + (int64_t)R * D / 2;
+#pragma unroll
+        for (int bk = 0; bk < D / kFp4Block; ++bk) {
+            float a[8];
+            float amax = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                a[c] = acc[8 * bk + c] * inv;
+                amax = fmaxf(amax, fabsf(a[c]));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+            const uint32_t E = fp4_scale_byte(amax);
+            const float X = fp4_scale(E), iX = fp4_inv_scale(E);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = 2 * bk + h;
+                uint32_t wv = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t code = fp4_code(a[4 * h + c] * iX);
+                    wv |= code << (4 * c);
+                    m[4 * i + c] = fp4_value(code, X);
+                }
+                if (store) *reinterpret_cast<uint16_t*>(cp + ((int64_t)r * D + 16 * i + 4 * q) / 2) = (uint16_t)wv;
+            }
+            if (store && q == 0) sp[(int64_t)r * (D / kFp4Block) + bk] = (uint8_t)E;
+        }
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) qm = fmaf(qv[k], m[k], qm);
+        qm = quad_sum(qm);
+        const float l = mx + logf(z);
+        if (store && q == 0) {
+            rec[b_offset(R, D, fmt) + r] = fmaf(-scale, qm, l);
+            lse[r] = l;
+        }
+        return l;
+    }
 #pragma unroll
     for (int i = 0; i < D / 16; ++i) {
         float a[4];
@@ -204,7 +257,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Streams the C^k_emit tokens of one level-k_emit node per worker and emits the summaries of
 // every node of levels 1..k_emit beneath it.  Level-1 state lives in registers, levels
 // 2..k_emit in shared memory ([level][field][thread]).
-template <int D>
+template <int D, int FMT>
 __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
     extern __shared__ float smem_state[];
     const int wt = 4 * a.R;
@@ -304,7 +357,7 @@ __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
                 const float l1 = finalize_store<D>(mx, z, acc, qv, a.scale,
                                                    a.rec[1] + ((int64_t)g * a.cap[1] + j1) * a.ns,
                                                    a.lse[1] + ((int64_t)g * a.cap[1] + j1) * a.R, r, q, a.R,
-                                                   active, a.rflag, m1, a.fmt);
+                                                   active, a.rflag, m1, FMT);
                 if (nst > 0) fold_into_smem<D>(smem_state + tid, stride, l1, m1);
                 mx = -INFINITY;
                 z = 0.0f;
@@ -322,7 +375,7 @@ __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
                     const float ll = finalize_store<D>(smx, sz, sacc, qv, a.scale,
                                                        a.rec[l] + ((int64_t)g * a.cap[l] + jl) * a.ns,
                                                        a.lse[l] + ((int64_t)g * a.cap[l] + jl) * a.R, r, q, a.R,
-                                                       active, a.rflag, ml, a.fmt);
+                                                       active, a.rflag, ml, FMT);
                     if (l < a.k_emit)
                         fold_into_smem<D>(smem_state + (int64_t)(l - 1) * (D / 4 + 2) * stride + tid, stride, ll, ml);
                     reset_smem<D>(st, stride);
@@ -336,7 +389,7 @@ __global__ void __launch_bounds__(128, 4) k_build_stream(BuildArgs a) {
 
 // Merges the C children (level l-1) of each parent node P in [p0, p0+np) at level l:
 // lse_P = log sum_c exp(lse_c), m_P = sum_c exp(lse_c - lse_P) m_c, b_P = lse_P - s q_r.m_P.
-template <int D>
+template <int D, int FMT>
 __global__ void __launch_bounds__(128) k_merge(MergeArgs a) {
     const int wt = 4 * a.R;
     const int wpb = blockDim.x / wt;
@@ -359,12 +412,12 @@ __global__ void __launch_bounds__(128) k_merge(MergeArgs a) {
 #pragma unroll
     for (int k = 0; k < D / 4; ++k) acc[k] = 0.0f;
     for (int c = 0; c < a.C; ++c) {
-        load_row_m<D>(crec + (int64_t)c * a.ns, a.R, r, q, mc, a.fmt);
+        load_row_m<D>(crec + (int64_t)c * a.ns, a.R, r, q, mc, FMT);
         const float lc = __ldg(clse + (int64_t)c * a.R + r);
         fold_child<D>(mx, z, acc, lc, mc);
     }
     finalize_store<D>(mx, z, acc, qv, a.scale, a.rec + ((int64_t)g * a.cap + P) * a.ns,
-                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, a.rflag, mo, a.fmt);
+                      a.lse + ((int64_t)g * a.cap + P) * a.R, r, q, a.R, active, a.rflag, mo, FMT);
 }
 
 // Decodes the m planes of nodes [0, n) of every KV head into f32 [Hkv][n][R][d].
@@ -405,12 +458,19 @@ cudaError_t launch_build_stream(const BuildArgs& a, int d, cudaStream_t st) {
     const size_t smem = (size_t)(a.k_emit - 1) * (d / 4 + 2) * threads * sizeof(float) +
                         (size_t)wpb * kStages * kTok * d * 2;
     ProfScope ps_("k_build_stream", st);
+    auto go = [&](auto kern) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<(unsigned)blocks, threads, smem, st>>>(a);
+    };
+    // one instance per head dimension and record format (the format's code only)
     if (d == 128) {
-        cudaFuncSetAttribute(k_build_stream<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_build_stream<128><<<(unsigned)blocks, threads, smem, st>>>(a);
+        if (a.fmt == kFmtBf16) go(k_build_stream<128, kFmtBf16>);
+        else if (a.fmt == kFmtFp4) go(k_build_stream<128, kFmtFp4>);
+        else go(k_build_stream<128, kFmtF16x2>);
     } else {
-        cudaFuncSetAttribute(k_build_stream<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_build_stream<64><<<(unsigned)blocks, threads, smem, st>>>(a);
+        if (a.fmt == kFmtBf16) go(k_build_stream<64, kFmtBf16>);
+        else if (a.fmt == kFmtFp4) go(k_build_stream<64, kFmtFp4>);
+        else go(k_build_stream<64, kFmtF16x2>);
     }
     return cudaGetLastError();
 }
@@ -421,10 +481,16 @@ cudaError_t launch_merge(const MergeArgs& a, int d, cudaStream_t st) {
     const int threads = wpb * 4 * a.R;
     const int64_t blocks = ((int64_t)a.Hkv * a.np + wpb - 1) / wpb;
     ProfScope ps_("k_merge", st);
-    if (d == 128)
-        k_merge<128><<<(unsigned)blocks, threads, 0, st>>>(a);
-    else
-        k_merge<64><<<(unsigned)blocks, threads, 0, st>>>(a);
+    auto go = [&](auto kern) { kern<<<(unsigned)blocks, threads, 0, st>>>(a); };
+    if (d == 128) {
+        if (a.fmt == kFmtBf16) go(k_merge<128, kFmtBf16>);
+        else if (a.fmt == kFmtFp4) go(k_merge<128, kFmtFp4>);
+        else go(k_merge<128, kFmtF16x2>);
+    } else {
+        if (a.fmt == kFmtBf16) go(k_merge<64, kFmtBf16>);
+        else if (a.fmt == kFmtFp4) go(k_merge<64, kFmtFp4>);
+        else go(k_merge<64, kFmtF16x2>);
+    }
     return cudaGetLastError();
 }
 

@@ -18,17 +18,28 @@ constexpr int kMaxL = ZHA_MAX_LEVELS;
 // sectors).  lse [R] f32 is kept in a separate array per level (read by merges and export).
 //   format 0 (ZHA_SUMMARY_F16X2): m as fp16 planes hi [R][d] then lo [R][d] (4 bytes a value)
 //   format 1 (ZHA_SUMMARY_BF16):  m as one bf16 plane [R][d] (2 bytes a value)
+//   format 2 (ZHA_SUMMARY_FP4):   m as MXFP4 (the OCP microscaling format): E2M1 codes [R][d]
+//                                 packed two to a byte (even dim in the low nibble), then one
+//                                 E8M0 scale byte per block of 32 dims [R][d/32], that area
+//                                 padded to 16 bytes (half a byte and 1/32 byte a value)
 constexpr int kFmtF16x2 = 0;
 constexpr int kFmtBf16 = 1;
+constexpr int kFmtFp4 = 2;
+constexpr int kFp4Block = 32;        // dims sharing one scale
+// Floats of an MXFP4 record's scale area.
+inline __host__ __device__ int64_t fp4_scale_floats(int R, int d) { return ((int64_t)R * d / kFp4Block + 15) / 16 * 4; }
 inline __host__ __device__ int32_t record_stride(int R, int d, int fmt = kFmtF16x2) {
+    if (fmt == kFmtFp4) return (int32_t)(((int64_t)R * d / 8 + fp4_scale_floats(R, d) + R + 7) / 8 * 8);
     return fmt == kFmtBf16 ? ((R * d / 2 + R + 7) / 8) * 8 : ((R * (d + 1) + 7) / 8) * 8;
 }
 // Floats from the start of a record to its b values.
 inline __host__ __device__ int64_t b_offset(int R, int d, int fmt) {
+    if (fmt == kFmtFp4) return (int64_t)R * d / 8 + fp4_scale_floats(R, d);
     return fmt == kFmtBf16 ? (int64_t)R * d / 2 : (int64_t)R * d;
 }
-// Bytes a scorer reads per node: the m planes and b.
+// Bytes a scorer reads per node: the m planes (codes and scales) and b.
 inline __host__ __device__ int64_t scored_node_bytes(int R, int d, int fmt) {
+    if (fmt == kFmtFp4) return (int64_t)R * d / 2 + (int64_t)R * d / kFp4Block + (int64_t)R * 4;
     return (fmt == kFmtBf16 ? (int64_t)R * d * 2 : (int64_t)R * d * 4) + (int64_t)R * 4;
 }
 
@@ -151,8 +162,62 @@ __device__ __forceinline__ float2 m_decode2(uint32_t hi, uint32_t lo) {
 __device__ __forceinline__ float2 m_decode_bf16(uint32_t w) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
 }
+// MXFP4 (OCP Microscaling Formats specification v1.0, the MXFP4 element and scale types and
+// the conversion to them): a block of 32 values shares the scale X = 2^(floor(log2 amax) - 2)
+// (2 = the largest exponent of E2M1), stored as its E8M0 byte floor(log2 amax) - 2 + 127
+// (clamped at 0: a zero or tiny block); each value is v / X rounded to the nearest E2M1 value
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6} (ties to the even code, magnitudes above 6 saturate to 6) with
+// v's sign (no negative zero).
+__host__ __device__ inline uint32_t fp4_scale_byte(float amax) {
+    union { float f; uint32_t u; } c;
+    c.f = amax;
+    const int ex = (int)((c.u >> 23) & 0xFFu);      // floor(log2 amax) + 127 for a normal amax
+    return (uint32_t)(ex >= 2 ? (ex > 255 ? 253 : ex - 2) : 0);
+}
+// 2^(E - 127) and 2^(127 - E) for an E8M0 byte E in [0, 253].
+__host__ __device__ inline float fp4_scale(uint32_t E) {
+    union { float f; uint32_t u; } c;
+    c.u = E ? (E << 23) : 0x00400000u;             // E = 0: 2^-127, a subnormal float
+    return c.f;
+}
+__host__ __device__ inline float fp4_inv_scale(uint32_t E) {
+    union { float f; uint32_t u; } c;
+    c.u = (254u - E) << 23;
+    return c.f;
+}
+// E2M1 code of y (already divided by the scale): the count of rounding boundaries below |y|,
+// a tie counting when the upper neighbour has the even code.
+__host__ __device__ inline uint32_t fp4_code(float y) {
+    const float a = fabsf(y);
+    const uint32_t c = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                       (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) + (uint32_t)(a > 5.0f);
+    return c | ((c != 0u && y < 0.0f) ? 8u : 0u);
+}
+// Value of an E2M1 code (bit 3 sign, bits 2-1 exponent, bit 0 mantissa) times a scale.
+__host__ __device__ inline float fp4_value(uint32_t code, float scale) {
+    const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+    uint32_t bits = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
+    bits |= (code & 8u) << 28;
+    union { float f; uint32_t u; } c;
+    c.u = bits;
+    return c.f * scale;
+}
+// Byte pointers of an MXFP4 record: the codes and the scales.
+__device__ __forceinline__ const uint8_t* fp4_codes(const float* rec) { return reinterpret_cast<const uint8_t*>(rec); }
+__device__ __forceinline__ const uint8_t* fp4_scales(const float* rec, int R, int D) {
+    return reinterpret_cast<const uint8_t*>(rec) + (int64_t)R * D / 2;
+}
+// Four consecutive values (dims k..k+3, k a multiple of 4) of slope r of an MXFP4 record.
+__device__ __forceinline__ float4 fp4_load4(const float* rec, int R, int D, int r, int k) {
+    const uint32_t w = *reinterpret_cast<const uint16_t*>(fp4_codes(rec) + ((int64_t)r * D + k) / 2);
+    const float X = fp4_scale(fp4_scales(rec, R, D)[(int64_t)r * (D / kFp4Block) + k / kFp4Block]);
+    return make_float4(fp4_value(w & 15u, X), fp4_value((w >> 4) & 15u, X), fp4_value((w >> 8) & 15u, X),
+                       fp4_value((w >> 12) & 15u, X));
+}
+
 // Four consecutive m values (dims k..k+3 of slope r) of a record in format fmt.
 __device__ __forceinline__ float4 m_load4(const float* rec, int R, int D, int r, int k, int fmt) {
+    if (fmt == kFmtFp4) return fp4_load4(rec, R, D, r, k);
     if (fmt == kFmtBf16) {
         const uint2 a = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(rec) + (int64_t)r * D + k);
         const float2 x = m_decode_bf16(a.x), y = m_decode_bf16(a.y);

@@ -220,8 +220,9 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
 // Warp = 8 lanes x 4 quarter-threads; thread (lane, quarter) keeps its lane's query
 // dimensions {16 i + 4 quarter + c} in registers.  WB warps split a block of 8*WB lanes,
 // 8/WB node slots run concurrently.  Each node record is read with 16-byte loads.
-template <int D, bool BF>
+template <int D, int FMT>
 __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float scale) {
+    constexpr bool BF = FMT == kFmtBf16;
     const int grp = blockIdx.z;
     const int s = grp / b.Hkv, g = grp % b.Hkv;
     const SeqDev& sq = b.seqs[s];
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
         const float* rec = base + j * ns;
         const __half* rh = reinterpret_cast<const __half*>(rec);
         float best = -INFINITY;
-        const float* brow = rec + (BF ? (int64_t)R * D / 2 : (int64_t)R * D);
+        const float* brow = rec + b_offset(R, D, FMT);
         for (int r = 0; r < R; ++r) {
             const uint2* hrow = reinterpret_cast<const uint2*>(rh + (int64_t)r * D);   // also the bf16 plane
             const uint2* lrow = reinterpret_cast<const uint2*>(rh + (int64_t)R * D + (int64_t)r * D);
@@ -278,7 +279,9 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) {
                 float4 m;
-                if constexpr (BF) {
+                if constexpr (FMT == kFmtFp4) {
+                    m = fp4_load4(rec, R, D, r, 16 * i + 4 * q);
+                } else if constexpr (BF) {
                     const uint2 hv = __ldg(hrow + 4 * i + q);
                     const float2 m01 = m_decode_bf16(hv.x), m23 = m_decode_bf16(hv.y);
                     m = make_float4(m01.x, m01.y, m23.x, m23.y);
@@ -323,8 +326,9 @@ __global__ void __launch_bounds__(256) k_score(Batch b, Work w, int it, float sc
 // k_score: e = max_r (s q.m_r + b_r), -inf off the lane's frontier, in candidate order.
 constexpr int kFewLanes = 16;
 
-template <int D, bool BF>
+template <int D, int FMT>
 __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, float scale) {
+    constexpr bool BF = FMT == kFmtBf16;
     constexpr int kHalf = D / 2;      // dims per thread
     constexpr int kV = kHalf / 8;     // 16-byte pieces per plane per thread
     constexpr int kRow = kHalf + 4;   // shared row stride of a query half (the two halves of a
@@ -369,13 +373,31 @@ __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, f
         const uint4* hp = reinterpret_cast<const uint4*>(rh + (int64_t)r * D + hf * kHalf);   // also the bf16 plane
         const uint4* lp = reinterpret_cast<const uint4*>(rh + (int64_t)R * D + (int64_t)r * D + hf * kHalf);
         uint4 hv[kV], lv[kV];
+        float m[kHalf];
+        const float br = __ldg(rec + b_offset(R, D, FMT) + r);
+        if constexpr (FMT == kFmtFp4) {
+            // this thread's D/2 codes (D/4 bytes) and the scales of their D/64 blocks
+            constexpr int kC4 = kHalf / 32;             // 16-byte pieces of codes
+            const uint4* cq = reinterpret_cast<const uint4*>(fp4_codes(rec) + ((int64_t)r * D + hf * kHalf) / 2);
+            uint4 cv[kC4];
+#pragma unroll
+            for (int v = 0; v < kC4; ++v) cv[v] = __ldg(cq + v);
+            const uint8_t* sc = fp4_scales(rec, R, D) + (int64_t)r * (D / kFp4Block) + hf * (kHalf / kFp4Block);
+#pragma unroll
+            for (int v = 0; v < kC4; ++v) {
+                const float X = fp4_scale(__ldg(sc + v));
+                const uint32_t cw[4] = {cv[v].x, cv[v].y, cv[v].z, cv[v].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) m[32 * v + 8 * c + t] = fp4_value((cw[c] >> (4 * t)) & 15u, X);
+            }
+        } else {
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             hv[v] = __ldg(hp + v);
             if constexpr (!BF) lv[v] = __ldg(lp + v);
         }
-        const float br = __ldg(rec + (BF ? (int64_t)R * D / 2 : (int64_t)R * D) + r);
-        float m[kHalf];
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             const uint32_t hw[4] = {hv[v].x, hv[v].y, hv[v].z, hv[v].w};
@@ -391,6 +413,7 @@ __global__ void __launch_bounds__(256, 2) k_score_few(Batch b, Work w, int it, f
                 m[8 * v + 2 * c] = f.x;
                 m[8 * v + 2 * c + 1] = f.y;
             }
+        }
         }
         float mine = -INFINITY;
 #pragma unroll 1
@@ -1008,7 +1031,7 @@ cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaSt
 }
 
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
-    const bool tc = b.all_r16 && w.tmaps &&
+    const bool tc = b.all_r16 && w.tmaps && b.fmt != kFmtFp4 &&
                     (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
     if (tc) return launch_score_tc(b, w, it, scale, st);
     if (b.all_r16 && b.n_gl <= kFewLanes && b.d == 128) {
@@ -1017,22 +1040,25 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
         const int bx = std::max(1, 2 * sm_count() / std::max(1, b.n_groups));
         ProfScope ps_("k_score", st);
         if (b.fmt == kFmtBf16)
-            k_score_few<128, true><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+            k_score_few<128, kFmtBf16><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+        else if (b.fmt == kFmtFp4)
+            k_score_few<128, kFmtFp4><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
         else
-            k_score_few<128, false><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
+            k_score_few<128, kFmtF16x2><<<dim3(bx, 1, b.n_groups), 256, 0, st>>>(b, w, it, scale);
         return cudaGetLastError();
     }
     const int WB = min(8, (b.n_gl + 7) / 8);
     const int lane_blocks = (b.n_gl + 8 * WB - 1) / (8 * WB);
     dim3 grid(score_blocks_x(lane_blocks, b.n_groups), lane_blocks, b.n_groups);
     ProfScope ps_("k_score", st);
-    const bool bf = b.fmt == kFmtBf16;
     if (b.d == 128) {
-        if (bf) k_score<128, true><<<grid, 256, 0, st>>>(b, w, it, scale);
-        else k_score<128, false><<<grid, 256, 0, st>>>(b, w, it, scale);
+        if (b.fmt == kFmtBf16) k_score<128, kFmtBf16><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else if (b.fmt == kFmtFp4) k_score<128, kFmtFp4><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else k_score<128, kFmtF16x2><<<grid, 256, 0, st>>>(b, w, it, scale);
     } else {
-        if (bf) k_score<64, true><<<grid, 256, 0, st>>>(b, w, it, scale);
-        else k_score<64, false><<<grid, 256, 0, st>>>(b, w, it, scale);
+        if (b.fmt == kFmtBf16) k_score<64, kFmtBf16><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else if (b.fmt == kFmtFp4) k_score<64, kFmtFp4><<<grid, 256, 0, st>>>(b, w, it, scale);
+        else k_score<64, kFmtF16x2><<<grid, 256, 0, st>>>(b, w, it, scale);
     }
     return cudaGetLastError();
 }

@@ -38,7 +38,7 @@ class ZhaError(RuntimeError):
         self.status = status
 
 
-ZHA_SUMMARY_F16X2, ZHA_SUMMARY_BF16 = 0, 1
+ZHA_SUMMARY_F16X2, ZHA_SUMMARY_BF16, ZHA_SUMMARY_FP4 = 0, 1, 2
 
 
 class Geometry(ctypes.Structure):

@@ -60,15 +60,27 @@ typedef enum zha_status {
 
 /* How a node record stores its R slopes m_r (b, lse and every computation stay f32).
  * The pages test a router with reduced-precision summaries next to the full one (wqu.guru,
- * summary bullets: an FP4 router variant); this library offers two formats:
+ * summary bullets: an FP4 router variant); this library offers three formats:
  *   ZHA_SUMMARY_F16X2  m as two fp16 planes hi + lo (m = hi + lo within 2^-22 |m| + 2^-25):
  *                      float32-grade summaries, 4 bytes per value.  Keys must stay below
  *                      65504 in magnitude.  The default.
  *   ZHA_SUMMARY_BF16   m as one bf16 plane (relative rounding 2^-9): half the bytes every
  *                      scored node costs, one tensor-core pass per node; routing decisions
  *                      follow the rounded slopes, so kept sets differ from the float32-grade
- *                      router's where estimates are close. */
-typedef enum zha_summary_format { ZHA_SUMMARY_F16X2 = 0, ZHA_SUMMARY_BF16 = 1 } zha_summary_format;
+ *                      router's where estimates are close.
+ *   ZHA_SUMMARY_FP4    m as MXFP4 (OCP Microscaling Formats v1.0): 4-bit E2M1 codes with one
+ *                      power-of-two E8M0 scale per 32 dims, 2^(floor(log2 max|block|) - 2);
+ *                      values rounded to nearest (ties to even), above 6 x scale saturated.
+ *                      About 1/7 of the two-plane bytes per scored node (1,152 B at R = 16,
+ *                      d = 128).  Level-1 slopes are the MXFP4 rounding of the exact slopes;
+ *                      merges read the stored (decoded) children, so the levels above carry
+ *                      the rounding of the levels below.  Scored on the CUDA cores
+ *                      (ZHA_KERNELS_TENSOR is refused); built by the streaming kernels. */
+typedef enum zha_summary_format {
+    ZHA_SUMMARY_F16X2 = 0,
+    ZHA_SUMMARY_BF16 = 1,
+    ZHA_SUMMARY_FP4 = 2
+} zha_summary_format;
 
 /* Tree geometry and the shape of the KV cache it indexes. */
 typedef struct zha_geometry {

@@ -193,3 +193,40 @@ def decode(K: np.ndarray, V: np.ndarray, qref: np.ndarray, C: int, L: int, N: in
     toks = [attended_set(kept1[x], N, C, L) for x in range(q.shape[0])]
     out = attend_batch(K, V, q, lane_g, toks)
     return r, out, toks
+
+
+# MXFP4 (OCP Microscaling Formats (MX) Specification v1.0: the E2M1 element type, the E8M0
+# shared scale and the conversion of a block of 32 values): the reduced-precision slope
+# records of an FP4 router.  E2M1 magnitudes, indexed by the 3 low bits of a code
+# (2 exponent bits, 1 mantissa bit, exponent bias 1):
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def mxfp4(x: np.ndarray, block: int = 32):
+    """Rounds x [..., n] (n a multiple of `block`) to MXFP4, block by block along the last axis.
+
+    Per block: shared scale X = 2^(floor(log2 max|x|) - 2), the largest power of two not above
+    the block maximum divided by 2^2 (2 being E2M1's largest exponent), as the E8M0 byte
+    floor(log2 max|x|) - 2 + 127 clamped to [0, 254] (0 for an all-zero block); every element
+    becomes the E2M1 value nearest to x / X, ties to the value with an even mantissa bit,
+    magnitudes beyond 6 saturated to 6, keeping the sign.
+    Returns (decoded values float64 [..., n], codes uint8 [..., n] (sign in bit 3; none for 0),
+    scale bytes uint8 [..., n / block])."""
+    x = np.asarray(x, dtype=np.float64)
+    shp = x.shape
+    xb = x.reshape(shp[:-1] + (shp[-1] // block, block))
+    amax = np.abs(xb).max(axis=-1)
+    _, ex = np.frexp(amax)                         # amax = f 2^ex, f in [0.5, 1): floor(log2) = ex - 1
+    E = np.where(amax > 0, np.clip(ex - 1 - 2 + 127, 0, 254), 0).astype(np.int64)
+    X = np.ldexp(1.0, E - 127)[..., None]
+    y = xb / X
+    a = np.abs(y)
+    # nearest E2M1 magnitude: the midpoints between neighbours, a tie going to the even code
+    mids = (E2M1_VALUES[:-1] + E2M1_VALUES[1:]) / 2       # 0.25 0.75 1.25 1.75 2.5 3.5 5
+    idx = np.zeros(a.shape, dtype=np.int64)
+    for k, mid in enumerate(mids):
+        up_is_even = (k + 1) % 2 == 0
+        idx += (a >= mid) if up_is_even else (a > mid)
+    val = np.sign(y) * E2M1_VALUES[idx] * X
+    codes = (idx | np.where((y < 0) & (idx > 0), 8, 0)).astype(np.uint8)
+    return val.reshape(shp), codes.reshape(shp), E.astype(np.uint8)

@@ -46,7 +46,7 @@ def test_build_targets_sm100a_only():
 
 @pytest.mark.parametrize("field,value", [("C", 1), ("C", 2048), ("L", 0), ("L", 17), ("R", 3), ("R", 64),
                                          ("d", 96), ("n_kv_heads", 0), ("n_q_heads", 3), ("capacity", 0),
-                                         ("capacity", 1 << 31), ("format", 2), ("format", -1)])
+                                         ("capacity", 1 << 31), ("format", 3), ("format", -1)])
 def test_tree_create_rejects_bad_geometry(libzha, field, value):
     g = zha.Geometry(4, 6, 16, 128, 16, 2, 65536)
     setattr(g, field, value)
@@ -68,6 +68,13 @@ def test_null_handles_are_rejected(libzha):
     assert libzha.zha_route(None, None, 1, 0.9, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_sparse_attn(None, None, None, None, 1, None, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_dense_attn(None, None, None, None, 1, None, None) == zha.ZHA_ERR_ARG
+    assert libzha.zha_shard_decoder_create(None, 1, 0, 1, 0, ctypes.byref(h)) == zha.ZHA_ERR_ARG
+    assert libzha.zha_shard_begin(None, None, 1, 0.9, None) == zha.ZHA_ERR_ARG
+    ex = zha.ShardExchange()
+    for fn in (libzha.zha_shard_score, libzha.zha_shard_hist, libzha.zha_shard_cut, libzha.zha_shard_finish):
+        assert fn(None, 1, ctypes.byref(ex), None) == zha.ZHA_ERR_ARG
+    assert libzha.zha_shard_attend(None, None, None, ctypes.byref(ex), None) == zha.ZHA_ERR_ARG
+    assert libzha.zha_shard_combine(None, ctypes.byref(ex), None, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_decoder_export_kept(None, 1, None, None, None) == zha.ZHA_ERR_ARG
     assert libzha.zha_decoder_words(None, 1) == 0
     assert libzha.zha_decoder_stats(None, None, None) == zha.ZHA_ERR_ARG
@@ -78,3 +85,16 @@ def test_binding_raises_on_error_status(libzha):
     with pytest.raises(zha.ZhaError) as ei:
         zha.zha_tree_create(zha.Geometry(1, 1, 1, 64, 1, 1, 16))
     assert ei.value.status == zha.ZHA_ERR_ARG
+
+
+def test_shard_exchange_layout_matches_the_header():
+    # eleven pointers, in the order zha.h declares them
+    assert ctypes.sizeof(zha.ShardExchange) == 11 * ctypes.sizeof(ctypes.c_void_p)
+    names = [f[0] for f in zha.ShardExchange._fields_]
+    hdr = open(os.path.join(ROOT, "include", "zha.h")).read()
+    body = hdr[hdr.index("typedef struct zha_shard_exchange"):hdr.index("} zha_shard_exchange;")]
+    flat = body.replace(" ", "")
+    pos = [flat.index("*" + n + ";") for n in names]
+    assert pos == sorted(pos)
+    assert "#define ZHA_SHARD_BINS %d" % zha.SHARD_BINS in hdr
+    assert "#define ZHA_SHARD_KEYS %d" % zha.SHARD_KEYS in hdr

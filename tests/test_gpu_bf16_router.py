@@ -83,35 +83,6 @@ def test_bf16_summaries_are_rounded_exact_summaries(geom, n):
     tree.close()
 
 
-def _replay_on_stored(tree, seq, n, q, lane_g, p, gk):
-    """Float64 replay of the routing on the tree's stored summaries: at every level the
-    frontier is the children of the GPU's kept set one level up; each frontier node's
-    estimate max_r (s q.m_r + b_r) is taken from the exported record; the cut is the
-    oracle's.  Returns per-(level, lane) (oracle kept bool row, info, estimates)."""
-    g = seq.geom
-    exp = {lev: [x.cpu().numpy().astype(np.float64) for x in tree.export(lev)] for lev in range(1, g.L + 1)}
-    out = {}
-    for lev in range(g.L, 0, -1):
-        m, _, b = exp[lev]
-        nl = n // g.C ** lev
-        for x in range(q.shape[0]):
-            h = lane_g[x]
-            if lev == g.L:
-                front = np.arange(nl)
-            else:
-                par = np.flatnonzero(gk[lev + 1][x])
-                front = (par[:, None] * g.C + np.arange(g.C)[None, :]).ravel()
-                front = front[front < nl]
-            est = np.array([O.plane_estimate(m[h, j], b[h, j], q[x]) for j in front])
-            keep, k, info = O.topp(est, front, p)
-            row = np.zeros(nl, dtype=bool)
-            row[front[keep]] = True
-            sc = np.full(nl, np.nan)
-            sc[front] = est
-            out[(lev, x)] = (row, info, sc)
-    return out
-
-
 @needs_cuda
 @pytest.mark.parametrize("score,geom,n,n_q", [
     (zha.ZHA_KERNELS_TENSOR, inputs.DEEP, 8 * 4096 + 333, 8),   # 64 lanes per group: tcgen05, one bf16 pass
@@ -131,7 +102,7 @@ def test_bf16_router_matches_replay_on_its_stored_summaries(score, geom, n, n_q)
     qs = [0, n_q - 1]
     q, lane_g, ids = TL.lanes_for(seq, Q, qs)
     gk = {lev: res.kept[0][lev - 1][ids] for lev in range(1, geom.L + 1)}
-    rep = _replay_on_stored(tree, seq, n, q, lane_g, 0.9, gk)
+    rep = TL.replay_on_stored(tree, seq, n, q, lane_g, 0.9, gk)
     exact = ties = 0
     for (lev, x), (row, info, sc) in rep.items():
         if np.array_equal(row, gk[lev][x]):

@@ -413,3 +413,74 @@ def test_tiny_workload_routing_keeps_sink_and_is_sparse():
     assert all(t.size < seq.n_tokens for t in toks)
     assert (r.kstar >= 1).all()
     assert (r.nfront[-1] == seq.n_tokens // g.top_span).all()
+
+
+# ----------------------------------------------------------------------------- MXFP4 rounding
+
+def _nearest_e2m1_brute(y):
+    """Nearest of the 15 signed E2M1 values to y by exhaustive search; a tie goes to the value
+    whose code has mantissa bit 0 (codes 0, 2, 4, 6 in each sign)."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    cands = [(abs(y - s * m), code % 2, s * m) for code, m in enumerate(mags) for s in (1.0, -1.0)]
+    best = min(c[0] for c in cands)
+    ties = [c for c in cands if c[0] == best]
+    ties.sort(key=lambda c: c[1])                   # even mantissa first
+    return ties[0][2]
+
+
+def test_mxfp4_hand_worked_block():
+    """Block max 7.9: floor(log2 7.9) = 2, so X = 2^0 = 1 and the E8M0 byte is 127.
+    1.0 -> 1; 0.3 -> 0.5; -0.76 -> -1 (nearer 1 than 0.5); 0.24 -> 0; 5.0 (tie 4|6) -> 4 (even);
+    7.9 -> 6 (saturated); 2.5 (tie 2|3) -> 2; 3.5 (tie 3|4) -> 4; 0.25 (tie 0|0.5) -> 0;
+    0.75 (tie 0.5|1) -> 1; -1.75 (tie 1.5|2) -> -2; 1.25 (tie 1|1.5) -> 1."""
+    x = np.zeros(32)
+    x[:12] = [1.0, 0.3, -0.76, 0.24, 5.0, 7.9, 2.5, 3.5, 0.25, 0.75, -1.75, 1.25]
+    v, codes, E = O.mxfp4(x)
+    assert E.tolist() == [127]
+    assert v[:12].tolist() == [1.0, 0.5, -1.0, 0.0, 4.0, 6.0, 2.0, 4.0, 0.0, 1.0, -2.0, 1.0]
+    assert codes[:12].tolist() == [2, 1, 8 + 2, 0, 6, 7, 4, 6, 0, 2, 8 + 4, 2]
+    assert (v[12:] == 0).all()
+
+
+def test_mxfp4_scale_is_the_blocks_binade():
+    """max |x| = 0.1 = 1.6 x 2^-4: X = 2^(-4 - 2) = 2^-6; 0.1 / X = 6.4 saturates to 6, so the
+    block maximum decodes to 6 / 64 = 0.09375.  An all-zero block has byte 0 and decodes to 0."""
+    x = np.zeros((2, 32))
+    x[0, 5] = 0.1
+    x[0, 6] = -0.05                                  # 3.2 -> 3
+    v, _, E = O.mxfp4(x)
+    assert E.ravel().tolist() == [127 - 6, 0]
+    assert v[0, 5] == 6 / 64 and v[0, 6] == -3 / 64
+    assert (v[1] == 0).all()
+
+
+def test_mxfp4_is_the_nearest_value_on_the_block_grid():
+    """Brute force: every element is the nearest signed E2M1 value times the block's scale."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((40, 64)) * np.exp(rng.uniform(-8, 8, (40, 1)))
+    x[:, ::7] *= 1e-3                                # small members of a block
+    v, _, E = O.mxfp4(x)
+    for i in range(x.shape[0]):
+        for j in range(x.shape[1]):
+            X = 2.0 ** (int(E[i, j // 32]) - 127)
+            assert v[i, j] == _nearest_e2m1_brute(x[i, j] / X) * X
+        for b in range(2):
+            blk = x[i, 32 * b:32 * b + 32]
+            X = 2.0 ** (int(E[i, b]) - 127)
+            # the scale's binade: 4 X <= max |x| < 8 X
+            assert 4 * X <= np.abs(blk).max() < 8 * X
+
+
+def test_mxfp4_representable_blocks_round_trip():
+    """A block of E2M1 values times 2^k whose maximum magnitude is 4 or 6 (times 2^k) decodes to
+    itself, codes and all."""
+    rng = np.random.default_rng(4)
+    for k in (-10, -1, 0, 3, 9):
+        idx = rng.integers(0, 8, 32)
+        idx[0] = 7
+        sgn = rng.choice([-1.0, 1.0], 32)
+        x = sgn * O.E2M1_VALUES[idx] * 2.0 ** k
+        v, codes, E = O.mxfp4(x)
+        assert np.array_equal(v, x)
+        assert E.tolist() == [127 + k]
+        assert np.array_equal(codes & 7, idx)

@@ -239,3 +239,32 @@ def check_decode(seq, n_tokens: int, Q_seq: torch.Tensor, p: float, res_out: np.
             e2 = rel_err(gpu[ok], o_e2e[ok])
             assert e2.max() <= OUT_TOL, "output vs end-to-end oracle: %g" % e2.max()
     return rep, e1, e2, toks
+
+
+def replay_on_stored(tree, seq, n, q, lane_g, p, gk):
+    """Float64 replay of the routing on the tree's stored summaries: at every level the
+    frontier is the children of the GPU's kept set one level up; each frontier node's
+    estimate max_r (s q.m_r + b_r) is taken from the exported record; the cut is the
+    oracle's.  Returns per-(level, lane) (oracle kept bool row, info, estimates)."""
+    g = seq.geom
+    exp = {lev: [x.cpu().numpy().astype(np.float64) for x in tree.export(lev)] for lev in range(1, g.L + 1)}
+    out = {}
+    for lev in range(g.L, 0, -1):
+        m, _, b = exp[lev]
+        nl = n // g.C ** lev
+        for x in range(q.shape[0]):
+            h = lane_g[x]
+            if lev == g.L:
+                front = np.arange(nl)
+            else:
+                par = np.flatnonzero(gk[lev + 1][x])
+                front = (par[:, None] * g.C + np.arange(g.C)[None, :]).ravel()
+                front = front[front < nl]
+            est = np.array([O.plane_estimate(m[h, j], b[h, j], q[x]) for j in front])
+            keep, k, info = O.topp(est, front, p)
+            row = np.zeros(nl, dtype=bool)
+            row[front[keep]] = True
+            sc = np.full(nl, np.nan)
+            sc[front] = est
+            out[(lev, x)] = (row, info, sc)
+    return out
