@@ -191,6 +191,18 @@ def kernel_algorithmic(name, st, geom, N, n_append, n_lanes, launches):
     return 0.0, 0.0
 
 
+def kernel_executed_flops(name, st, geom, n_lanes_group, planes, launches):
+    """Tensor work one launch of `name` executes: every lane of a (sequence, KV head) group
+    against every union node (R rows of d, `planes` passes for the two-plane records), resp.
+    every union token (Q K^T and the two P V passes, P = P_hi + P_lo)."""
+    R, d = geom.R, geom.d
+    if name == "k_score_tc":
+        return sum(st.union_nodes) * n_lanes_group * R * d * 2 * planes / launches
+    if name == "k_attn_tc":
+        return st.union_tokens * n_lanes_group * d * 2 * 3 / launches
+    return 0.0
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The largest of every rank's x (the job's time is its slowest rank's); x itself on one
     rank.  Every rank must call it at the same point."""
@@ -276,6 +288,10 @@ def run_ours(args, rank, world, dev):
         ach = nflops / (avg_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                 "traffic": None, "kernel": name, "peak_source": src}
+        ex = kernel_executed_flops(name, st, g, n_q * (g.Hq // g.Hkv), 2 if name == "k_score_tc" else 1,
+                                   per_step_launches)
+        roof["executed_flops_per_launch"] = ex
+        roof["executed_frac"] = ex / (avg_ms / 1e3) / 1e12 / peak
     elif nflops and intensity > FP32_PEAK_TFLOPS * 1e12 / (hbm_peak * 1e9):
         ach = nflops / (avg_ms / 1e3) / 1e12
         roof = {"bound": "alu", "achieved": ach, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",

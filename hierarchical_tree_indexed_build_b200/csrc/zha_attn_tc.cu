@@ -30,12 +30,13 @@ namespace zha {
 namespace {
 
 constexpr int kRows = 128;      // lanes per tile (MMA M)
-constexpr int kPos = 128;       // token positions per tile (MMA N of QK^T, K of PV)
-constexpr int kThreads = 512;   // 16 warps: 4 per TMEM lane quarter, each a quarter of the positions
+constexpr int kPos = 64;        // token positions per tile (MMA N of QK^T, K of PV)
+constexpr int kThreads = 256;   // 8 warps: 2 per TMEM lane quarter, each half of the positions
 constexpr int kParts = kThreads / 128;
 constexpr float kLazy = 8.0f;   // raise the running max only when exceeded by this much
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
-constexpr int kBlock = kRows * 128;   // bytes of one 128-byte-wide block of 128 rows
+constexpr int kBlock = kRows * 128;   // bytes of one 128-byte-wide block of 128 rows (Q)
+constexpr int kBlockT = kPos * 128;   // the same for the tile's kPos token rows (K, V)
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -117,41 +118,67 @@ __device__ __forceinline__ void tst16(uint32_t taddr, const float (&v)[16]) {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Offset of 16-byte chunk c16 (8 bf16) of row r in a K-major tile of 128-byte blocks.
-__device__ __forceinline__ uint32_t kmaj(int r, int c16) {
-    return (uint32_t)((c16 >> 3) * kBlock + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
+// Offset of 16-byte chunk c16 (8 bf16) of row r in a K-major tile of 128-byte blocks of
+// `blk` bytes (Q: 128 rows, K: kPos rows).
+__device__ __forceinline__ uint32_t kmaj(int r, int c16, int blk) {
+    return (uint32_t)((c16 >> 3) * blk + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
 }
 // Offset of 16-byte chunk c16 (8 bf16 along d) of token row t in the MN-major V tile.
 __device__ __forceinline__ uint32_t mnmaj(int t, int c16) {
-    return (uint32_t)((c16 >> 3) * kBlock + (t >> 3) * 1024 + (t & 7) * 128 + (((c16 & 7) ^ (t & 7)) << 4));
+    return (uint32_t)((c16 >> 3) * kBlockT + (t >> 3) * 1024 + (t & 7) * 128 + (((c16 & 7) ^ (t & 7)) << 4));
 }
 
+// A operand in tensor memory (the P tile), B from shared memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        :
+        : "r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Writes 16 consecutive 32-bit columns of this thread's tensor-memory lane (no wait).
+__device__ __forceinline__ void tst16u(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+// Kernel layout.  One CTA of 256 threads per (lane tile of 128 lanes, split, group); two CTAs
+// share an SM (about 86 KB of shared memory and 256 tensor-memory columns each), so one CTA's
+// waits are covered by the other's work.  Warp w reads TMEM lane quarter w % 4 and handles
+// positions [32 (w / 4), 32 (w / 4) + 32) of a tile of 64; row group rg = warps rg, rg + 4.
+// Tensor memory: S/P of tile buffers 0, 1 at columns [0, 64), [64, 128) (P over S in place:
+// positions 16 j .. 16 j + 15 at columns 16 j, 8 columns of P_hi then 8 of P_lo); O at
+// [128, 128 + D).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float scale) {
+__global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float scale) {
     constexpr int KBD = D / 64;                 // 128-byte blocks along d (bf16)
     constexpr int PR = D + 4;
-    constexpr int TCOLS = 256;                  // S: columns [0,128), O: [128, 128+D)
+    constexpr uint32_t TCOLS = 256;
+    constexpr uint32_t kColO = 128;
     constexpr int kPart = kPos / kParts;        // positions per warp of a row (32)
+    constexpr int kRgPos = kPos / 4;            // positions a row group resolves and gathers (16)
     constexpr float kLog2e = 1.4426950408889634f;
+    static_assert(kPart == 32, "a warp's part of a tile is one 32-bit membership word");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte aligned start, reached by pointer arithmetic on the shared array so that every
     // pointer derived from it stays a shared-memory pointer (plain shared loads and stores)
     unsigned char* base = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
-    unsigned char* sQ = base;                               // KBD blocks
-    unsigned char* sK = sQ + KBD * kBlock;                  // KBD blocks
-    unsigned char* sV0 = sK + KBD * kBlock;                 // 2 x KBD blocks (MN-major, double buffer)
-    unsigned char* sPh = sV0 + 2 * KBD * kBlock;            // 2 blocks
-    unsigned char* sPl = sPh + 2 * kBlock;                  // 2 blocks
-    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sPl + 2 * kBlock);  // [2][kPos] token (-1: none)
+    unsigned char* sQ = base;                               // KBD blocks of 128 rows
+    unsigned char* sK = sQ + KBD * kBlock;                  // KBD blocks of kPos rows (K-major)
+    unsigned char* sV0 = sK + KBD * kBlockT;                // 2 x KBD blocks (MN-major, double buffer)
+    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sV0 + 2 * KBD * kBlockT);   // [2][kPos] token (-1: none)
     int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: union index, -1 all, -2 none
-    uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_slot0 + 2 * kPos);   // [2][kPos] slot of each position
-    uint32_t* s_valid0 = reinterpret_cast<uint32_t*>(s_pslot0 + 2 * kPos); // [2][kPos/32] positions with a token
-    uint32_t* s_mw0 = s_valid0 + 2 * (kPos / 32);                          // [2][4][kPos] lane masks: [lane word][slot]
-    float* s_xmax = reinterpret_cast<float*>(s_mw0 + 2 * kPos * 4);        // [kParts][kRows] tile max per part
+    uint32_t* s_mw0 = reinterpret_cast<uint32_t*>(s_slot0 + 2 * kPos);     // [2][4][kPos] lane masks: [lane word][slot]
+    uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_mw0 + 2 * 4 * kPos);  // [2][kPos] slot of each position
+    float* s_xmax = reinterpret_cast<float*>(s_pslot0 + 2 * kPos);        // [kParts][kRows] tile max per part
     float* s_xsum = s_xmax + kParts * kRows;                                // [kParts][kRows] row sums per part
-    // mbS: the S = Q K^T of a tile is done; mbO: the P V of a tile is done (O, sP and that
-    // tile's V buffer free again).  One arrival each per tile, each waited once per tile.
-    __shared__ __align__(8) uint64_t mbS, mbO;
+    // mbS: the S = Q K^T of a tile is done; mbO: the P V of a tile is done (its V buffer free
+    // again); mbDone: every MMA issued has completed.  One arrival each per completion.
+    __shared__ __align__(8) uint64_t mbS, mbO, mbDone;
     __shared__ uint32_t tmem_sh;
     __shared__ int abort_flag;
     volatile int& abort_sh = abort_flag;
@@ -172,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     const int64_t sg0 = split * SEGS;
     if (sg0 >= nseg) return;
     const int64_t npos = (min(nseg, sg0 + SEGS) - sg0) * C;
+    const int nt = (int)((npos + kPos - 1) / kPos);       // tiles of this split
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int y0 = blockIdx.x * kRows;
 
@@ -182,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbS)));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbO)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&mbDone)));
         asm volatile("fence.mbarrier_init.release.cluster;");
         abort_sh = 0;
     }
@@ -191,43 +220,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         const int y = y0 + r;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (y < b.n_gl) v = __ldg(reinterpret_cast<const uint4*>(b.Q + lane_of(b, s, g, y) * D) + c16);
-        *reinterpret_cast<uint4*>(sQ + kmaj(r, c16)) = v;
+        *reinterpret_cast<uint4*>(sQ + kmaj(r, c16, kBlock)) = v;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_sh;
-    const uint32_t tS = tmem, tO = tmem + 128;
+    const uint32_t tO = tmem + kColO;
 
-    // Row (lane) state.  Warps w, w+4, w+8, w+12 read the same TMEM lanes 32(w%4).. and share
-    // the row; `part` selects positions [32 part, 32 part + 32) and O columns [D/4 part, ...).
+    // Row (lane) state.  Warps w and w + 4 read the same TMEM lanes 32 (w % 4).. and share the
+    // row; `part` selects positions [32 part, 32 part + 32) and O columns [D/2 part, ...).
     const int part = warp >> 2;
-    const int row = (warp & 3) * 32 + lane;
+    const int rg = warp & 3;
+    const int row = rg * 32 + lane;
     const int y = y0 + row;
     const bool y_ok = y < b.n_gl;
     const int64_t x = lane_of(b, s, g, y_ok ? y : 0);
-    const uint32_t lane_t = (uint32_t)((warp & 3) * 32) << 16;
-    float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in the 4 warps of a row
+    const uint32_t lane_t = (uint32_t)(rg * 32) << 16;
+    float m_ref = -INFINITY, lsum = 0.0f;   // identical m_ref in the 2 warps of a row
 
     const int32_t* ul = w.ulist + (int64_t)grp * w.us;
     const __nv_bfloat16* Kg = sq.K + (int64_t)g * sq.ld * D;
     const __nv_bfloat16* Vg = sq.V + (int64_t)g * sq.ld * D;
-    uint32_t phS = 0, phO = 0;
-    bool first_pv = true;
 
-    // Tokens of tile p0 into buffer st (threads 0..127, one position each): sink segment
-    // (position 0 only), kept chunks, tail.  Also the slot table: slot k of the tile is the
-    // k-th segment it touches; s_slot holds the segment's index in the group's union list
-    // (-1: every lane, -2: none), s_mw the 32-lane membership words of the CTA's 128 lanes
-    // for that union chunk, s_pslot the slot of each position; s_valid marks positions
-    // holding a token.  Positions and tokens fit 32 bits (caches hold < 2^31 rows).
+    // Tokens of tile t into staging buffer t % 2: row group rg resolves positions
+    // [16 rg, 16 rg + 16) (lanes 0..15 of warp rg): sink segment (position 0 only), kept
+    // chunks, tail.  Also the slot table: slot k of the tile is the k-th segment it touches;
+    // s_slot holds the segment's index in the group's union list (-1: every lane, -2: none),
+    // s_mw the 32-lane membership words of the CTA's 128 lanes for that union chunk (copied
+    // asynchronously, with the next committed group), s_pslot the slot of each position.
+    // Positions and tokens fit 32 bits (caches hold < 2^31 rows).
     const int cs = (C & (C - 1)) == 0 ? __ffs((int)C) - 1 : -1;   // shift for power-of-two C
     const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.x * 4;
-    auto resolve = [&](int64_t p0, int st) {
-        if (tid < kPos) {
-            const int pp = (int)p0 + tid;
-            const int segl = cs >= 0 ? (pp >> cs) : pp / (int)C;     // segment within the split
+    auto resolve = [&](int t) {
+        if (part == 0 && lane < kRgPos) {
+            const int stg = t & 1;
+            const int64_t p0 = (int64_t)t * kPos;
+            const int q = kRgPos * rg + lane;                      // position in the tile
+            const int pp = (int)p0 + q;
+            const int segl = cs >= 0 ? (pp >> cs) : pp / (int)C;    // segment within the split
             const int off = pp - segl * (int)C;
             int32_t tok = -1, code = -2;
             if (pp < npos) {
@@ -238,99 +270,111 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 } else {
                     const int k = (int)(seg - has_sink);
                     if (k < nu) {
-                        const int t = ul[k] * (int)C + off;
+                        const int tk = ul[k] * (int)C + off;
                         code = k;
-                        if (t != 0 || !has_sink) tok = t;
+                        if (tk != 0 || !has_sink) tok = tk;
                     } else {
-                        const int64_t t = tail0 + (int64_t)(k - nu) * C + off;
+                        const int64_t tk = tail0 + (int64_t)(k - nu) * C + off;
                         code = -1;
-                        if (t < N) tok = (int32_t)t;
+                        if (tk < N) tok = (int32_t)tk;
                     }
                 }
             }
             const int p0s = cs >= 0 ? ((int)p0 >> cs) : (int)p0 / (int)C;
             const int slot = segl - p0s;
-            s_tok0[st * kPos + tid] = tok;
-            s_pslot0[st * kPos + tid] = (uint8_t)slot;
-            if (tid == 0 || off == 0) {
-                s_slot0[st * kPos + slot] = code;
-                // lane masks land asynchronously with the tile's K/V gather (same commit
-                // group, waited at the top of the tile that uses them); zero-filled if none
+            s_tok0[stg * kPos + q] = tok;
+            s_pslot0[stg * kPos + q] = (uint8_t)slot;
+            if (q == 0 || off == 0) {
+                s_slot0[stg * kPos + slot] = code;
                 const uint32_t* src = memb + (int64_t)(code >= 0 ? code : 0) * w.mwords;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int k = 0; k < 4; ++k)
                     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
-                                     su32(s_mw0 + (st * 4 + q) * kPos + slot)),
-                                 "l"(src + q), "r"(code >= 0 ? 4u : 0u)
+                                     su32(s_mw0 + (stg * 4 + k) * kPos + slot)),
+                                 "l"(src + k), "r"(code >= 0 ? 4u : 0u)
                                  : "memory");
             }
-            const unsigned vb = __ballot_sync(0xffffffffu, tok >= 0);
-            if (lane == 0) s_valid0[st * (kPos / 32) + warp] = vb;
         }
     };
-    // Asynchronous gather of the K (K-major) and V (MN-major) rows of buffer st's tokens;
-    // empty positions are zero-filled.
-    // Row group g (warps g, g+4, g+8, g+12: one TMEM lane quarter) gathers positions
-    // [32g, 32g + 32), the ones warp g resolved, so one 128-thread named barrier per group
-    // orders the resolve before the gather.
-    const int rg = warp & 3, rt = (warp >> 2) * 32 + lane;
-    auto issue_kv = [&](int st) {
-        for (int i = rt; i < 32 * (D / 8); i += 128) {
-            const int t = 32 * rg + i / (D / 8), c16 = i % (D / 8);
-            const int32_t tok = s_tok0[st * kPos + t];
+    // Asynchronous gather of tile t's K rows (K-major, the one K buffer) and V rows (MN-major,
+    // buffer t % 2) for the positions row group rg resolved; empty positions are zero-filled.
+    const int rt = part * 32 + lane;                               // thread within the row group
+    auto gather = [&](int t) {
+        const int stg = t & 1;
+        unsigned char* vb = sV0 + stg * KBD * kBlockT;
+        for (int i = rt; i < kRgPos * (D / 8); i += 64) {
+            const int p = kRgPos * rg + i / (D / 8), c16 = i % (D / 8);
+            const int32_t tok = s_tok0[stg * kPos + p];
             const uint32_t n = tok >= 0 ? 16u : 0u;
             const int64_t rw = tok >= 0 ? tok : 0;
             const void* gk = reinterpret_cast<const uint4*>(Kg + rw * D) + c16;
             const void* gv = reinterpret_cast<const uint4*>(Vg + rw * D) + c16;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sK + kmaj(t, c16))), "l"(gk), "r"(n) : "memory");
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sV0 + st * KBD * kBlock + mnmaj(t, c16))),
-                         "l"(gv), "r"(n) : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sK + kmaj(p, c16, kBlockT))),
+                         "l"(gk), "r"(n) : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(vb + mnmaj(p, c16))), "l"(gv),
+                         "r"(n) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-
-    // S = Q K^T of the tile whose keys sit in sK (issued by thread 0)
-    auto issue_s = [&]() {
+    // S = Q K^T of the tile whose keys sit in sK into S/P buffer t % 2 (thread 0)
+    auto issue_s = [&](int t) {
         const uint32_t q0 = su32(sQ), k0 = su32(sK);
+        const uint32_t dS = tmem + (uint32_t)((t & 1) * kPos);
 #pragma unroll
         for (int kb = 0; kb < KBD; ++kb)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t off = kb * kBlock + kk * 32;
-                mma_bf16(tS, desc_sw128(q0 + off, 16, 1024), desc_sw128(k0 + off, 16, 1024), idesc_bf16(kPos, 0),
-                         (kb | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(dS, desc_sw128(q0 + kb * kBlock + kk * 32, 16, 1024),
+                         desc_sw128(k0 + kb * kBlockT + kk * 32, 16, 1024), idesc_bf16(kPos, 0), (kb | kk) ? 1u : 0u);
+        commit(su32(&mbS));
+    };
+    // O += P_hi V + P_lo V of tile t (P in S/P buffer t % 2, V in buffer t % 2; thread 0)
+    auto issue_pv = [&](int t) {
+        const uint32_t tP = tmem + (uint32_t)((t & 1) * kPos);
+        const uint32_t v0 = su32(sV0 + (t & 1) * KBD * kBlockT);
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+            for (int j = 0; j < kPos / 16; ++j)
+                mma_bf16_ts(tO, tP + (uint32_t)(16 * j + 8 * pass), desc_sw128(v0 + j * 2048, kBlockT, 1024),
+                            idesc_bf16(D, 1), (t == 0 && pass == 0 && j == 0) ? 0u : 1u);
+        commit(su32(&mbO));
+    };
+    auto give_up = [&]() {
+        if (lane == 0) {
+            atomicOr(w.status, kStatusTimeout);
+            abort_sh = 1;
+        }
     };
 
-    // Pipeline: tile i's S was issued at the end of the previous iteration, ahead of tile
-    // i-1's P V, so the softmax of tile i waits only for S; the P V runs under tile i's
-    // membership and row maxima and is waited for just before O, sP or its V buffer is
-    // reused.  Tile i's K/V were gathered during tile i-1's softmax.
-    resolve(0, 0);
+    // Pipeline: tile t + 1's S is issued at the end of iteration t, ahead of tile t's P V, so
+    // tile t + 1's softmax waits only for S; tile t's P V runs under tile t + 1's membership
+    // and row maxima and is waited for before O is rescaled or its V buffer refilled.  Tile
+    // t + 1's K/V are gathered during tile t's softmax.  S of tile t + 1 goes to the S/P
+    // buffer of tile t - 1, whose P V has completed by then.
+    resolve(0);
     __syncthreads();
-    issue_kv(0);
+    gather(0);
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
-    if (tid == 0) {
-        issue_s();
-        commit(su32(&mbS));
-    }
+    if (tid == 0) issue_s(0);
     __syncwarp();
-    int st = 0;
-    for (int64_t p0 = 0; p0 < npos; p0 += kPos, st ^= 1) {
-        const bool more = p0 + kPos < npos;
+    for (int t = 0; t < nt; ++t) {
+        const int stg = t & 1;
+        const int64_t p0 = (int64_t)t * kPos;
+        const bool more = t + 1 < nt;
 
         // This row's membership on its part of the tile from the staged lane masks.  When C
-        // divides 8 (tiles start on multiples of 128 positions) the part holds 32/C whole
-        // slots, a multiple of 4: gather their bits (vector loads of the lane word's slot row)
-        // and spread each over its C positions; otherwise walk the slots.
+        // divides 32 and is at most 8 (tiles start on multiples of 64 positions) the part holds
+        // 32/C whole slots, a multiple of 4: gather their bits (vector loads of the lane
+        // word's slot row) and spread each over its C positions; otherwise walk the slots.
         uint32_t mem = 0;
         {
             const int hs = part * kPart;
             const int lw = row >> 5, bit = row & 31;
-            const uint32_t* mrow = s_mw0 + (st * 4 + lw) * kPos;
-            const int32_t* codes = s_slot0 + st * kPos;
+            const uint32_t* mrow = s_mw0 + (stg * 4 + lw) * kPos;
+            const int32_t* codes = s_slot0 + stg * kPos;
             if (C <= 8 && 32 % C == 0) {               // slot rows read as 16-byte vectors
                 const int ns_ = 32 / (int)C, k0 = hs / (int)C;
                 uint32_t sb = 0;                       // bit k: slot k0 + k holds the row
@@ -349,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 for (int k = 0; k < ns_; ++k)
                     if ((sb >> k) & 1u) mem |= ones << (k * (int)C);
             } else {
-                const uint8_t* ps = s_pslot0 + st * kPos;
+                const uint8_t* ps = s_pslot0 + stg * kPos;
                 const int k0 = ps[hs], k1 = ps[hs + kPart - 1];
                 // slot k spans positions [k C - o0, (k+1) C - o0) of the tile, o0 = p0 mod C
                 const int o0 = (int)(p0 % C);
@@ -363,49 +407,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                     }
                 }
             }
-            mem &= s_valid0[st * (kPos / 32) + part];
+            mem &= __ballot_sync(0xffffffffu, s_tok0[stg * kPos + hs + lane] >= 0);   // positions with a token
             if (!y_ok) mem = 0;
         }
-        if (more) resolve(p0 + kPos, st ^ 1);
-        if (!wait_phase(su32(&mbS), phS) && lane == 0) {
-            atomicOr(w.status, kStatusTimeout);
-            abort_sh = 1;
-        }
-        phS ^= 1;
+        if (more) resolve(t + 1);
+        if (!wait_phase(su32(&mbS), (uint32_t)(t & 1))) give_up();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-        // tile max over this part's member positions, combined with the row's other parts
+        // tile max over this part's member positions, combined with the row's other part
+        const uint32_t tS = tmem + lane_t + (uint32_t)((t & 1) * kPos + part * kPart);
         float tmax = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < kPart / 16; ++c) {
             float v[16];
-            tld16(tS + lane_t + part * kPart + c * 16, v);
+            tld16(tS + c * 16, v);
             const uint32_t m16 = mem >> (c * 16);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 if ((m16 >> i) & 1u) tmax = fmaxf(tmax, v[i]);
         }
         s_xmax[part * kRows + row] = tmax;
-        // the previous tile's P V must be done before O is rescaled, sP rewritten and its V
-        // buffer refilled by the gather below
-        if (!first_pv) {
-            if (!wait_phase(su32(&mbO), phO) && lane == 0) {
-                atomicOr(w.status, kStatusTimeout);
-                abort_sh = 1;
-            }
-            phO ^= 1;
+        // the previous tile's P V must be done before O is rescaled and its V buffer refilled
+        if (t > 0) {
+            if (!wait_phase(su32(&mbO), (uint32_t)((t - 1) & 1))) give_up();
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         }
-        // partner maxima of the row and the next tile's tokens (resolved by warp rg of this
-        // group) visible to the group: every thread passes here once per tile
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + rg) : "memory");
-        if (more) issue_kv(st ^ 1);            // overlaps this tile's softmax and P V
-        tmax = fmaxf(fmaxf(s_xmax[row], s_xmax[kRows + row]), fmaxf(s_xmax[2 * kRows + row], s_xmax[3 * kRows + row]));
+        // partner maximum of the row and the next tile's tokens (resolved in this row group)
+        // visible to the group
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + rg) : "memory");
+        if (more) gather(t + 1);               // K: this tile's S is done; V: buffer (t + 1) % 2
+        tmax = fmaxf(s_xmax[row], s_xmax[kRows + row]);
         tmax = tmax > -INFINITY ? scale * tmax : -INFINITY;
 
-        // Raise the row's reference max if the tile exceeds it by more than kLazy; the 4 warps
+        // Raise the row's reference max if the tile exceeds it by more than kLazy; both warps
         // of the row take the same decision.  O is rescaled warp-collectively (factor 1 on
-        // rows that keep theirs), each warp its quarter of the columns.
+        // rows that keep theirs), each warp its half of the columns.
         const bool need = tmax > -INFINITY && m_ref > -INFINITY && tmax > m_ref + kLazy;
         const float f = need ? exp2f((m_ref - tmax) * kLog2e) : 1.0f;
         if (tmax > -INFINITY && m_ref == -INFINITY) m_ref = tmax;
@@ -413,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
             lsum *= f;
             m_ref = tmax;
         }
-        if (__any_sync(0xffffffffu, need) && !first_pv) {
+        if (__any_sync(0xffffffffu, need) && t > 0) {
 #pragma unroll 1
             for (int c = 0; c < D / (16 * kParts); ++c) {
                 float o[16];
@@ -424,14 +460,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 tst16(col, o);
             }
         }
-        // P = exp(s S - m) on member positions, split into bf16 hi + lo
+        // P = exp(s S - m) on member positions, split into bf16 hi + lo, written over S
         const float sl = scale * kLog2e, ml = m_ref * kLog2e;
 #pragma unroll 1
         for (int c = 0; c < kPart / 16; ++c) {
             float v[16];
-            tld16(tS + lane_t + part * kPart + c * 16, v);
+            tld16(tS + c * 16, v);
             const uint32_t m16 = mem >> (c * 16);
-            uint32_t hi[8], lo[8];
+            uint32_t pk[16];                      // 8 columns of P_hi, then 8 of P_lo
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
                 const float2 a2 = __ffma2_rn(make_float2(sl, sl), make_float2(v[i], v[i + 1]), make_float2(-ml, -ml));
@@ -442,65 +478,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
                 lsum += p0v;
                 lsum += p1v;
                 // bf16 hi = p rounded to 8 significant bits (integer add on the bits), lo =
-                // the exact remainder rounded likewise; packed by byte permutes, so the split
-                // stays off the conversion unit
+                // the exact remainder rounded likewise; packed by byte permutes (even position
+                // in the low half), so the split stays off the conversion unit
                 const uint32_t h0 = (__float_as_uint(p0v) + 0x8000u) & 0xffff0000u;
                 const uint32_t h1 = (__float_as_uint(p1v) + 0x8000u) & 0xffff0000u;
                 const uint32_t l0 = __float_as_uint(p0v - __uint_as_float(h0)) + 0x8000u;
                 const uint32_t l1 = __float_as_uint(p1v - __uint_as_float(h1)) + 0x8000u;
-                hi[i / 2] = __byte_perm(h0, h1, 0x7632);
-                lo[i / 2] = __byte_perm(l0, l1, 0x7632);
+                pk[i / 2] = __byte_perm(h0, h1, 0x7632);
+                pk[8 + i / 2] = __byte_perm(l0, l1, 0x7632);
             }
-            // positions 32 part + 16 c .. +15 are 16-byte chunks 4 part + 2c, +1 of this row
-            const int c16 = part * 4 + 2 * c;
-            *reinterpret_cast<uint4*>(sPh + kmaj(row, c16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(sPh + kmaj(row, c16 + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-            *reinterpret_cast<uint4*>(sPl + kmaj(row, c16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            *reinterpret_cast<uint4*>(sPl + kmaj(row, c16 + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            tst16u(tS + c * 16, pk);
         }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         // the next tile's K/V (gathered during this softmax) and lane masks must have landed
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0) {
-            // S of the next tile first (it reads only sQ / sK and writes the S columns, which
-            // this tile has finished reading), then this tile's P V
-            if (more && !abort_sh) {
-                issue_s();
-                commit(su32(&mbS));
-            }
-            const uint32_t v0 = su32(sV0 + st * KBD * kBlock);
-#pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
-                const uint32_t a0 = su32(pass == 0 ? sPh : sPl);
-#pragma unroll
-                for (int ks = 0; ks < kPos / 16; ++ks) {
-                    // A: K-major P, 16 positions = 32 bytes; B: MN-major V, 16 tokens = 2 atoms
-                    const uint32_t aoff = (ks >> 2) * kBlock + (ks & 3) * 32;
-                    const uint32_t boff = ks * 2048;
-                    mma_bf16(tO, desc_sw128(a0 + aoff, 16, 1024), desc_sw128(v0 + boff, kBlock, 1024),
-                             idesc_bf16(D, 1), (first_pv && pass == 0 && ks == 0) ? 0u : 1u);
-                }
-            }
-            commit(su32(&mbO));
+        if (tid == 0 && !abort_sh) {
+            if (more) issue_s(t + 1);
+            issue_pv(t);
         }
         __syncwarp();
-        first_pv = false;
         if (abort_sh) break;
     }
-    // the commit of the last tile (its P V): wait once more, then O is final
-    if (!wait_phase(su32(&mbO), phO) && lane == 0) {
-        atomicOr(w.status, kStatusTimeout);
-        abort_sh = 1;
+    // every MMA issued above completes before O is read and tensor memory is released
+    if (tid == 0) {
+        commit(su32(&mbDone));
+        if (!wait_phase(su32(&mbDone), 0)) give_up();
     }
-    phO ^= 1;
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // partial (o, m, l) of every lane row of the tile: each warp writes its quarter of o
     s_xsum[part * kRows + row] = lsum;
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    // partial (o, m, l) of every lane row of the tile: each warp writes its half of o
     {
         float* pp = w.part + (x * w.s_cap + split) * PR;
 #pragma unroll 1
@@ -517,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
         }
         if (part == 0 && y_ok && !abort_sh) {
             pp[D] = m_ref;
-            pp[D + 1] = (s_xsum[row] + s_xsum[kRows + row]) + (s_xsum[2 * kRows + row] + s_xsum[3 * kRows + row]);
+            pp[D + 1] = s_xsum[row] + s_xsum[kRows + row];
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -530,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(Batch b, Work w, float 
 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
-    return (size_t)(4 * kbd + 4) * kBlock + 2 * kPos * 4 + 2 * kPos * 4 + 2 * kPos + 2 * (kPos / 32) * 4 +
-           2 * kPos * 4 * 4 + 2 * kParts * kRows * 4 + 1024;
+    return (size_t)kbd * kBlock + (size_t)3 * kbd * kBlockT + 2 * kPos * 4 + 2 * kPos * 4 + 2 * 4 * kPos * 4 +
+           2 * kPos + 2 * kParts * kRows * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
