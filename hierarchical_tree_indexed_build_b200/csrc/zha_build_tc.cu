@@ -24,18 +24,21 @@
 //            folds level 2 (4 chunks = the rows of 4 neighbouring lanes: a butterfly
 //            reduce-scatter, each lane keeping a quarter of the dimensions) and level 3 (16
 //            chunks = two groups: the first group's level-2 rows pass through shared memory
-//            to the other epilogue warpgroup).  The parents' b follow from the children's:
+//            to the warpgroup that takes the second).  The parents' b follow from the children's:
 //            s q_r.m_r(P) = sum_c exp(lse_c - lse_P) (lse_c - b_c).  Levels above 3 come from
 //            k_merge.
 // A node's summary depends only on its own rows of K (other rows enter with weight exactly
 // 0 and rows past the cache read as 0), so a tile recomputed by an append gives the same
 // bits as the full build.
 //
-// Warp roles (320 threads): warp 0 TMA loads of K tiles; warp 1 MMA issue (one thread);
-// warpgroups A (warps 2-5) and B (warps 6-9) each own one pair of tensor-memory buffers (S:
-// 32 columns, m: d columns) and one set of weight planes, and take the even / odd groups.  Every
-// wait is bounded (about 2 s); a wait that gives up sets bit 1 of the tree's flag word (the
-// routing calls report it as a device status) and the CTA drains and leaves.
+// Warp roles (448 threads): warp 0 TMA loads of K tiles; warp 1 MMA issue (one thread);
+// epilogue warpgroups 0, 1, 2 (warps 2-5, 6-9, 10-13) take groups q = w, w + 3, ... of the
+// CTA's sequence; each owns a pair of tensor-memory buffers (S: 32 columns, m: d columns) and
+// three weight planes of 32 tokens (warpgroups 0 and 1 share one set of 128-byte rows, each
+// its half).  Three warpgroups keep more record stores in flight than two.  The level-3
+// exchange goes through one of two shared-memory buffers by the parity of the group pair.
+// Every wait is bounded (about 2 s); a wait that gives up sets bit 1 of the tree's flag word
+// (the routing calls report it as a device status) and the CTA drains and leaves.
 #include <math.h>
 
 #include <algorithm>
@@ -131,7 +134,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 
 // Starts the load of 32 consecutive columns of this thread's tensor-memory lane into r; the
-// registers hold the values only after tld_wait().
+// registers hold the values only after tld_wait(r).
 __device__ __forceinline__ void tld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -143,8 +146,7 @@ __device__ __forceinline__ void tld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr)
         : "memory");
 }
-__device__ __forceinline__ void tld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// The same wait, with the loaded registers as its operands, so that no use of them can be
+// The wait for it, with the loaded registers as its operands, so that no use of them can be
 // scheduled before it.
 __device__ __forceinline__ void tld_wait(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
@@ -189,8 +191,6 @@ __device__ __forceinline__ float lse2f(float a, float b) {
     return m + __logf(__expf(a - m) + __expf(b - m));
 }
 
-// fp16 hi and lo planes of n consecutive m values at hp / lp (n = 8: 16 bytes each;
-// n = 4: 8 bytes each); `bad` for |m| >= 65504.
 // One 32-byte store (a whole sector) of 8 32-bit words.
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
     asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
@@ -214,6 +214,8 @@ __device__ __forceinline__ void store_planes16(const float* v, __half* hp, __hal
     st_global_v8(lp, l);
 }
 
+// fp16 hi and lo planes of n consecutive m values at hp / lp (n = 8: 16 bytes each;
+// n = 4: 8 bytes each); `bad` for |m| >= 65504.
 template <int n>
 __device__ __forceinline__ void store_planes(const float* v, __half* hp, __half* lp, bool& bad) {
     uint32_t h[n / 2], l[n / 2];
@@ -242,27 +244,32 @@ struct Smem {
     static constexpr int kQBytes = KB * kBlk;             // q_r over 128 rows
     static constexpr int kWBytes = kBlk;                  // one weight plane (128 rows x 64 tokens)
     static constexpr int kXFloats = kR * 2 * D;           // level-2 exchange [r][P][d]
+    // two sets of weight planes (warpgroups 0 and 1 in the halves of set 0, warpgroup 2 in
+    // set 0's layout of set 1) and two level-3 exchange buffers
     static constexpr size_t bytes = (size_t)kStagesK * kTileBytes + kQBytes + 2 * kWPlanes * (size_t)kWBytes +
-                                    (size_t)kXFloats * 4 + (size_t)kR * 2 * 2 * 4 + 1024;
+                                    2 * ((size_t)kXFloats * 4 + (size_t)kR * 2 * 2 * 4) + 1024;
 };
 
+constexpr int kEpiWG = 3;             // epilogue warpgroups
+constexpr int kBuildThreads = 64 + 128 * kEpiWG;
+
 template <int D>
-__global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUtensorMap kmap, BuildTcArgs a) {
+__global__ void __launch_bounds__(kBuildThreads, 1) k_build_tc(const __grid_constant__ CUtensorMap kmap, BuildTcArgs a) {
     using S = Smem<D>;
     constexpr int KB = S::KB;
     constexpr uint32_t kColS = 0;          // S of warpgroup w: columns 32 w
-    constexpr uint32_t kColM = 64;         // m of warpgroup w: columns 64 + w D
+    constexpr uint32_t kColM = 32 * kEpiWG;   // m of warpgroup w: columns 96 + w D
     constexpr uint32_t kCols = 512;
     static_assert(kColM + 2 * D <= kCols, "tensor memory");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sK = base;                                       // [kStagesK][tile]
     unsigned char* sQ = sK + kStagesK * S::kTileBytes;              // A of MMA 1
-    unsigned char* sW = sQ + S::kQBytes;                            // [wg][plane][kWBytes]
-    float* sX = reinterpret_cast<float*>(sW + 2 * kWPlanes * S::kWBytes);   // level-2 exchange [r][P][D]
-    float* sXl = sX + S::kXFloats;                                  // its (lse, lse - b) [r][P][2]
-    __shared__ __align__(8) uint64_t bK_full[kStagesK], bK_empty[kStagesK], bS_full[2], bS_empty[2], bW_full[2],
-        bM_full[2], bM_empty[2], bX_full, bX_empty, bDone;
+    unsigned char* sW = sQ + S::kQBytes;                            // [set][plane][kWBytes]
+    float* sX0 = reinterpret_cast<float*>(sW + 2 * kWPlanes * S::kWBytes);  // [2] level-2 exchange [r][P][D]
+    float* sXl0 = sX0 + 2 * S::kXFloats;                            // [2] its (lse, s q.m) [r][P][2]
+    __shared__ __align__(8) uint64_t bK_full[kStagesK], bK_empty[kStagesK], bS_full[kEpiWG], bS_empty[kEpiWG],
+        bW_full[kEpiWG], bM_full[kEpiWG], bM_empty[kEpiWG], bX_full[2], bX_empty[2], bDone;
     __shared__ uint32_t tmem_sh;
     __shared__ int abort_flag;
     volatile int& abort_sh = abort_flag;
@@ -282,15 +289,17 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
             mbar_init(su32(&bK_full[i]), 1);
             mbar_init(su32(&bK_empty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kEpiWG; ++i) {
             mbar_init(su32(&bS_full[i]), 1);
             mbar_init(su32(&bS_empty[i]), 128);
             mbar_init(su32(&bW_full[i]), 128);
             mbar_init(su32(&bM_full[i]), 1);
             mbar_init(su32(&bM_empty[i]), 128);
         }
-        mbar_init(su32(&bX_full), 128);
-        mbar_init(su32(&bX_empty), 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(su32(&bX_full[i]), 128);
+            mbar_init(su32(&bX_empty[i]), 128);
+        }
         mbar_init(su32(&bDone), 1);
         asm volatile("fence.mbarrier_init.release.cluster;");
         abort_sh = 0;
@@ -336,11 +345,11 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issue (one thread).  Group q = 4 i + g of tile i uses the
-        // buffers of warpgroup q & 1 for the (q >> 1)-th time.
+        // buffers of warpgroup q % 3 for the (q / 3)-th time.
         if (lane == 0) {
             const int nq = nt * kGroups;
             auto mma1 = [&](int q) -> bool {
-                const int i = q / kGroups, g = q % kGroups, w = q & 1, u = q >> 1, st = i % kStagesK;
+                const int i = q / kGroups, g = q % kGroups, w = q % kEpiWG, u = q / kEpiWG, st = i % kStagesK;
                 if (g == 0 && !mbar_wait(su32(&bK_full[st]), (uint32_t)((i / kStagesK) & 1))) return false;
                 if (u >= 1 && !mbar_wait(su32(&bS_empty[w]), (uint32_t)((u - 1) & 1))) return false;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -358,14 +367,15 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                 return true;
             };
             auto mma2 = [&](int q) -> bool {
-                const int i = q / kGroups, g = q % kGroups, w = q & 1, u = q >> 1, st = i % kStagesK;
+                const int i = q / kGroups, g = q % kGroups, w = q % kEpiWG, u = q / kEpiWG, st = i % kStagesK;
                 if (!mbar_wait(su32(&bW_full[w]), (uint32_t)(u & 1))) return false;
                 if (u >= 1 && !mbar_wait(su32(&bM_empty[w]), (uint32_t)((u - 1) & 1))) return false;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t k0 = su32(sK + (size_t)st * S::kTileBytes) + g * kGroupTok * 128;
 #pragma unroll
                 for (int pl = 0; pl < kWPlanes; ++pl) {
-                    const uint32_t a0 = su32(sW + (w * kWPlanes + pl) * S::kWBytes);
+                    // warpgroup w's 32 tokens: bytes 64 (w & 1) .. of the rows of set w >> 1
+                    const uint32_t a0 = su32(sW + ((w >> 1) * kWPlanes + pl) * S::kWBytes) + (w & 1) * 64;
 #pragma unroll
                     for (int ks = 0; ks < kGroupTok / 16; ++ks)
                         mma(tmem + kColM + w * D, desc_sw128(a0 + ks * 32, 16, 1024),
@@ -391,7 +401,7 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
         __syncwarp();
     } else {
         // ---------------- epilogue warpgroups: thread = TMEM lane r*8 + j
-        const int w = (warp - 2) >> 2;                       // warpgroup: groups q with q & 1 == w
+        const int w = (warp - 2) >> 2;                       // warpgroup: groups q with q % 3 == w
         const int quad = warp & 3;                           // TMEM lane quarter of this warp
         const int row = quad * 32 + lane;
         const int r = row >> 3, j = row & 7;
@@ -399,17 +409,22 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
         const uint32_t tl = (uint32_t)(quad * 32) << 16;
         const uint32_t tS = tmem + tl + kColS + w * 32;
         const uint32_t tM = tmem + tl + kColM + w * D;
-        unsigned char* wPl = sW + w * kWPlanes * S::kWBytes;   // this warpgroup's weight planes
-        const uint32_t woff = kmaj(row, j >> 1) + (j & 1) * 8;   // tokens 4j .. 4j+3 of the row
+        unsigned char* wPl = sW + (w >> 1) * kWPlanes * S::kWBytes;   // this warpgroup's weight planes
+        // tokens 4j .. 4j+3 of the row, in this warpgroup's 64-byte half of the 128-byte row
+        const uint32_t woff = kmaj(row, (j >> 1) + 4 * (w & 1)) + (j & 1) * 8;
         const int nq = nt * kGroups;
-        int npair = 0;                                       // level-3 exchanges taken part in
         bool bad = false;
         auto give_up = [&]() {
             atomicOr(a.rflag, kFlagTimeout);
             abort_sh = 1;
         };
-        for (int q = w; q < nq; q += 2) {
-            const int i = q / kGroups, g = q % kGroups, u = q >> 1;
+        for (int q = w; q < nq; q += kEpiWG) {
+            const int i = q / kGroups, g = q % kGroups, u = q / kEpiWG;
+            // level-3 exchange of group pair q >> 1: buffer (q >> 1) & 1, its (q >> 2)-th use
+            const int xb = (q >> 1) & 1;
+            const uint32_t xuse = (uint32_t)(q >> 2);
+            float* sX = sX0 + xb * S::kXFloats;
+            float* sXl = sXl0 + xb * (kR * 2 * 2);
             const int64_t t = a.t0 + blockIdx.x + (int64_t)i * gridDim.x;
             // -- scores of chunk j, softmax, weights, b
             if (!mbar_wait(su32(&bS_full[w]), (uint32_t)(u & 1))) give_up();
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
             const bool lv3 = a.k_emit >= 3;
             float l3 = 0.0f, wX0 = 0.0f, wX1 = 0.0f, w32 = 0.0f, wa3 = 0.0f;
             if (lv3 && second) {
-                if (!mbar_wait(su32(&bX_full), (uint32_t)(npair & 1))) give_up();
+                if (!mbar_wait(su32(&bX_full[xb]), xuse & 1u)) give_up();
                 const float la0 = sXl[(r * 2 + 0) * 2], la1 = sXl[(r * 2 + 1) * 2];
                 const float lo = __shfl_xor_sync(0xffffffffu, l2, 4);   // this group's other level-2 node
                 l3 = lse2f(lse2f(la0, la1), lse2f(l2, lo));
@@ -483,8 +498,9 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                 y += __shfl_xor_sync(0xffffffffu, y, 4);
                 wa3 = fmaf(wX0, sXl[(r * 2 + 0) * 2 + 1], wX1 * sXl[(r * 2 + 1) * 2 + 1]) + y;
             }
-            if (lv3 && !second && npair >= 1) {
-                if (!mbar_wait(su32(&bX_empty), (uint32_t)((npair - 1) & 1))) give_up();   // partner read the last one
+            if (lv3 && !second && xuse >= 1) {
+                // the second group of this buffer's previous pair has read it
+                if (!mbar_wait(su32(&bX_empty[xb]), (xuse - 1) & 1u)) give_up();
             }
 
             if (!mbar_wait(su32(&bM_full[w]), (uint32_t)(u & 1))) give_up();
@@ -568,15 +584,14 @@ __global__ void __launch_bounds__(320, 1) k_build_tc(const __grid_constant__ CUt
                         sXl[(r * 2 + P) * 2] = l2;
                         sXl[(r * 2 + P) * 2 + 1] = wa2;
                     }
-                    mbar_arrive(su32(&bX_full));            // this pair's exchange is written
+                    mbar_arrive(su32(&bX_full[xb]));        // this pair's exchange is written
                 } else {
                     if (st3 && j == 0) {
                         reinterpret_cast<float*>(r3)[kR * D + r] = l3 - wa3;
                         a.lse[3][((int64_t)hg * a.cap[3] + j3) * kR + r] = l3;
                     }
-                    mbar_arrive(su32(&bX_empty));           // exchange read
+                    mbar_arrive(su32(&bX_empty[xb]));       // exchange read
                 }
-                ++npair;
             }
         }
         if (bad) atomicOr(a.rflag, kFlagRange);
@@ -624,11 +639,11 @@ cudaError_t launch_build_tc(const BuildTcArgs& a, int d, cudaStream_t st) {
     if (d == 128) {
         const size_t smem = Smem<128>::bytes;
         cudaFuncSetAttribute(k_build_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_build_tc<128><<<grid, 320, smem, st>>>(map, a);
+        k_build_tc<128><<<grid, kBuildThreads, smem, st>>>(map, a);
     } else {
         const size_t smem = Smem<64>::bytes;
         cudaFuncSetAttribute(k_build_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_build_tc<64><<<grid, 320, smem, st>>>(map, a);
+        k_build_tc<64><<<grid, kBuildThreads, smem, st>>>(map, a);
     }
     return cudaGetLastError();
 }
