@@ -302,7 +302,21 @@ def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--k", type=int, nargs="+", default=[64, 1024],
                     help="kept nodes per lane per level (fixed budget) for the projections")
+    ap.add_argument("--record", nargs="+", metavar="LOG",
+                    help="rewrite the recorded measurements from the JSON lines of `bench.py --stage-sweep` "
+                         "logs (one per command in --commands), then fit")
+    ap.add_argument("--commands", nargs="+", default=[], help="the commands that wrote the --record logs")
     args = ap.parse_args()
+    if args.record:
+        runs = []
+        for path in args.record:
+            with open(path) as fh:
+                runs += [json.loads(l) for l in fh if l.startswith("{") and '"stage"' in l]
+        with open(MEASURED, "w") as fh:
+            json.dump({"what": "per-kernel device times (ms per call, the library's CUDA-event profile) and "
+                               "decoder work counters of the build and of the decode at several p, one B200",
+                       "commands": args.commands, "runs": runs}, fh, indent=1)
+        print("recorded %d runs into %s" % (len(runs), MEASURED))
     pk = peaks()
     runs = load_measured()
     f, resid = fit(points_from_runs(runs), pk)
