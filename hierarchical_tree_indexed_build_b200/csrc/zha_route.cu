@@ -510,18 +510,16 @@ __device__ __forceinline__ void hist_add(uint32_t alo, uint32_t ahi, uint32_t lo
 struct SelMath {
     float nl2M;     // -M log2(e)
     float m64;      // M kBinScale
-    // fixed-point mass floor(exp(e - M) 2^39) as 32-bit words (lo, hi), read from the bits of
-    // the float f = exp(e - M) in [0, 1]: the 24-bit significand shifted by exponent - 111
-    // (2^39 / 2^23 = 2^16 at f = 1), without branches: the clamped funnel shifts give 0 for
-    // shifts of 32 or more, which covers f = 0 (exponent field 0, shift -111)
+    // fixed-point mass floor(exp(e - M) 2^39) as 32-bit words (lo, hi): f = exp(e - M) in
+    // [0, 1] (flushed to 0 below the normal range) times 2^39 is exact in float32, and its
+    // truncation to a 64-bit integer is the floor; one conversion on the otherwise lightly
+    // used conversion pipe instead of shifts and selects on the integer pipe
     __device__ __forceinline__ void mass2(float e, uint32_t& lo, uint32_t& hi) const {
         const float f = ex2_approx(fmaf(e, 1.4426950408889634f, nl2M));
-        const uint32_t u = __float_as_uint(f);
-        const int sh = (int)(u >> 23) - 111;                                  // f >= 0: no sign bit
-        const uint32_t mant = (u & 0x7fffffu) | 0x800000u;
-        const uint32_t up = (uint32_t)max(sh, 0), dn = (uint32_t)max(-sh, 0);
-        hi = __funnelshift_lc(mant, 0u, up);                                  // (0:mant) << up, high word
-        lo = __funnelshift_rc(__funnelshift_lc(0u, mant, up), 0u, dn);        // low word, then >> dn
+        unsigned long long m;
+        asm("cvt.rzi.u64.f32 %0, %1;" : "=l"(m) : "f"(f * 549755813888.0f));   // 2^39
+        lo = (uint32_t)m;
+        hi = (uint32_t)(m >> 32);
     }
     __device__ __forceinline__ unsigned long long mass(float e) const {
         uint32_t lo, hi;
