@@ -776,6 +776,9 @@ def cpu_baseline(wl, p, min_s=10.0, max_queries=64):
 def base_line(args, world, wl):
     seq = wl.seqs[0]
     g = seq.geom
+    n = seq.n_tokens + wl.n_append
+    kv_gb = 2 * g.Hkv * n * g.d * 2 / 1e9
+    tree_gb = g.Hkv * sum(n // g.C ** l for l in range(1, g.L + 1)) * (g.R * g.d + 2 * g.R) * 4 / 1e9
     return {
         "metric": METRIC, "unit": "queries/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -783,7 +786,8 @@ def base_line(args, world, wl):
                    "n_queries": int(wl.Q.shape[2]), "p": args.p, "C": g.C, "L": g.L, "R": g.R, "d": g.d,
                    "Hq": g.Hq, "Hkv": g.Hkv, "step": "build + append + decode of all queries",
                    "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (K+V 1.08 GB, tree 5.8 GB), no flush"},
+                   "inputs": "bf16 K, V, Q and reference queries; f32 summaries, scores and outputs",
+                   "l2": "inputs larger than L2 (K+V %.2f GB, tree %.2f GB; L2 126 MB), no flush" % (kv_gb, tree_gb)},
     }
 
 
