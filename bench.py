@@ -492,7 +492,7 @@ def fp4_measure(args, dev, stream, zha, seq, K, V, qref, Q, N0, n_app, dec, out)
         st = d.stats()
         obj["one_query_decode_ms"][name] = a.elapsed_time(b) / args.steps
         obj["node_bytes"][name] = st.node_bytes
-        for kn in ("k_score_few", "k_score"):
+        for kn in ("k_score_tc", "k_score_few", "k_score"):
             if kn in pr:
                 la, tms = pr[kn]
                 nb = sum(st.union_nodes) * st.node_bytes

@@ -75,7 +75,6 @@ cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cud
 cudaError_t launch_member(const Batch& b, const Work& w, int it, int mode, cudaStream_t st);
 cudaError_t launch_score_tc(const Batch& b, const Work& w, int it, float scale, cudaStream_t st);
 // Lanes per group from which the automatic choice scores on tensor cores.
-constexpr int kTensorScoreMinLanes = 64;
 // max_cands: an upper bound on any lane's candidates at this iteration (picks the block size).
 cudaError_t launch_select(const Batch& b, const Work& w, int it, int64_t max_cands, cudaStream_t st);
 cudaError_t launch_attn(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st);

@@ -1030,7 +1030,7 @@ cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaSt
 
 cudaError_t launch_score(const Batch& b, const Work& w, int it, float scale, cudaStream_t st) {
     const bool tc = b.all_r16 && w.tmaps && b.fmt != kFmtFp4 &&
-                    (b.score_path == 2 || (b.score_path == 0 && b.n_gl >= kTensorScoreMinLanes));
+                    (b.score_path == 2 || b.score_path == 0);
     if (tc) return launch_score_tc(b, w, it, scale, st);
     if (b.all_r16 && b.n_gl <= kFewLanes && b.d == 128) {
         // one wave: 2 blocks of 8 warps per SM, shared by the groups (d = 128, the geometry

@@ -174,9 +174,12 @@ zha_status zha_sparse_attn(zha_decoder* dec, const void* const* K, const void* c
                            const void* Q, int32_t n_q, float* out, void* stream);
 
 /* Which kernels a decoder uses (both choices give the same result up to float32
- * rounding).  ZHA_KERNELS_AUTO scores on the tensor cores (tcgen05) when a (sequence, KV
- * head) group has >= 64 lanes and every tree has R = 16, on the CUDA cores otherwise, and
- * attends on the tensor cores at every lane count; SIMT and TENSOR force one kind.
+ * rounding).  ZHA_KERNELS_AUTO scores on the tensor cores (tcgen05, records fed by TMA)
+ * at every lane count when every tree has R = 16 and fp16 or bf16 records (at one query
+ * token the node scan then runs at the HBM rate), on the CUDA cores otherwise (MXFP4
+ * records, R != 16), and attends on the tensor cores at every lane count; SIMT and TENSOR
+ * force one kind (SIMT with at most 16 lanes per group, R = 16 and d = 128 takes the
+ * few-lane CUDA-core scorer).
  *   score  plane estimates: CUDA-core fp32 FMA, or tcgen05 kind::f16 (ZHA_ERR_ARG for
  *          TENSOR unless every tree has R = 16).  With ZHA_SUMMARY_F16X2 records Q is
  *          taken in fp16 and each summary in two passes (hi, lo); the tensor path then

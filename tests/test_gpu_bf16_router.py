@@ -87,7 +87,7 @@ def test_bf16_summaries_are_rounded_exact_summaries(geom, n):
 @pytest.mark.parametrize("score,geom,n,n_q", [
     (zha.ZHA_KERNELS_TENSOR, inputs.DEEP, 8 * 4096 + 333, 8),   # 64 lanes per group: tcgen05, one bf16 pass
     (zha.ZHA_KERNELS_SIMT, inputs.DEEP, 8 * 4096 + 333, 8),     # CUDA-core scorer
-    (zha.ZHA_KERNELS_AUTO, inputs.DEEP, 8 * 4096 + 333, 2),     # 16 lanes: the few-lane scorer
+    (zha.ZHA_KERNELS_SIMT, inputs.DEEP, 8 * 4096 + 333, 2),     # 16 lanes: the few-lane CUDA-core scorer
     (zha.ZHA_KERNELS_TENSOR, inputs.MID, 3 * 4096 + 900, 8),
 ])
 def test_bf16_router_matches_replay_on_its_stored_summaries(score, geom, n, n_q):

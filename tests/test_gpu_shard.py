@@ -78,7 +78,7 @@ def _check_kept(seq, n, one, sh, engines):
 @pytest.mark.parametrize("geom,n,n_q,world,score", [
     (inputs.DEEP, 3 * 4096 + 1234, 8, 2, zha.ZHA_KERNELS_AUTO),      # 64 lanes per group: tcgen05 scorer
     (inputs.DEEP, 5 * 4096 + 77, 8, 3, zha.ZHA_KERNELS_SIMT),        # CUDA-core scorer, 3 ranks
-    (inputs.DEEP, 4 * 4096, 1, 4, zha.ZHA_KERNELS_AUTO),              # one query: few-lane scorer, no tail
+    (inputs.DEEP, 4 * 4096, 1, 4, zha.ZHA_KERNELS_SIMT),              # one query: few-lane scorer, no tail
     (inputs.MID, 3 * 4096 + 500, 4, 2, zha.ZHA_KERNELS_AUTO),        # C = 16
     (inputs.WIDE, 40 * 256 + 100, 4, 3, zha.ZHA_KERNELS_TENSOR),     # C = 256, L = 1
 ])
