@@ -37,7 +37,6 @@ constexpr float kLazy = 8.0f;   // raise the running max only when exceeded by t
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on any wait for the tensor pipeline
 constexpr int kBlock = kRows * 128;   // bytes of one 128-byte-wide block of 128 rows (Q)
 constexpr int kBlockT = kPos * 128;   // the same for the tile's kPos token rows (K, V)
-constexpr int kStage = 3;             // token / lane-mask staging buffers (tiles t, t + 1, t + 2)
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -169,13 +168,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
     // pointer derived from it stays a shared-memory pointer (plain shared loads and stores)
     unsigned char* base = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sQ = base;                               // KBD blocks of 128 rows
-    unsigned char* sK0 = sQ + KBD * kBlock;                 // 2 x KBD blocks of kPos rows (K-major, double buffer)
-    unsigned char* sV0 = sK0 + 2 * KBD * kBlockT;           // 2 x KBD blocks (MN-major, double buffer)
-    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sV0 + 2 * KBD * kBlockT);   // [3][kPos] token (-1: none)
-    int32_t* s_slot0 = s_tok0 + kStage * kPos;                       // [3][kPos] per slot: union index, -1 all, -2 none
-    uint32_t* s_mw0 = reinterpret_cast<uint32_t*>(s_slot0 + kStage * kPos);   // [3][4][kPos] lane masks: [lane word][slot]
-    uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_mw0 + kStage * 4 * kPos);  // [3][kPos] slot of each position
-    float* s_xmax = reinterpret_cast<float*>(s_pslot0 + kStage * kPos);        // [kParts][kRows] tile max per part
+    unsigned char* sK = sQ + KBD * kBlock;                  // KBD blocks of kPos rows (K-major)
+    unsigned char* sV0 = sK + KBD * kBlockT;                // 2 x KBD blocks (MN-major, double buffer)
+    int32_t* s_tok0 = reinterpret_cast<int32_t*>(sV0 + 2 * KBD * kBlockT);   // [2][kPos] token (-1: none)
+    int32_t* s_slot0 = s_tok0 + 2 * kPos;                            // [2][kPos] per slot: union index, -1 all, -2 none
+    uint32_t* s_mw0 = reinterpret_cast<uint32_t*>(s_slot0 + 2 * kPos);     // [2][4][kPos] lane masks: [lane word][slot]
+    uint8_t* s_pslot0 = reinterpret_cast<uint8_t*>(s_mw0 + 2 * 4 * kPos);  // [2][kPos] slot of each position
+    float* s_xmax = reinterpret_cast<float*>(s_pslot0 + 2 * kPos);        // [kParts][kRows] tile max per part
     float* s_xsum = s_xmax + kParts * kRows;                                // [kParts][kRows] row sums per part
     // mbS: the S = Q K^T of a tile is done; mbO: the P V of a tile is done (its V buffer free
     // again); mbDone: every MMA issued has completed.  One arrival each per completion.
@@ -245,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
     const __nv_bfloat16* Kg = sq.K + (int64_t)g * sq.ld * D;
     const __nv_bfloat16* Vg = sq.V + (int64_t)g * sq.ld * D;
 
-    // Tokens of tile t into staging buffer t % 3: row group rg resolves positions
+    // Tokens of tile t into staging buffer t % 2: row group rg resolves positions
     // [16 rg, 16 rg + 16) (lanes 0..15 of warp rg): sink segment (position 0 only), kept
     // chunks, tail.  Also the slot table: slot k of the tile is the k-th segment it touches;
     // s_slot holds the segment's index in the group's union list (-1: every lane, -2: none),
@@ -256,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
     const uint32_t* memb = w.memb + (int64_t)grp * w.ms * w.mwords + (int64_t)blockIdx.x * 4;
     auto resolve = [&](int t) {
         if (part == 0 && lane < kRgPos) {
-            const int stg = t % kStage;
+            const int stg = t & 1;
             const int64_t p0 = (int64_t)t * kPos;
             const int q = kRgPos * rg + lane;                      // position in the tile
             const int pp = (int)p0 + q;
@@ -297,27 +296,29 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
             }
         }
     };
-    // Asynchronous gather of tile t's K rows (K-major) or V rows (MN-major) into buffer t % 2
-    // for the positions row group rg resolved; empty positions are zero-filled.
+    // Asynchronous gather of tile t's K rows (K-major, the one K buffer) and V rows (MN-major,
+    // buffer t % 2) for the positions row group rg resolved; empty positions are zero-filled.
     const int rt = part * 32 + lane;                               // thread within the row group
-    auto gather = [&](int t, bool is_v) {
-        const int stg = t % kStage;
-        const __nv_bfloat16* src = is_v ? Vg : Kg;
-        unsigned char* dst = (is_v ? sV0 : sK0) + (t & 1) * KBD * kBlockT;
+    auto gather = [&](int t) {
+        const int stg = t & 1;
+        unsigned char* vb = sV0 + stg * KBD * kBlockT;
         for (int i = rt; i < kRgPos * (D / 8); i += 64) {
             const int p = kRgPos * rg + i / (D / 8), c16 = i % (D / 8);
             const int32_t tok = s_tok0[stg * kPos + p];
             const uint32_t n = tok >= 0 ? 16u : 0u;
             const int64_t rw = tok >= 0 ? tok : 0;
-            const void* gsrc = reinterpret_cast<const uint4*>(src + rw * D) + c16;
-            const uint32_t o = is_v ? mnmaj(p, c16) : kmaj(p, c16, kBlockT);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(dst + o)), "l"(gsrc), "r"(n) : "memory");
+            const void* gk = reinterpret_cast<const uint4*>(Kg + rw * D) + c16;
+            const void* gv = reinterpret_cast<const uint4*>(Vg + rw * D) + c16;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(sK + kmaj(p, c16, kBlockT))),
+                         "l"(gk), "r"(n) : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(vb + mnmaj(p, c16))), "l"(gv),
+                         "r"(n) : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    auto commit_group = [&]() { asm volatile("cp.async.commit_group;" ::: "memory"); };
-    // S = Q K^T of tile t (keys in K buffer t % 2) into S/P buffer t % 2 (thread 0)
+    // S = Q K^T of the tile whose keys sit in sK into S/P buffer t % 2 (thread 0)
     auto issue_s = [&](int t) {
-        const uint32_t q0 = su32(sQ), k0 = su32(sK0 + (t & 1) * KBD * kBlockT);
+        const uint32_t q0 = su32(sQ), k0 = su32(sK);
         const uint32_t dS = tmem + (uint32_t)((t & 1) * kPos);
 #pragma unroll
         for (int kb = 0; kb < KBD; ++kb)
@@ -348,25 +349,19 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
 
     // Pipeline: tile t + 1's S is issued at the end of iteration t, ahead of tile t's P V, so
     // tile t + 1's softmax waits only for S; tile t's P V runs under tile t + 1's membership
-    // and row maxima and is waited for before O is rescaled or its V buffer refilled.  During
-    // iteration t the K rows of tile t + 2 and the V rows of tile t + 1 are gathered (one
-    // commit group), so each gather has a whole tile to land: the end of iteration t waits
-    // only for the group of iteration t - 1.  S of tile t + 1 goes to the S/P buffer of tile
-    // t - 1, whose P V has completed by then.
+    // and row maxima and is waited for before O is rescaled or its V buffer refilled.  Tile
+    // t + 1's K/V are gathered during tile t's softmax.  S of tile t + 1 goes to the S/P
+    // buffer of tile t - 1, whose P V has completed by then.
     resolve(0);
-    if (nt > 1) resolve(1);
     __syncthreads();
-    gather(0, false);
-    gather(0, true);
-    if (nt > 1) gather(1, false);
-    commit_group();
+    gather(0);
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (tid == 0) issue_s(0);
     __syncwarp();
     for (int t = 0; t < nt; ++t) {
-        const int stg = t % kStage;
+        const int stg = t & 1;
         const int64_t p0 = (int64_t)t * kPos;
         const bool more = t + 1 < nt;
 
@@ -415,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
             mem &= __ballot_sync(0xffffffffu, s_tok0[stg * kPos + hs + lane] >= 0);   // positions with a token
             if (!y_ok) mem = 0;
         }
-        if (t + 2 < nt) resolve(t + 2);
+        if (more) resolve(t + 1);
         if (!wait_phase(su32(&mbS), (uint32_t)(t & 1))) give_up();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
@@ -437,12 +432,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
             if (!wait_phase(su32(&mbO), (uint32_t)((t - 1) & 1))) give_up();
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         }
-        // partner maximum of the row and tile t + 2's tokens (resolved in this row group)
+        // partner maximum of the row and the next tile's tokens (resolved in this row group)
         // visible to the group
         asm volatile("bar.sync %0, 64;" ::"r"(1 + rg) : "memory");
-        if (t + 2 < nt) gather(t + 2, false);  // K buffer t % 2: this tile's S is done
-        if (more) gather(t + 1, true);         // V buffer (t + 1) % 2: tile t - 1's P V is done
-        commit_group();
+        if (more) gather(t + 1);               // K: this tile's S is done; V: buffer (t + 1) % 2
         tmax = fmaxf(s_xmax[row], s_xmax[kRows + row]);
         tmax = tmax > -INFINITY ? scale * tmax : -INFINITY;
 
@@ -497,9 +490,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
             tst16u(tS + c * 16, pk);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        // the next tile's K and this tile's V (gathered during the previous iteration) and the
-        // lane masks of tile t + 1 have landed; this iteration's group may still be in flight
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        // the next tile's K/V (gathered during this softmax) and lane masks must have landed
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
@@ -551,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(Batch b, Work w, float 
 
 size_t attn_tc_smem(int d) {
     const int kbd = d / 64;
-    return (size_t)kbd * kBlock + (size_t)4 * kbd * kBlockT + kStage * kPos * 4 + kStage * kPos * 4 +
-           kStage * 4 * kPos * 4 + kStage * kPos + 2 * kParts * kRows * 4 + 1024;
+    return (size_t)kbd * kBlock + (size_t)3 * kbd * kBlockT + 2 * kPos * 4 + 2 * kPos * 4 + 2 * 4 * kPos * 4 +
+           2 * kPos + 2 * kParts * kRows * 4 + 1024;
 }
 
 cudaError_t launch_attn_tc(const Batch& b, const Work& w, int64_t max_splits, float scale, cudaStream_t st) {
