@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--no-shard", action="store_true",
                     help="skip the sequence-sharded decode measurement (shards held on this one GPU)")
     ap.add_argument("--shards", type=int, default=2, help="shards of the sharded decode measurement")
+    ap.add_argument("--shard", action="store_true",
+                    help="under torchrun: one sequence split over the ranks (each rank builds its shard's "
+                         "tree and the ranks decode the queries together over NCCL); strong scaling")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the wide 256K and batched 32 x 128K measurements")
     ap.add_argument("--n-q", type=int, default=0, help="decode only the workload's first n query tokens (profiling)")
@@ -456,6 +459,71 @@ def run_ours(args, rank, world, dev):
     return res
 
 
+def run_sharded(args, rank, world, dev):
+    """One sequence split over the ranks: rank r holds its token range of the workload's cache
+    (the last rank also takes the appended tokens), builds its shard's tree and decodes the
+    workload's queries with the other ranks through the sharded protocol (NCCL collectives
+    between the select phases and for the output merge; device copies when world is 1).
+    Step = shard build + append + sharded decode; value = the job's queries per second
+    (strong scaling: the work is one sequence whatever the number of ranks)."""
+    from hierarchical_tree_indexed_build_b200 import zha
+    torch.cuda.set_device(dev)
+    wl = load_workload(args.workload)
+    seq = wl.seqs[0]
+    g = seq.geom
+    N0, n_app = seq.n_tokens, wl.n_append
+    n_all = N0 + n_app
+    off, cnt = zha.shard_ranges(n_all, g.C, g.L, world)[rank]
+    cnt0 = min(cnt, max(0, N0 - off))              # rows present before the append
+    K = seq.K[:, off:off + cnt].contiguous().to(dev)
+    V = seq.V[:, off:off + cnt].contiguous().to(dev)
+    qref = seq.qref.to(dev)
+    Q = wl.Q[0][0].contiguous().to(dev)           # [n_q][Hq][d]
+    n_q = Q.shape[0]
+    out = torch.empty((n_q, g.Hq, g.d), dtype=torch.float32, device=dev)
+    tree = zha.Tree(g.C, g.L, g.R, g.d, g.Hq, g.Hkv, cnt)
+    eng = zha.ShardedDecoder(tree, n_q, rank, world, off)
+    coll = zha.TorchCollectives() if world > 1 else None
+    stream = torch.cuda.current_stream()
+
+    def step():
+        tree.build(K, cnt0, qref)
+        if cnt > cnt0:
+            tree.append(K, cnt0, cnt - cnt0)
+        if coll is None:
+            zha.decode_local_shards([eng], [K], [V], Q, args.p, [out])
+        else:
+            zha.decode_sharded(eng, K, V, Q, args.p, out, coll=coll)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(dev)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    line = base_line(args, world, wl)
+    line["config"].update({"parallelism": "sequence sharded over %d ranks" % world,
+                           "step": "shard tree build + append + sharded decode of all queries",
+                           "shard_tokens": [c for _, c in zha.shard_ranges(n_all, g.C, g.L, world)]})
+    line.update({"scaling": "strong", "value": n_q / (ms / 1e3), "ms_per_step": ms, "clocks": clk,
+                 "impl": "ours", "vs_baseline": None})
+    eng.close()
+    tree.close()
+    return line
+
+
 def fp4_measure(args, dev, stream, zha, seq, K, V, qref, Q, N0, n_app, dec, out):
     g = seq.geom
     Q1 = Q[:, :1].contiguous()
@@ -817,6 +885,14 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
                                              timeout=__import__("datetime").timedelta(seconds=120))
+    if args.shard:
+        line = run_sharded(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     res = run_ours(args, rank, world, local)
     wl = res.pop("wl")
     if rank == 0:

@@ -171,3 +171,37 @@ def test_shard_protocol_is_enforced():
     assert ei.value.status == zha.ZHA_ERR_STATE
     for x in (e, e2):
         x.close()
+
+
+@needs_cuda
+def test_sharded_decode_through_nccl_collectives(tmp_path):
+    """The protocol over torch.distributed with the NCCL backend (one rank: the whole sequence
+    as one shard), so the collective calls themselves - in-place MAX / SUM all-reduces of int32
+    and int64 buffers and rank-major all_gather_into_tensor - run on the device; the result
+    must equal the single tree's decode."""
+    import torch.distributed as dist
+    geom = inputs.DEEP
+    n = 3 * 4096 + 321
+    seq = inputs.make_sequence(geom, n, n, seed=31)
+    Q, _ = inputs.make_queries(seq, 4, 6, n, np.random.default_rng(3))
+    one, sh, engines, outs, keep = _run(seq, n, Q, 0.9, 1)
+    own = not dist.is_initialized()
+    if own:
+        dist.init_process_group("nccl", init_method="file://" + str(tmp_path / "pg"), rank=0, world_size=1)
+    try:
+        e = engines[0]
+        out = torch.empty((Q.shape[0], geom.Hq, geom.d), dtype=torch.float32, device="cuda")
+        zha.decode_sharded(e, sh[0][3], sh[0][4], Q.cuda().contiguous(), 0.9, out)
+        torch.cuda.synchronize()
+        for lev in range(1, geom.L + 1):
+            n_l = n // geom.C ** lev
+            assert np.array_equal(TL.bits_to_bool(e.export_kept(lev)[0], n_l), one.kept[0][lev - 1]), lev
+        got = out.cpu().numpy().astype(np.float64).reshape(-1, geom.d)
+        assert TL.rel_err(got, one.out[0].reshape(-1, geom.d)).max() <= 1e-4
+    finally:
+        if own:
+            dist.destroy_process_group()
+    for x in engines:
+        x.close()
+    keep[1].close()
+    keep[0].close()
