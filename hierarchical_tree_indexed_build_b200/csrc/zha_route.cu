@@ -166,27 +166,41 @@ __global__ void __launch_bounds__(256) k_union_or(Batch b, Work w, int it, int m
     if (word) atomicOr(w.uword + (int64_t)grp * w.uw + wi, word);
 }
 
-// Compacts a group's union bitmap into the sorted list of set bits.
-__global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it, int mode) {
+// Compacts a group's union bitmap into the sorted list of set bits.  Grid (chunks, groups):
+// block c writes the entries of words [c kCompactWords, (c + 1) kCompactWords); its offset in
+// the list is the number of set bits in the words before its chunk, which the block counts
+// itself (at most a few tens of KB from L2), so one launch suffices and every chunk is written
+// in parallel (each thread one word: at most 32 entries).  The block holding the group's last
+// word writes the count.
+constexpr int kCompactThreads = 256;
+constexpr int kCompactWords = 256;
+
+__global__ void __launch_bounds__(kCompactThreads) k_union_compact(Batch b, Work w, int it, int mode) {
     __shared__ int red[33];
-    const int grp = blockIdx.x;
+    const int grp = blockIdx.y;
     const int s = grp / b.Hkv;
     const SeqDev& sq = b.seqs[s];
     const int ulev = union_level(sq, it, mode);
     if (ulev == 0) {
-        if (threadIdx.x == 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
             w.ucount[grp] = 0;
             if (mode == 1) atomicAdd(&w.ctr[kCtrUnionTokens], (unsigned long long)sq.N);   // dense: A = [0, N)
         }
         return;
     }
     const int64_t nwords = (union_limit(sq, ulev, mode) + 31) / 32;
+    const int64_t c0 = (int64_t)blockIdx.x * kCompactWords;
+    if (c0 >= nwords && !(nwords == 0 && blockIdx.x == 0)) return;   // whole block, before any barrier
     const uint32_t* uwp = w.uword + (int64_t)grp * w.uw;
     int32_t* out = w.ulist + (int64_t)grp * w.us;
-    int base = 0;
-    for (int64_t w0 = 0; w0 < nwords; w0 += blockDim.x) {
+    // set bits before this chunk
+    int pre = 0;
+    for (int64_t wi = threadIdx.x; wi < c0; wi += kCompactThreads) pre += __popc(uwp[wi]);
+    int base = block_sum<int>(pre, red);
+    const int64_t c1 = c0 + kCompactWords < nwords ? c0 + kCompactWords : nwords;
+    for (int64_t w0 = c0; w0 < c1; w0 += kCompactThreads) {
         const int64_t wi = w0 + threadIdx.x;
-        uint32_t word = wi < nwords ? uwp[wi] : 0u;
+        uint32_t word = wi < c1 ? uwp[wi] : 0u;
         int total;
         const int excl = block_excl_scan<int>(__popc(word), red, total);
         int k = base + excl;
@@ -198,6 +212,7 @@ __global__ void __launch_bounds__(1024) k_union_compact(Batch b, Work w, int it,
         }
         base += total;
     }
+    if (c1 < nwords) return;                                   // not the group's last chunk
     if (base > w.us) {                                         // cannot happen with the limit above
         if (threadIdx.x == 0) atomicOr(w.status, kStatusCapacity);
         base = (int)w.us;
@@ -1024,7 +1039,8 @@ cudaError_t launch_union(const Batch& b, const Work& w, int it, int mode, cudaSt
     const int lanes_per_block = 64;
     dim3 grid((unsigned)((w.uw + 255) / 256), (b.n_gl + lanes_per_block - 1) / lanes_per_block, b.n_groups);
     k_union_or<<<grid, 256, 0, st>>>(b, w, it, mode, lanes_per_block);
-    k_union_compact<<<b.n_groups, 1024, 0, st>>>(b, w, it, mode);
+    const unsigned chunks = (unsigned)std::max<int64_t>(1, (w.uw + kCompactWords - 1) / kCompactWords);
+    k_union_compact<<<dim3(chunks, b.n_groups), kCompactThreads, 0, st>>>(b, w, it, mode);
     return cudaGetLastError();
 }
 

@@ -147,13 +147,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 x 32 bit transpose across a warp: lane y holds row y (bit t = element (y, t)); the result
+// in lane t is column t (bit y = element (y, t)).  Five butterfly stages exchange ever smaller
+// blocks with the partner lane (16, 8, 4, 2, 1 apart): about a quarter of the instructions of
+// 32 ballots.
+__device__ __forceinline__ uint32_t transpose32(uint32_t v, int lane) {
+    const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int j = 16 >> k;
+        const uint32_t m = masks[k];
+        const uint32_t t = __shfl_xor_sync(0xffffffffu, v, j);
+        v = (lane & j) ? ((v & ~m) | ((t & ~m) >> j)) : ((v & m) | ((t & m) << j));
+    }
+    return v;
+}
+
 // Lanes' kept bits of one level, transposed over the group's union list of that level:
 // memb[grp][u][w] bit t = lane 32 w + t kept union node u.  Mode 0: the level above the one
 // routing iteration `it` scores (its nodes are the candidates' parents); mode 1: level 1
 // (the chunks attention gathers).  A block transposes a tile of 256 union entries x 256
 // lanes (8 lane words): where the tile's entries are 256 consecutive nodes (a dense stretch
 // of the union), each lane reads the 9 bitmap words covering them and realigns them by
-// funnel shifts, warps transpose 32 x 32 bit blocks with ballots through shared memory, and
+// funnel shifts, warps transpose 32 x 32 bit blocks (butterfly shuffles) through shared memory, and
 // each entry's 8 words are written as one 32-byte segment.  A tile whose entries lie within
 // 1,024 nodes stages each lane's words of that window and transposes entry by entry from
 // shared memory; sparser tiles read each entry's word from global memory.
@@ -196,17 +212,8 @@ __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mod
             for (int k = 0; k < 8; ++k) T[tid][k] = __funnelshift_r(wv[k], wv[k + 1], sh);
             __syncthreads();
             // warp i: node word i of the tile, for each of the 8 lane words
-#pragma unroll 1
-            for (int lw = 0; lw < 8; ++lw) {
-                const uint32_t v = T[lw * 32 + lane][warp];
-                uint32_t mine = 0;
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const uint32_t r = __ballot_sync(0xffffffffu, (v >> t) & 1u);
-                    if (lane == t) mine = r;
-                }
-                O[warp * 32 + lane][lw] = mine;
-            }
+#pragma unroll 2
+            for (int lw = 0; lw < 8; ++lw) O[warp * 32 + lane][lw] = transpose32(T[lw * 32 + lane][warp], lane);
             __syncthreads();
             uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(u0 + tid) * w.mwords);
             dst[0] = make_uint4(O[tid][0], O[tid][1], O[tid][2], O[tid][3]);
@@ -253,19 +260,14 @@ __global__ void __launch_bounds__(256) k_member(Batch b, Work w, int it, int mod
                     if ((lw0 + lw) * 32 >= b.n_gl) break;             // uniform in the warp
                     const bool ok = yl < b.n_gl;
                     const uint32_t* kl = w.kept[pl] + lane_of(b, s, g, ok ? yl : 0) * w.W[pl];
-                    // all 32 entries' bits of this lane first (independent loads), then ballots
+                    // all 32 entries' bits of this lane first (independent loads), then the transpose
                     uint32_t bits = 0;
 #pragma unroll
                     for (int t = 0; t < 32; ++t) {
                         const int pt = __shfl_sync(0xffffffffu, pmy, t);
                         if (t < n && ok) bits |= ((__ldg(kl + (pt >> 5)) >> (pt & 31)) & 1u) << t;
                     }
-                    uint32_t mine = 0;
-#pragma unroll
-                    for (int t = 0; t < 32; ++t) {
-                        const uint32_t r = __ballot_sync(0xffffffffu, (bits >> t) & 1u);
-                        if (lane == t) mine = r;
-                    }
+                    const uint32_t mine = transpose32(bits, lane);
                     if (lane < n) out[(int64_t)(e0 + lane) * w.mwords + lw] = mine;
                 }
             }
