@@ -299,7 +299,7 @@ def test_tensor_core_scoring_needs_r16():
 
 
 @needs_cuda
-@pytest.mark.parametrize("n_q,p", [(1, 0.95), (8, 0.9), (64, 0.95), (64, 1.0)])
+@pytest.mark.parametrize("n_q,p", [(1, 0.95), (8, 0.9), (40, 0.9), (64, 0.95), (64, 1.0)])
 def test_tensor_core_and_cuda_core_attention_agree(n_q, p):
     """The tcgen05 attention (exact QK^T, bf16 hi+lo P) and the CUDA-core attention give the
     same outputs on the same routed sets, and the tensor-core output matches the oracle."""
@@ -403,6 +403,10 @@ R32 = inputs.Geometry(C=4, L=4, R=32, d=128, Hq=16, Hkv=2)
     ("C2 R16 tensor", C2R16, 40 * 128 + 33, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
     ("C16 MID tensor", inputs.MID, 3 * 4096 + 900, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
     ("C16 MID tensor 24q", inputs.MID, 3 * 4096 + 900, 24, (zha.ZHA_KERNELS_TENSOR, zha.ZHA_KERNELS_TENSOR)),
+    # more than 128 lanes per group: the attention pairs lane tiles in one CTA (320 lanes: one
+    # full pair and one CTA holding a single lane tile)
+    ("d64 tensor 40q", D64, 10 * 256 + 77, 40, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
+    ("C6 R16 tensor 40q", C6R16, 14 * 216 + 101, 40, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
     # R = 32: scoring on CUDA cores (k_score), attention both ways
     ("R32 simt", R32, 12 * 256 + 5, 2, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
     ("R32 simt score, tensor attn", R32, 12 * 256 + 5, 8, (zha.ZHA_KERNELS_AUTO, zha.ZHA_KERNELS_AUTO)),
