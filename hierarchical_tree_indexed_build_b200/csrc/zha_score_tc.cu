@@ -502,33 +502,42 @@ __global__ void __launch_bounds__(64 + 128 * LT, 1) k_score_tc(Batch b, Work w, 
                 mbar_wait(smem_u32(&bar_full[i % kStages]), (uint32_t)((i / kStages) & 1));
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (lane 0)
-        if (lane == 0) {
+        // ---------------- MMA issuer: the whole warp waits, one elected lane issues (a
+        // converged warp issues tcgen05.mma at about twice the rate of a lone thread)
+        {
             const int jobs = nt * LT;
-            for (int q = 0; q < jobs && !abort_sh; ++q) {
+            for (int q = 0; q < jobs; ++q) {
+                if (__any_sync(0xffffffffu, abort_sh != 0)) break;
                 const int i = q / LT, t = q % LT, st = i % kStages, slot = q % kAcc;
                 bool okw = true;
                 if (t == 0) okw = mbar_wait(smem_u32(&bar_full[st]), (uint32_t)((i / kStages) & 1));
                 if (okw && q >= kAcc) okw = mbar_wait(smem_u32(&bar_acc_empty[slot]), (uint32_t)(((q / kAcc) - 1) & 1));
-                if (!okw) {
-                    atomicOr(w.status, kStatusTimeout);
-                    abort_sh = 1;
+                if (!__all_sync(0xffffffffu, okw)) {
+                    if (lane == 0) {
+                        atomicOr(w.status, kStatusTimeout);
+                        abort_sh = 1;
+                    }
                     break;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t d = tmem + (uint32_t)(slot * kTileN);
-                const uint32_t ta = tmem + kColA + (uint32_t)(t * (D / 2));
-                const uint64_t db = umma_desc(smem_u32(sB0 + (size_t)st * STAGE));
+                uint32_t leader;
+                asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(leader));
+                if (leader) {
+                    const uint32_t d = tmem + (uint32_t)(slot * kTileN);
+                    const uint32_t ta = tmem + kColA + (uint32_t)(t * (D / 2));
+                    const uint64_t db = umma_desc(smem_u32(sB0 + (size_t)st * STAGE));
 #pragma unroll 1
-                for (int pk = 0; pk < kPlanes * KB; ++pk) {
-                    const int pass = pk / KB, kb = pk % KB;
-                    const uint64_t b1 = db + (uint64_t)((pass * P_BYTES + kb * (kTileN * 128)) >> 4);
-                    const uint32_t a1 = ta + (uint32_t)(kb * 32);
+                    for (int pk = 0; pk < kPlanes * KB; ++pk) {
+                        const int pass = pk / KB, kb = pk % KB;
+                        const uint64_t b1 = db + (uint64_t)((pass * P_BYTES + kb * (kTileN * 128)) >> 4);
+                        const uint32_t a1 = ta + (uint32_t)(kb * 32);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ts(d, a1 + (uint32_t)(kk * 8), b1 + (uint64_t)(kk * 2), kId, (pk | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16_ts(d, a1 + (uint32_t)(kk * 8), b1 + (uint64_t)(kk * 2), kId, (pk | kk) ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&bar_acc_full[slot]));
                 }
-                mma_commit(smem_u32(&bar_acc_full[slot]));
+                __syncwarp();
             }
         }
         __syncwarp();
